@@ -1,0 +1,328 @@
+"""Pins for the fp64 oracle: each check ties it to something other than itself
+(hand-worked values, closed forms, special cases, an independent formulation,
+a library FFT), chosen so that a dropped term, a wrong sign or index, or a
+transposed operand fails at least one.  CPU only."""
+import numpy as np
+import pytest
+
+from oracle import ssm_oracle as O
+from oracle import cref
+from fft_long_convolution_flashconv_b200 import workloads as W
+
+
+def _cplx(pair):
+    return complex(pair[0], pair[1])
+
+
+# ---------------------------------------------------------------- hand-worked fixtures
+def test_golden_real_n1(golden):
+    g = golden("hand_worked_real_n1.txt")
+    A = np.array([[g["a"][0]]], dtype=np.complex128)
+    Bc = np.array([[_cplx(g["B"])]])
+    Cc = np.array([[_cplx(g["C"])]])
+    D = np.array(g["D"])
+    u = np.array(g["u"]).reshape(1, 1, -1)
+    L = u.shape[-1]
+    f = O.ssm_filter_from_A(A, Bc, Cc, L)
+    assert np.array_equal(f[0], np.array(g["f"]))
+    y = O.causal_conv_direct(u, f, D)
+    assert np.allclose(y[0, 0], g["y"], rtol=0, atol=1e-15)
+    y2, x = O.ssm_recurrence(u, A, Bc, Cc, D)
+    assert np.allclose(y2[0, 0], g["y"], rtol=0, atol=1e-15)
+    assert abs(x[0, 0, 0] - _cplx(g["x_last"])) < 1e-15
+    yc = cref.causal_conv(u, f, D)
+    assert np.allclose(yc[0, 0], g["y"], rtol=0, atol=1e-15)
+    yr, xr = cref.ssm_recurrence(u, A, Bc, Cc, D)
+    assert np.allclose(yr[0, 0], g["y"], rtol=0, atol=1e-15)
+    assert abs(xr[0, 0, 0] - _cplx(g["x_last"])) < 1e-15
+
+
+def test_golden_complex_rotation(golden):
+    g = golden("hand_worked_complex_rotation.txt")
+    A = np.array([[_cplx(g["A"])]])
+    f = O.ssm_filter_from_A(A, np.array([[_cplx(g["B"])]]), np.array([[_cplx(g["C"])]]), 8)
+    assert np.allclose(f[0], g["f"], atol=1e-14)
+    # the exp(dt*lambda) form reaches the same A with dt = 1, lambda = i*pi/2
+    lam = np.array([[[0.0, np.pi / 2]]])
+    f2 = O.ssm_filter(np.array([1.0]), lam, np.array([[[1.0, 0.0]]]), np.array([[g["C"]]]), 8)
+    assert np.allclose(f2[0], g["f"], atol=1e-12)
+
+
+def test_golden_shift_ssm(golden):
+    g = golden("hand_worked_shift_ssm.txt")
+    k = np.array(g["k"]).reshape(1, -1, 1)
+    Cs = np.array(g["Cshift"]).reshape(1, -1)
+    out = O.shift_ssm(k, Cs)
+    assert np.array_equal(out[0, :, 0], np.array(g["ktilde"]))
+
+
+def test_golden_h3_mixer(golden):
+    g = golden("hand_worked_h3_mixer.txt")
+    q = np.array(g["q"]).reshape(1, 2, 2)
+    k = np.array(g["k"]).reshape(1, 2, 2)
+    v = np.array(g["v"]).reshape(1, 2, 2)
+    Cs = np.array([[1.0, 0, 0, 0], [1.0, 0, 0, 0]])
+    f = np.array(g["f"]).reshape(1, 2)
+    D = np.array(g["D"])
+    o1 = O.h3_mixer_outer(q, k, v, Cs, f, D, heads=1)
+    o2 = O.h3_mixer_toeplitz(q, k, v, Cs, f, D, heads=1)
+    want = np.array(g["o"]).reshape(1, 2, 2)
+    assert np.allclose(o1, want, atol=1e-14)
+    assert np.allclose(o2, want, atol=1e-14)
+
+
+# ---------------------------------------------------------------- closed forms / invariants
+def _small(seed=11, B=2, H=3, L=64, N=8, dt=("loguniform", -3.0, -1.0)):
+    wl = W.make_conv(B=B, H=H, L=L, N=N, dtype="f32", seed=seed, dt_range=dt)
+    A = O.discretize(wl.dt, wl.lam)
+    return wl, A, O.as_complex(wl.Bp), O.as_complex(wl.Cp)
+
+
+def test_filter_exp_form_vs_repeated_product():
+    wl, A, Bc, Cc = _small(L=300)
+    f1 = O.ssm_filter(wl.dt, wl.lam, wl.Bp, wl.Cp, wl.L)
+    f2 = O.ssm_filter_from_A(A, Bc, Cc, wl.L)
+    assert O.row_rel_err(f1, f2) < 1e-11
+
+
+def test_filter_spectrum_closed_form():
+    """FFT_{2L} of the zero-padded filter equals the finite geometric sum
+    sum_n c_n (1 - A^L z^-L)/(1 - A z^-1) + conj pair, z = exp(2 pi i m / 2L)."""
+    wl, A, Bc, Cc = _small(L=128, N=6)
+    L = wl.L
+    f = O.ssm_filter(wl.dt, wl.lam, wl.Bp, wl.Cp, L)
+    M = 2 * L
+    F = np.fft.fft(np.concatenate([f, np.zeros_like(f)], axis=1), axis=1)
+    zinv = np.exp(-2j * np.pi * np.arange(M) / M)
+    c = Cc * Bc
+    for h in range(wl.H):
+        a = A[h][:, None]
+        term = c[h][:, None] * (1 - a ** L * zinv[None] ** L) / (1 - a * zinv[None])
+        ac = np.conj(A[h])[:, None]
+        term2 = np.conj(c[h])[:, None] * (1 - ac ** L * zinv[None] ** L) / (1 - ac * zinv[None])
+        closed = np.sum(term + term2, axis=0)
+        assert np.max(np.abs(F[h] - closed)) < 1e-9 * np.max(np.abs(closed))
+
+
+def test_special_cases():
+    wl, A, Bc, Cc = _small(L=50)
+    u = wl.u
+    f0 = O.ssm_filter(wl.dt, wl.lam, wl.Bp, np.zeros_like(wl.Cp), wl.L)
+    assert np.all(f0 == 0)
+    y = O.causal_conv_direct(u, f0, wl.D)
+    assert np.array_equal(y, wl.D.astype(np.float64)[None, :, None] * u)  # C = 0 -> y = D u
+    # A = 0 -> f = [2 Re(CB), 0, 0, ...]
+    fz = O.ssm_filter_from_A(np.zeros_like(A), Bc, Cc, 10)
+    assert np.allclose(fz[:, 0], 2 * np.real(np.sum(Cc * Bc, axis=1)), atol=1e-15)
+    assert np.all(fz[:, 1:] == 0)
+    # N = 1, real a: f = 2 a^k
+    a = 0.93
+    fr = O.ssm_filter_from_A(np.array([[a + 0j]]), np.array([[1 + 0j]]), np.array([[1 + 0j]]), 40)
+    assert np.allclose(fr[0], 2 * a ** np.arange(40), rtol=1e-13)
+
+
+def test_impulse_response_equals_filter():
+    wl, A, Bc, Cc = _small(L=200)
+    u = np.zeros((1, wl.H, wl.L))
+    u[0, :, 0] = 1.0
+    f = O.ssm_filter(wl.dt, wl.lam, wl.Bp, wl.Cp, wl.L)
+    y, _ = O.ssm_recurrence(u, A, Bc, Cc, wl.D)
+    want = f.copy()
+    want[:, 0] += wl.D
+    assert O.row_rel_err(y[0], want) < 1e-12
+    yc, _ = cref.ssm_recurrence(u, A, Bc, Cc, wl.D)
+    assert O.row_rel_err(yc[0], want) < 1e-12
+
+
+def test_conv_equals_recurrence():
+    for dt in [("loguniform", -3.0, -1.0), ("split", (-3.0, -2.9), (-1.1, -1.0))]:
+        wl, A, Bc, Cc = _small(L=512, H=4, dt=dt)
+        f = O.ssm_filter(wl.dt, wl.lam, wl.Bp, wl.Cp, wl.L)
+        y1 = O.causal_conv_direct(wl.u, f, wl.D)
+        y2, _ = O.ssm_recurrence(wl.u, A, Bc, Cc, wl.D)
+        assert O.row_rel_err(y1, y2) < 1e-10
+        y3 = cref.causal_conv(wl.u, f, wl.D)
+        assert O.row_rel_err(y3, y1) < 1e-13
+
+
+def test_linearity():
+    wl, A, Bc, Cc = _small(L=128)
+    f = O.ssm_filter(wl.dt, wl.lam, wl.Bp, wl.Cp, wl.L)
+    rng = np.random.default_rng(5)
+    u1 = rng.normal(size=wl.u.shape)
+    u2 = rng.normal(size=wl.u.shape)
+    al, be = 0.7, -1.3
+    lhs = O.causal_conv_direct(al * u1 + be * u2, f, wl.D)
+    rhs = al * O.causal_conv_direct(u1, f, wl.D) + be * O.causal_conv_direct(u2, f, wl.D)
+    assert O.row_rel_err(lhs, rhs) < 1e-12
+
+
+def test_shift_equivariance_bit_exact_zeros():
+    wl, A, Bc, Cc = _small(L=96, B=1)
+    f = O.ssm_filter(wl.dt, wl.lam, wl.Bp, wl.Cp, wl.L)
+    s = 17
+    u = np.zeros((1, wl.H, wl.L))
+    u[0, :, s:] = wl.u[0, :, : wl.L - s]
+    y = O.causal_conv_direct(u, f, wl.D)
+    assert np.all(y[0, :, :s] == 0.0)
+    y0 = O.causal_conv_direct(wl.u, f, wl.D)
+    assert O.row_rel_err(y[0, :, s:], y0[0, :, : wl.L - s]) < 1e-13
+    # delayed impulse: output is f shifted by s
+    d = np.zeros((1, wl.H, wl.L))
+    d[0, :, s] = 1.0
+    yd = O.causal_conv_direct(d, f, np.zeros(wl.H))
+    assert np.all(yd[0, :, :s] == 0.0)
+    assert np.array_equal(yd[0, :, s:], f[:, : wl.L - s])
+
+
+def test_library_fft_crosscheck():
+    wl, A, Bc, Cc = _small(L=256)
+    f = O.ssm_filter(wl.dt, wl.lam, wl.Bp, wl.Cp, wl.L)
+    L = wl.L
+    U = np.fft.rfft(wl.u, n=2 * L, axis=-1)
+    F = np.fft.rfft(f, n=2 * L, axis=-1)
+    yf = np.fft.irfft(U * F[None], n=2 * L, axis=-1)[..., :L] + wl.D[None, :, None] * wl.u
+    y = O.causal_conv_direct(wl.u, f, wl.D)
+    assert O.row_rel_err(yf, y) < 1e-12
+
+
+def test_statepass_equals_unchunked():
+    wl, A, Bc, Cc = _small(L=256, H=3, B=2)
+    y_ref, x_ref = O.ssm_recurrence(wl.u, A, Bc, Cc, wl.D)
+    for T in (16, 64, 256):
+        y, x = O.statepass_chunked(wl.u, A, Bc, Cc, wl.D, T)
+        assert O.row_rel_err(y, y_ref) < 1e-10, T
+        assert np.max(np.abs(x - x_ref)) < 1e-10 * np.max(np.abs(x_ref))
+    # chunk = L reduces to the plain convolution
+    f = O.ssm_filter_from_A(A, Bc, Cc, wl.L)
+    yT, _ = O.statepass_chunked(wl.u, A, Bc, Cc, wl.D, wl.L)
+    assert O.row_rel_err(yT, O.causal_conv_direct(wl.u, f, wl.D)) < 1e-12
+    # state_out of call 1 fed as state_in of call 2 == one call on the concatenation
+    h = wl.L // 2
+    y1, x1 = O.statepass_chunked(wl.u[..., :h], A, Bc, Cc, wl.D, 32)
+    y2, x2 = O.statepass_chunked(wl.u[..., h:], A, Bc, Cc, wl.D, 32, x0=x1)
+    assert O.row_rel_err(np.concatenate([y1, y2], -1), y_ref) < 1e-10
+    assert np.max(np.abs(x2 - x_ref)) < 1e-10 * np.max(np.abs(x_ref))
+    # a nonzero initial state reaches y through A^(t+1): compare with the recurrence
+    x0 = np.random.default_rng(3).normal(size=x_ref.shape) + 1j
+    y3, _ = O.statepass_chunked(wl.u, A, Bc, Cc, wl.D, 64, x0=x0)
+    y4, _ = O.ssm_recurrence(wl.u, A, Bc, Cc, wl.D, x0=x0)
+    assert O.row_rel_err(y3, y4) < 1e-10
+    y5, _ = cref.ssm_recurrence(wl.u, A, Bc, Cc, wl.D, x0=x0)
+    assert O.row_rel_err(y5, y4) < 1e-12
+
+
+def test_shift_ssm_impulse_gives_taps():
+    rng = np.random.default_rng(2)
+    Cs = rng.normal(size=(5, 4))
+    k = np.zeros((1, 10, 5))
+    k[0, 3, :] = 1.0
+    out = O.shift_ssm(k, Cs)
+    assert np.all(out[0, :3] == 0)
+    assert np.array_equal(out[0, 3:7].T, Cs)
+    assert np.all(out[0, 7:] == 0)
+
+
+def _mixer_small(hd=3, heads=2, L=12, B=2, seed=9):
+    mw = W.make_mixer(B=B, L=L, heads=heads, head_dim=hd, N=4, shift_len=4, dtype="f32", seed=seed)
+    f = O.ssm_filter(mw.dt, mw.lam, mw.Bp, mw.Cp, L)
+    return mw, f
+
+
+def test_mixer_forms_agree():
+    mw, f = _mixer_small()
+    o1 = O.h3_mixer_outer(mw.q, mw.k, mw.v, mw.Cshift, f, mw.D, mw.heads)
+    o2 = O.h3_mixer_toeplitz(mw.q, mw.k, mw.v, mw.Cshift, f, mw.D, mw.heads)
+    assert np.max(np.abs(o1 - o2)) < 1e-12 * np.max(np.abs(o1))
+
+
+def test_mixer_hd1_reduces_to_gated_conv():
+    mw, f = _mixer_small(hd=1, heads=3)
+    o = O.h3_mixer_outer(mw.q, mw.k, mw.v, mw.Cshift, f, mw.D, mw.heads)
+    kt = O.shift_ssm(mw.k, mw.Cshift)
+    x = np.transpose(kt * mw.v, (0, 2, 1))                       # B x C x L
+    y = O.causal_conv_direct(x, f, mw.D)
+    want = mw.q * np.transpose(y, (0, 2, 1))
+    assert np.max(np.abs(o - want)) < 1e-13 * np.max(np.abs(want))
+
+
+def test_mixer_delta_filter():
+    """f = delta (A = 0, C B = 1/2) -> o_j = (D + 1) (q . k~) v_j."""
+    mw, _ = _mixer_small()
+    heads, L = mw.heads, mw.L
+    A = np.zeros((heads, 1), dtype=np.complex128)
+    f = O.ssm_filter_from_A(A, np.ones((heads, 1)), 0.5 * np.ones((heads, 1)), L)
+    assert np.all(f[:, 0] == 1.0) and np.all(f[:, 1:] == 0)
+    o = O.h3_mixer_outer(mw.q, mw.k, mw.v, mw.Cshift, f, mw.D, heads)
+    kt = O.shift_ssm(mw.k, mw.Cshift)
+    hd = mw.head_dim
+    for h in range(heads):
+        sl = slice(h * hd, (h + 1) * hd)
+        qk = np.sum(mw.q[:, :, sl] * kt[:, :, sl], axis=-1, keepdims=True)
+        want = (np.float64(mw.D[h]) + 1.0) * qk * mw.v[:, :, sl]
+        assert np.max(np.abs(o[:, :, sl] - want)) < 1e-13 * np.max(np.abs(want))
+
+
+# ---------------------------------------------------------------- planted mistakes
+def test_pins_catch_planted_mistakes(golden):
+    """Mutated copies of oracle steps (made here, on the CPU) must fail a pin."""
+    g = golden("hand_worked_real_n1.txt")
+    u = np.array(g["u"]).reshape(1, 1, -1)
+    f = np.array(g["f"]).reshape(1, -1)
+    # 1. dropped D term
+    y_noD = O.causal_conv_direct(u, f, np.zeros(1))
+    assert not np.allclose(y_noD[0, 0], g["y"])
+    # 2. off-by-one causal index (y[t] uses u up to t-1)
+    y_shift = np.concatenate([[0.0], O.causal_conv_direct(u, f, np.zeros(1))[0, 0, :-1]]) + 0.25 * u[0, 0]
+    assert not np.allclose(y_shift, g["y"])
+    # 3. conj(C) instead of C in the filter
+    gr = golden("hand_worked_complex_rotation.txt")
+    A = np.array([[_cplx(gr["A"])]])
+    fbad = O.ssm_filter_from_A(A, np.array([[1 + 0j]]), np.conj(np.array([[_cplx(gr["C"])]])), 8)
+    assert not np.allclose(fbad[0], gr["f"])
+    # 4. state correction through A^t instead of A^(t+1)
+    wl, A, Bc, Cc = _small(L=64, H=2, B=1)
+    y_ref, _ = O.ssm_recurrence(wl.u, A, Bc, Cc, wl.D)
+    T = 16
+    fT = O.ssm_filter_from_A(A, Bc, Cc, T)
+    x = np.zeros((1, wl.H, A.shape[1]), dtype=np.complex128)
+    yb = np.empty_like(wl.u)
+    for c in range(wl.L // T):
+        uc = wl.u[:, :, c * T:(c + 1) * T]
+        p = A[:, :, None] ** np.arange(T)[None, None, :]            # wrong: A^t
+        yb[:, :, c * T:(c + 1) * T] = O.causal_conv_direct(uc, fT, wl.D) + \
+            2 * np.real(np.einsum("hn,hnt,bhn->bht", Cc, p, x))
+        Mux = (A[:, :, None] ** (T - 1 - np.arange(T))[None, None, :]) * Bc[:, :, None]
+        x = (A ** T)[None] * x + np.einsum("hni,bhi->bhn", Mux, uc)
+    assert O.row_rel_err(yb, y_ref) > 1e-3
+    # 5. shift taps reversed
+    gs = golden("hand_worked_shift_ssm.txt")
+    out = O.shift_ssm(np.array(gs["k"]).reshape(1, -1, 1), np.array(gs["Cshift"])[::-1].reshape(1, -1))
+    assert not np.array_equal(out[0, :, 0], np.array(gs["ktilde"]))
+    # 6. q and k~ swapped in the mixer (q is not shifted; k is)
+    gm = golden("hand_worked_h3_mixer.txt")
+    q = np.array(gm["q"]).reshape(1, 2, 2)
+    k = np.array(gm["k"]).reshape(1, 2, 2)
+    v = np.array(gm["v"]).reshape(1, 2, 2)
+    Cs = np.array([[1.0, 0, 0, 0]] * 2)
+    obad = O.h3_mixer_outer(k, q, v, Cs, np.array([gm["f"]]), np.array(gm["D"]), 1)
+    assert not np.allclose(obad.ravel(), gm["o"])
+
+
+# ---------------------------------------------------------------- input module sanity
+def test_workload_rounding_matches_torch():
+    import torch
+    x = np.random.default_rng(0).normal(size=10000) * 3
+    for dt, td in (("f16", torch.float16), ("bf16", torch.bfloat16), ("f32", torch.float32)):
+        want = torch.tensor(x, dtype=torch.float64).to(torch.float32).to(td).to(torch.float64).numpy()
+        assert np.array_equal(W.round_to(x, dt), want), dt
+
+
+def test_workloads_deterministic():
+    a = W.make("cfg1_conv_f32_B1_H4_L256")
+    b = W.make("cfg1_conv_f32_B1_H4_L256")
+    assert np.array_equal(a.u, b.u) and np.array_equal(a.dt, b.dt)
+    assert a.u.shape == (1, 4, 256) and a.N == 32
+    assert np.all((a.dt >= 1e-3 * 0.999) & (a.dt <= 1e-1 * 1.001))
+    c3 = W.make("cfg3_conv_bf16_B4_H1024_L8192", B=1, L=16)
+    assert np.all(c3.dt[:512] < 1.3e-3) and np.all(c3.dt[512:] > 0.079)
