@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""Benchmark of the SSM long convolution hot path on B200.
+
+One JSON line on stdout (rank 0).  A step is one pass of the hot path over one
+batch: the headline workload is the H3-125M-layer-shaped convolution
+(B=8, H=768, L=1024, N=64, fp16 I/O, filter regenerated on the device every
+step): ssm_kernel_gen followed by the fused FFT convolution.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--others] [--impl ours|reference]
+
+Timing: W untimed warm-up steps; then K steps, each preceded by an L2 flush
+(a 256 MiB write, outside the per-step CUDA events) and bracketed by events
+on the launching stream; a barrier and a synchronize bracket the loop; the
+value is the max over ranks.  Multi-GPU runs shard nothing: every rank runs
+its own full batch (weak scaling, no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from fft_long_convolution_flashconv_b200 import workloads as W  # noqa: E402
+
+HEADLINE = "cfg2_conv_f16_B8_H768_L1024"
+METRIC = "conv elements/s (B·H·L per sec) and achieved HBM GB/s fraction, L=1K–64K"
+FALLBACK_HBM_GBS = 6650.0
+DT_BYTES = {"f32": 4, "f16": 2, "bf16": 2}
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as fh:
+            return float(json.load(fh)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sms, maxs, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sms.append(float(parts[1]))
+                maxs.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sms) if sms else None,
+                "sm_max_mhz": max(maxs) if maxs else None,
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+# ------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from fft_long_convolution_flashconv_b200 import _lib, api
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    lib = _lib.load()
+    wl = W.make(args.workload)
+    stream = torch.cuda.current_stream()
+
+    def T(x, dt="f32"):
+        td = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[dt]
+        return torch.tensor(np.asarray(x), dtype=torch.float64).to(td).to(dev).contiguous()
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    res = {}
+    step_fn, conv_fn, units, alg_bytes, kern_per_step, e2e_fn, e2e_bytes = build_step(wl, T, dev, api, lib)
+    # warm-up
+    for _ in range(args.warmup):
+        step_fn()
+    torch.cuda.synchronize()
+    # clocks: sample over a sustained-load phase plus the timed loop
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    t_end = time.time() + args.load_seconds
+    while time.time() < t_end:
+        for _ in range(20):
+            step_fn()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    wall0 = time.time()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        conv_fn(ev[i][1])         # records ev[i][1] between filter generation and the conv kernel
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    wall = time.time() - wall0
+    clocks = sampler.stop()
+    step_ms = [a.elapsed_time(c) for a, b, c in ev]
+    conv_ms = [b.elapsed_time(c) for a, b, c in ev]
+    tot_ms = sum(step_ms)
+    conv_avg = sum(conv_ms) / len(conv_ms)
+    t = torch.tensor([tot_ms, conv_avg], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    tot_ms, conv_avg = float(t[0]), float(t[1])
+    ms_per_step = tot_ms / args.steps
+    value = units * world / (tot_ms / 1e3 / args.steps)
+
+    # end to end through the C ABI with pinned host buffers
+    e2e_ms = e2e_fn(args.e2e_steps)
+    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_val = units * world / (float(te[0]) / 1e3)
+
+    peak, peak_kind = hbm_peak()
+    achieved = alg_bytes / (conv_avg / 1e3) / 1e9
+    traffic = profiled_traffic(args.workload)
+    res.update(dict(
+        metric=METRIC, value=value, unit="conv elements/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
+        ms_per_step=ms_per_step, higher_is_better=True, scaling="weak", vs_baseline=None,
+        dtype="f32",
+        data="synthetic",
+        config=dict(workload=args.workload, B=wl.B, H=wl.H, L=wl.L, N=wl.N, io_dtype=wl.dtype,
+                    filter="generated on device every step" if "conv" in args.workload else None,
+                    l2="flushed before every step (256 MiB write, outside the per-step events)",
+                    parallelism=f"replicas x{world} (rows independent, no collective)"),
+        roofline=dict(bound="hbm", achieved=achieved, peak=peak, unit="GB/s", frac=achieved / peak,
+                      traffic=traffic, kernel="fftconv_kernel", peak_source=peak_kind,
+                      algorithmic_bytes_per_launch=alg_bytes, avg_launch_ms=conv_avg),
+        e2e=dict(value=e2e_val, unit="conv elements/s", h2d_bytes_per_step=e2e_bytes[0],
+                 d2h_bytes_per_step=e2e_bytes[1]),
+        gpu_launches=kern_per_step * args.steps,
+        clocks=clocks, wall_s=wall,
+    ))
+    if args.others and rank == 0:
+        res["other_workloads"] = other_workloads(T, dev, api, args)
+    return res
+
+
+def build_step(wl, T, dev, api, lib):
+    """Return the step closures for a convolution workload."""
+    import torch
+    if not isinstance(wl, W.ConvWorkload) or wl.chunk:
+        raise SystemExit("headline workload must be a fused-convolution config")
+    u = T(wl.u, wl.dtype)
+    dt, lam, Bp, Cp, D = T(wl.dt), T(wl.lam), T(wl.Bp), T(wl.Cp), T(wl.D)
+    f = torch.empty((wl.H, wl.L), dtype=torch.float32, device=dev)
+    y = torch.empty_like(u)
+    s = DT_BYTES[wl.dtype]
+    units = wl.B * wl.H * wl.L
+    alg = units * 2 * s + wl.H * wl.L * 4   # u read + y write + f read, per conv launch
+
+    def step():
+        api.ssm_kernel_gen(dt, lam, Bp, Cp, wl.L, out=f)
+        api.fftconv_fwd(u, f, D, out=y)
+
+    def conv(ev_mid):
+        api.ssm_kernel_gen(dt, lam, Bp, Cp, wl.L, out=f)
+        ev_mid.record(torch.cuda.current_stream())
+        api.fftconv_fwd(u, f, D, out=y)
+
+    # e2e: pinned host inputs -> device, one ssm_conv_fwd C-ABI call, result -> pinned host
+    hu = torch.empty(u.shape, dtype=u.dtype, pin_memory=True)
+    hu.copy_(u.cpu())
+    hp = [x.cpu().pin_memory() for x in (dt, lam, Bp, Cp, D)]
+    dp = [torch.empty_like(x, device=dev) for x in hp]
+    hy = torch.empty(u.shape, dtype=u.dtype, pin_memory=True)
+    ws = torch.empty(max(int(lib.ssm_conv_workspace(wl.H, wl.L)), 1), dtype=torch.uint8, device=dev)
+    du = torch.empty_like(u)
+    h2d = hu.numel() * hu.element_size() + sum(x.numel() * x.element_size() for x in hp)
+    d2h = hy.numel() * hy.element_size()
+
+    def e2e(n):
+        for _ in range(2):
+            one()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            one()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    def one():
+        du.copy_(hu, non_blocking=True)
+        for a, b in zip(dp, hp):
+            a.copy_(b, non_blocking=True)
+        api.ssm_conv_fwd(du, dp[0], dp[1], dp[2], dp[3], dp[4], workspace=ws, out=y)
+        hy.copy_(y, non_blocking=True)
+
+    return step, conv, units, alg, 2, e2e, (h2d, d2h)
+
+
+def other_workloads(T, dev, api, args):
+    """Secondary numbers: the long fused regime, state passing, the H3 mixer."""
+    import torch
+    out = {}
+    peak, _ = hbm_peak()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def timeit(fn, n):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        tot = 0.0
+        for _ in range(n):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            tot += a.elapsed_time(b)
+        return tot / n
+
+    wl = W.make("cfg3_conv_bf16_B4_H1024_L8192")
+    u = T(wl.u, "bf16")
+    dt, lam, Bp, Cp, D = T(wl.dt), T(wl.lam), T(wl.Bp), T(wl.Cp), T(wl.D)
+    f = torch.empty((wl.H, wl.L), dtype=torch.float32, device=dev)
+    y = torch.empty_like(u)
+    api.ssm_kernel_gen(dt, lam, Bp, Cp, wl.L, out=f)
+    ms = timeit(lambda: api.fftconv_fwd(u, f, D, out=y), args.other_steps)
+    units = wl.B * wl.H * wl.L
+    gb = (units * 4 + wl.H * wl.L * 4) / 1e9
+    out[wl.name] = dict(conv_ms=ms, elems_per_s=units / (ms / 1e3), hbm_frac=gb / (ms / 1e3) / peak)
+    ms_full = timeit(lambda: (api.ssm_kernel_gen(dt, lam, Bp, Cp, wl.L, out=f), api.fftconv_fwd(u, f, D, out=y)),
+                     args.other_steps)
+    out[wl.name]["step_ms_with_filter_gen"] = ms_full
+    cfg3_ns_per_elem = ms * 1e6 / units
+    del u, y, f
+
+    wl = W.make("cfg4_statepass_f16_B1_H2560_L65536_T8192")
+    u = T(wl.u, "f16")
+    dt, lam, Bp, Cp, D = T(wl.dt), T(wl.lam), T(wl.Bp), T(wl.Cp), T(wl.D)
+    y = torch.empty_like(u)
+    ws = torch.empty(api.statepass_workspace_bytes(wl.B, wl.H, wl.L, wl.N, wl.chunk), dtype=torch.uint8,
+                     device=dev)
+    ms = timeit(lambda: api.fftconv_statepass(u, dt, lam, Bp, Cp, D, wl.chunk, workspace=ws, out=y),
+                max(2, args.other_steps // 4))
+    units = wl.B * wl.H * wl.L
+    out[wl.name] = dict(step_ms=ms, elems_per_s=units / (ms / 1e3),
+                        hbm_frac=(units * 4) / 1e9 / (ms / 1e3) / peak,
+                        per_elem_vs_cfg3=(ms * 1e6 / units) / cfg3_ns_per_elem)
+    del u, y, ws
+
+    mw = W.make("cfg5_h3mixer_f16_B8_L2048_d768")
+    q, k, v = T(mw.q, "f16"), T(mw.k, "f16"), T(mw.v, "f16")
+    Cs, dt, lam, Bp, Cp, D = T(mw.Cshift), T(mw.dt), T(mw.lam), T(mw.Bp), T(mw.Cp), T(mw.D)
+    o = torch.empty_like(q)
+    ws = torch.empty(api.h3_mixer_workspace_bytes(mw.B, mw.L, mw.heads, mw.head_dim, mw.N), dtype=torch.uint8,
+                     device=dev)
+    ms = timeit(lambda: api.h3_mixer_fwd(q, k, v, Cs, dt, lam, Bp, Cp, D, mw.heads, workspace=ws, out=o),
+                max(2, args.other_steps // 4))
+    flops = 2.0 * 2.0 * mw.B * mw.heads * (mw.L * (mw.L + 1) / 2) * mw.head_dim
+    out[mw.name] = dict(step_ms=ms, toeplitz_tflops=flops / (ms / 1e3) / 1e12,
+                        hbm_frac=(4 * mw.B * mw.L * mw.heads * mw.head_dim * 2) / 1e9 / (ms / 1e3) / peak)
+    return out
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per conv launch from a committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "fftconv_traffic.json")
+    try:
+        with open(p) as fh:
+            d = json.load(fh)
+    except Exception:
+        return None
+    if d.get("workload") != workload or d.get("source_sha1") != kernel_source_sha1():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+def kernel_source_sha1():
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "fft_long_convolution_flashconv_b200", "csrc")
+    for name in ("fftconv.cu", "fft_stockham.cuh", "common.cuh"):
+        with open(os.path.join(csrc, name), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+# ------------------------------------------------------------------------- oracle arm
+def oracle_sample(wl, rows_per_step):
+    """One bounded sample of the headline workload on the CPU oracle: filter
+    generation for the channels touched + the direct causal convolution of
+    ``rows_per_step`` rows (fp64)."""
+    from oracle import cref
+    from oracle import ssm_oracle as O
+    rows = np.arange(rows_per_step) % (wl.B * wl.H)
+    bs, hs = rows // wl.H, rows % wl.H
+    uh = np.unique(hs)
+    t0 = time.perf_counter()
+    f = O.ssm_filter(wl.dt[uh], wl.lam[uh], wl.Bp[uh], wl.Cp[uh], wl.L)
+    fmap = {h: i for i, h in enumerate(uh)}
+    u = wl.u[bs, hs][None]                                     # 1 x rows x L
+    fr = f[[fmap[h] for h in hs]]
+    cref.causal_conv(u, fr, wl.D[hs].astype(np.float64))
+    return time.perf_counter() - t0, len(rows) * wl.L
+
+
+def cpu_baseline(wl, target_s):
+    from oracle import cref
+    dt, n = oracle_sample(wl, 64)
+    rows = int(min(wl.B * wl.H, max(64, 64 * target_s / max(dt, 1e-6))))
+    dt, n = oracle_sample(wl, rows)
+    return dict(value=n / dt, unit="conv elements/s", cores=cref.num_threads(), kind="oracle",
+                sample=f"{rows} rows of {wl.name} (filter generation for their channels + fp64 direct "
+                       f"causal convolution, plain C with OpenMP), {dt:.1f} s")
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    from oracle import cref
+    wl = W.make(args.workload)
+    rows = max(8, int(args.ref_rows))
+    for _ in range(args.warmup):
+        oracle_sample(wl, 8)
+    tot, units = 0.0, 0
+    for _ in range(args.steps):
+        dt, n = oracle_sample(wl, rows)
+        tot += dt
+        units += n
+    value = units / tot
+    return dict(metric=METRIC, value=value, unit="conv elements/s", n_gpus=world, steps=args.steps,
+                warmup=args.warmup, ms_per_step=tot / args.steps * 1e3, higher_is_better=True, scaling="weak",
+                vs_baseline=None, dtype="f64", data="synthetic", impl="reference",
+                config=dict(workload=args.workload, B=wl.B, H=wl.H, L=wl.L, N=wl.N, io_dtype=wl.dtype,
+                            note=f"each step is a bounded sample of {rows} rows on the CPU oracle"),
+                cpu_baseline=dict(value=value, unit="conv elements/s", cores=cref.num_threads(), kind="oracle",
+                                  sample=f"{rows} rows per step of {wl.name}"),
+                e2e=dict(value=value, unit="conv elements/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=HEADLINE)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--others", action="store_true", help="also time the other workloads (rank 0)")
+    ap.add_argument("--other-steps", type=int, default=20)
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--load-seconds", type=float, default=1.5)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-rows", type=int, default=512)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            raise SystemExit("for --gpus N > 1 launch with torch.distributed.run --nproc-per-node N")
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if not args.no_cpu_baseline:
+                res["cpu_baseline"] = cpu_baseline(W.make(args.workload), args.cpu_seconds)
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

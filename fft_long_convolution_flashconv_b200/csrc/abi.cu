@@ -1,0 +1,226 @@
+// C ABI of libflashconv_b200.so: argument validation and dispatch.  Every
+// check runs on the host before anything is launched; on failure the call
+// returns a negative fc_status, writes nothing, and records a message for
+// fc_last_error().
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "../../include/flashconv.h"
+#include "kernels.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+fc_status fail(fc_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+fc_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return FC_OK;
+  return fail(FC_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool pow2(long long x) { return x > 0 && (x & (x - 1)) == 0; }
+size_t dtype_size(int d) { return d == FC_F32 ? 4 : 2; }
+bool dtype_ok(int d) { return d == FC_F32 || d == FC_F16 || d == FC_BF16; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+#define FC_REQUIRE(cond, st, ...) \
+  do {                            \
+    if (!(cond)) return fail(st, __VA_ARGS__); \
+  } while (0)
+
+fc_status check_params(const float* dt, const float* lambda, const float* Bp, const float* Cp) {
+  FC_REQUIRE(dt && lambda && Bp && Cp, FC_EINVAL, "null SSM parameter pointer");
+  FC_REQUIRE(aligned(dt, 4) && aligned(lambda, 8) && aligned(Bp, 8) && aligned(Cp, 8), FC_EINVAL,
+             "SSM parameter pointers must be 4-byte (dt) / 8-byte (complex) aligned");
+  return FC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+FC_API int fc_version(void) { return 100; }
+
+FC_API const char* fc_status_string(int s) {
+  switch (s) {
+    case FC_OK: return "ok";
+    case FC_EINVAL: return "invalid argument";
+    case FC_EUNSUPPORTED: return "unsupported configuration";
+    case FC_ECUDA: return "CUDA error";
+    case FC_ENOMEM: return "out of memory";
+    default: return "unknown status";
+  }
+}
+
+FC_API const char* fc_last_error(void) { return g_err; }
+
+FC_API fc_status ssm_kernel_gen(const float* dt, const float* lambda, const float* Bp, const float* Cp, int H, int N,
+                                int L, float* f_out, void* stream) {
+  g_err[0] = 0;
+  FC_REQUIRE(H >= 1 && N >= 1 && L >= 1, FC_EINVAL, "H, N, L must be >= 1 (got %d, %d, %d)", H, N, L);
+  FC_REQUIRE(N <= 1024, FC_EUNSUPPORTED, "N = %d > 1024", N);
+  FC_REQUIRE(L <= (1 << 20), FC_EUNSUPPORTED, "L = %d > 1048576", L);
+  fc_status s = check_params(dt, lambda, Bp, Cp);
+  if (s != FC_OK) return s;
+  FC_REQUIRE(f_out && aligned(f_out, 16), FC_EINVAL, "f_out must be non-null and 16-byte aligned");
+  FC_REQUIRE(H <= 65535, FC_EUNSUPPORTED, "H = %d > 65535", H);
+  return cuda_status(fc::launch_ssm_gen(dt, lambda, Bp, Cp, H, N, L, f_out, (cudaStream_t)stream),
+                     "ssm_kernel_gen launch");
+}
+
+static fc_status check_conv_io(const void* u, const void* y, int B, int H, long long L, int dtype) {
+  FC_REQUIRE(dtype_ok(dtype), FC_EINVAL, "unknown dtype %d", dtype);
+  FC_REQUIRE(B >= 1 && H >= 1, FC_EINVAL, "B, H must be >= 1 (got %d, %d)", B, H);
+  FC_REQUIRE(u && y, FC_EINVAL, "null u or y");
+  FC_REQUIRE(aligned(u, 16) && aligned(y, 16), FC_EINVAL, "u and y must be 16-byte aligned");
+  const size_t bytes = (size_t)B * H * (size_t)L * dtype_size(dtype);
+  const char* pu = (const char*)u;
+  const char* py = (const char*)y;
+  FC_REQUIRE(pu + bytes <= py || py + bytes <= pu, FC_EINVAL, "u and y overlap");
+  return FC_OK;
+}
+
+FC_API fc_status fftconv_fwd(const void* u, const float* f, const float* D, void* y, int B, int H, int L,
+                             fc_dtype dtype, void* stream) {
+  g_err[0] = 0;
+  fc_status s = check_conv_io(u, y, B, H, L, dtype);
+  if (s != FC_OK) return s;
+  FC_REQUIRE(f && D, FC_EINVAL, "null f or D");
+  FC_REQUIRE(aligned(f, 16) && aligned(D, 4), FC_EINVAL, "f must be 16-byte aligned, D 4-byte aligned");
+  FC_REQUIRE(pow2(L) && L >= 16 && L <= 8192, FC_EUNSUPPORTED,
+             "fftconv_fwd: L must be a power of two in [16, 8192] (got %d)", L);
+  FC_REQUIRE((long long)B * 1 <= (1LL << 30), FC_EUNSUPPORTED, "B too large");
+  return cuda_status(fc::launch_fftconv(u, f, L, D, y, B, H, L, L, 1, dtype, (cudaStream_t)stream),
+                     "fftconv_fwd launch");
+}
+
+FC_API size_t ssm_conv_workspace(int H, int L) {
+  if (H < 1 || L < 1) return 0;
+  return round_up((size_t)H * L * sizeof(float), 256);
+}
+
+FC_API fc_status ssm_conv_fwd(const void* u, const float* dt, const float* lambda, const float* Bp, const float* Cp,
+                              const float* D, void* y, int B, int H, int L, int N, void* workspace,
+                              size_t ws_bytes, fc_dtype dtype, void* stream) {
+  g_err[0] = 0;
+  fc_status s = check_conv_io(u, y, B, H, L, dtype);
+  if (s != FC_OK) return s;
+  s = check_params(dt, lambda, Bp, Cp);
+  if (s != FC_OK) return s;
+  FC_REQUIRE(D && aligned(D, 4), FC_EINVAL, "null or misaligned D");
+  FC_REQUIRE(N >= 1 && N <= 1024, FC_EUNSUPPORTED, "N must be in [1, 1024] (got %d)", N);
+  FC_REQUIRE(pow2(L) && L >= 16 && L <= 8192, FC_EUNSUPPORTED,
+             "ssm_conv_fwd: L must be a power of two in [16, 8192] (got %d)", L);
+  FC_REQUIRE(H <= 65535, FC_EUNSUPPORTED, "H = %d > 65535", H);
+  FC_REQUIRE(workspace && aligned(workspace, 256), FC_EINVAL, "workspace must be non-null and 256-byte aligned");
+  FC_REQUIRE(ws_bytes >= ssm_conv_workspace(H, L), FC_EINVAL, "workspace too small: %zu < %zu bytes", ws_bytes,
+             ssm_conv_workspace(H, L));
+  float* f = (float*)workspace;
+  cudaStream_t st = (cudaStream_t)stream;
+  s = cuda_status(fc::launch_ssm_gen(dt, lambda, Bp, Cp, H, N, L, f, st), "ssm_conv_fwd: filter launch");
+  if (s != FC_OK) return s;
+  return cuda_status(fc::launch_fftconv(u, f, L, D, y, B, H, L, L, 1, dtype, st), "ssm_conv_fwd: conv launch");
+}
+
+// workspace layout: [f_T: H*T floats][s: B*H*C*N complex][x: B*H*C*N complex], each 256-aligned
+FC_API size_t fftconv_statepass_workspace(int B, int H, int L, int N, int chunk) {
+  if (B < 1 || H < 1 || L < 1 || N < 1 || chunk < 1 || L % chunk) return 0;
+  const size_t C = (size_t)(L / chunk);
+  const size_t fb = round_up((size_t)H * chunk * sizeof(float), 256);
+  const size_t sb = round_up((size_t)B * H * C * N * 2 * sizeof(float), 256);
+  return fb + 2 * sb;
+}
+
+FC_API fc_status fftconv_statepass(const void* u, const float* dt, const float* lambda, const float* Bp,
+                                   const float* Cp, const float* D, void* y, int B, int H, int L, int N, int chunk,
+                                   const float* state_in, float* state_out, void* workspace, size_t ws_bytes,
+                                   fc_dtype dtype, void* stream) {
+  g_err[0] = 0;
+  FC_REQUIRE(L >= 1, FC_EINVAL, "L must be >= 1");
+  fc_status s = check_conv_io(u, y, B, H, L, dtype);
+  if (s != FC_OK) return s;
+  s = check_params(dt, lambda, Bp, Cp);
+  if (s != FC_OK) return s;
+  FC_REQUIRE(D && aligned(D, 4), FC_EINVAL, "null or misaligned D");
+  FC_REQUIRE(N >= 1 && N <= 256, FC_EUNSUPPORTED, "N must be in [1, 256] (got %d)", N);
+  FC_REQUIRE(pow2(chunk) && chunk >= 16 && chunk <= 8192, FC_EUNSUPPORTED,
+             "chunk must be a power of two in [16, 8192] (got %d)", chunk);
+  FC_REQUIRE(L % chunk == 0, FC_EINVAL, "L = %d is not a multiple of chunk = %d", L, chunk);
+  FC_REQUIRE(H <= 65535 && B <= 65535 && L / chunk <= 2147483647, FC_EUNSUPPORTED, "B or H > 65535");
+  FC_REQUIRE(!state_in || aligned(state_in, 8), FC_EINVAL, "state_in must be 8-byte aligned");
+  FC_REQUIRE(!state_out || aligned(state_out, 8), FC_EINVAL, "state_out must be 8-byte aligned");
+  FC_REQUIRE(workspace && aligned(workspace, 256), FC_EINVAL, "workspace must be non-null and 256-byte aligned");
+  const size_t need = fftconv_statepass_workspace(B, H, L, N, chunk);
+  FC_REQUIRE(ws_bytes >= need, FC_EINVAL, "workspace too small: %zu < %zu bytes", ws_bytes, need);
+  const int C = L / chunk;
+  const size_t fb = round_up((size_t)H * chunk * sizeof(float), 256);
+  const size_t sb = round_up((size_t)B * H * C * N * 2 * sizeof(float), 256);
+  float* fT = (float*)workspace;
+  float* s_ws = (float*)((char*)workspace + fb);
+  float* x_ws = (float*)((char*)workspace + fb + sb);
+  cudaStream_t st = (cudaStream_t)stream;
+  s = cuda_status(fc::launch_ssm_gen(dt, lambda, Bp, Cp, H, N, chunk, fT, st), "statepass: filter launch");
+  if (s != FC_OK) return s;
+  s = cuda_status(fc::launch_fftconv(u, fT, chunk, D, y, B, H, L, chunk, C, dtype, st),
+                  "statepass: chunk conv launch");
+  if (s != FC_OK) return s;
+  return cuda_status(fc::launch_statepass_tail(u, dt, lambda, Bp, Cp, y, B, H, L, N, chunk, state_in, state_out,
+                                               s_ws, x_ws, dtype, st),
+                     "statepass: state launch");
+}
+
+FC_API size_t h3_mixer_workspace(int B, int L, int heads, int head_dim, int N) {
+  (void)B;
+  (void)head_dim;
+  (void)N;
+  if (heads < 1 || L < 1) return 0;
+  return round_up((size_t)heads * L * sizeof(float), 256);
+}
+
+FC_API fc_status h3_mixer_fwd(const void* q, const void* k, const void* v, const float* Cshift, const float* dt,
+                              const float* lambda, const float* Bp, const float* Cp, const float* D, void* o, int B,
+                              int L, int heads, int head_dim, int N, int shift_len, void* workspace,
+                              size_t ws_bytes, fc_dtype dtype, void* stream) {
+  g_err[0] = 0;
+  FC_REQUIRE(dtype_ok(dtype), FC_EINVAL, "unknown dtype %d", dtype);
+  FC_REQUIRE(q && k && v && o, FC_EINVAL, "null q, k, v or o");
+  FC_REQUIRE(aligned(q, 16) && aligned(k, 16) && aligned(v, 16) && aligned(o, 16), FC_EINVAL,
+             "q, k, v, o must be 16-byte aligned");
+  FC_REQUIRE(Cshift && D && aligned(Cshift, 4) && aligned(D, 4), FC_EINVAL, "null or misaligned Cshift / D");
+  fc_status s = check_params(dt, lambda, Bp, Cp);
+  if (s != FC_OK) return s;
+  FC_REQUIRE(B >= 1 && L >= 1 && heads >= 1, FC_EINVAL, "B, L, heads must be >= 1");
+  FC_REQUIRE(head_dim == 64, FC_EUNSUPPORTED, "head_dim must be 64 (got %d)", head_dim);
+  FC_REQUIRE(shift_len >= 1 && shift_len <= 8, FC_EUNSUPPORTED, "shift_len must be in [1, 8] (got %d)",
+             shift_len);
+  FC_REQUIRE(L <= 65536, FC_EUNSUPPORTED, "L = %d > 65536", L);
+  FC_REQUIRE(N >= 1 && N <= 1024, FC_EUNSUPPORTED, "N must be in [1, 1024]");
+  FC_REQUIRE(heads <= 65535 && B <= 65535, FC_EUNSUPPORTED, "B or heads > 65535");
+  const size_t bytes = (size_t)B * L * heads * head_dim * dtype_size(dtype);
+  const char* po = (const char*)o;
+  for (const void* in : {q, k, v}) {
+    const char* pi = (const char*)in;
+    FC_REQUIRE(po + bytes <= pi || pi + bytes <= po, FC_EINVAL, "o overlaps an input");
+  }
+  FC_REQUIRE(workspace && aligned(workspace, 256), FC_EINVAL, "workspace must be non-null and 256-byte aligned");
+  const size_t need = h3_mixer_workspace(B, L, heads, head_dim, N);
+  FC_REQUIRE(ws_bytes >= need, FC_EINVAL, "workspace too small: %zu < %zu bytes", ws_bytes, need);
+  float* f = (float*)workspace;
+  cudaStream_t st = (cudaStream_t)stream;
+  s = cuda_status(fc::launch_ssm_gen(dt, lambda, Bp, Cp, heads, N, L, f, st), "h3_mixer: filter launch");
+  if (s != FC_OK) return s;
+  return cuda_status(fc::launch_h3_mixer(q, k, v, Cshift, f, D, o, B, L, heads, shift_len, dtype, st),
+                     "h3_mixer launch");
+}
+
+}  // extern "C"

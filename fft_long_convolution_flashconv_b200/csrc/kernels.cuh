@@ -1,0 +1,27 @@
+// Internal launchers (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "common.cuh"
+
+namespace fc {
+
+cudaError_t launch_ssm_gen(const float* dt, const float* lam, const float* Bp, const float* Cp, int H, int N, int L,
+                           float* f, cudaStream_t st);
+
+// dtype: 0 f32, 1 f16, 2 bf16.  Lc = transform half-length (chunk), C chunks per row.
+cudaError_t launch_fftconv(const void* u, const float* f, int fstride, const float* D, void* y, int B, int H,
+                           long long Lrow, int Lc, int C, int dtype, cudaStream_t st);
+
+cudaError_t launch_statepass_tail(const void* u, const float* dt, const float* lam, const float* Bp,
+                                  const float* Cp, void* y, int B, int H, int L, int N, int T,
+                                  const float* state_in, float* state_out, float* s_ws, float* x_ws, int dtype,
+                                  cudaStream_t st);
+
+cudaError_t launch_h3_mixer(const void* q, const void* k, const void* v, const float* Cshift, const float* fdiag,
+                            const float* D, void* o, int B, int L, int heads, int shift_len, int dtype,
+                            cudaStream_t st);
+
+}  // namespace fc

@@ -1,0 +1,145 @@
+/* flashconv.h -- C ABI of libflashconv_b200.so: the diagonal-SSM long
+ * convolution of H3 / FlashConv on B200 (sm_100a).
+ *
+ * Source of every operation: "Hungry Hungry Hippos: Towards Language Modeling
+ * with State Space Models" (arXiv 2212.14052v3) as summarised section by
+ * section ("H3 summary") and retold in plain language ("H3 blog").  The
+ * pages give no API; arguments follow their problem statement (SSM matrices
+ * A, B, C, D, input u, output y).
+ *
+ * Conventions shared by all entry points
+ * --------------------------------------
+ *  - Every array pointer is caller-owned DEVICE memory on the current CUDA
+ *    device, unless a comment says otherwise.  The library never allocates
+ *    device memory; scratch space is passed in as `workspace`.
+ *  - Sequences are row-major B x H x L (t contiguous); the H3 mixer's q, k, v,
+ *    o are B x L x (heads*head_dim) (channel contiguous).
+ *  - Complex arrays are interleaved (re, im) float32 pairs.
+ *  - SSM parameters and filters are float32 whatever the I/O dtype.
+ *  - I/O dtype: FC_F32, FC_F16 or FC_BF16 (u, y, q, k, v, o).  Arithmetic is
+ *    float32 throughout (fp32 accumulate); the one rounding to a 16-bit I/O
+ *    dtype is round-to-nearest-even at the store.
+ *  - u/y/q/k/v/o and filter pointers must be 16-byte aligned; parameter
+ *    arrays 4-byte aligned (8-byte for complex).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls are asynchronous on that stream, stateless, and safe to
+ *    issue from several host threads.
+ *  - Return value: FC_OK, or a negative fc_status.  Argument errors are found
+ *    on the host before anything is launched (nothing is written).  Launch
+ *    errors come back as FC_ECUDA; faults during execution surface at the
+ *    caller's next synchronisation.  fc_last_error() gives a message for the
+ *    last failure on the calling host thread.
+ */
+#ifndef FLASHCONV_B200_H
+#define FLASHCONV_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define FC_API __attribute__((visibility("default")))
+#else
+#define FC_API
+#endif
+
+typedef enum {
+  FC_OK = 0,
+  FC_EINVAL = -1,        /* bad argument: null pointer, size, alignment, workspace too small */
+  FC_EUNSUPPORTED = -2,  /* valid but outside what is built (e.g. L not a power of two) */
+  FC_ECUDA = -3,         /* a CUDA runtime call or kernel launch failed */
+  FC_ENOMEM = -4         /* reserved */
+} fc_status;
+
+typedef enum { FC_F32 = 0, FC_F16 = 1, FC_BF16 = 2 } fc_dtype;
+
+/* Library version (major*10000 + minor*100 + patch). */
+FC_API int fc_version(void);
+
+/* Static text for a status code. */
+FC_API const char* fc_status_string(int status);
+
+/* Message describing the last failing call on this host thread ("" if none). */
+FC_API const char* fc_last_error(void);
+
+/* ssm_kernel_gen -- diagonal-SSM convolution filter (A1).
+ * H3 blog "The Convolution Connection": unrolling the recurrence gives the
+ * filter f = [CB, CAB, CA^2B, ...]; H3 summary section 2 "Convolutional view".
+ *   A[h,n]  = exp(dt[h] * lambda[h,n])
+ *   f[h,k]  = 2 Re sum_{n<N} C[h,n] A[h,n]^k B[h,n],   0 <= k < L
+ * (2 Re: conjugate-pair convention of the S4D-based diagonal SSM.)
+ * Arguments: dt (H floats); lambda, Bp, Cp (H x N complex); f_out (H x L
+ * floats, written).  Limits: H >= 1, 1 <= N <= 1024, 1 <= L <= 1048576.
+ * A^k is evaluated with its phase k*dt*Im(lambda) reduced modulo 2 pi in
+ * double precision, so long, slowly decaying filters keep their phase. */
+FC_API fc_status ssm_kernel_gen(const float* dt, const float* lambda, const float* Bp, const float* Cp,
+                                int H, int N, int L, float* f_out, void* stream);
+
+/* fftconv_fwd -- fused FFT causal convolution (A2-A4).
+ * H3 summary section 4 "Short-sequence computation": the FFT, the pointwise
+ * multiply and the inverse FFT run fused in one kernel; section 2
+ * "Convolutional view": zero initial state gives a linear convolution plus a
+ * residual term.
+ *   y[b,h,t] = sum_{s<=t} f[h,t-s] u[b,h,s] + D[h] u[b,h,t]
+ * evaluated as IFFT_{2L}(FFT_{2L}(pad u) * FFT_{2L}(pad f)) cropped to t < L.
+ * u, y: B x H x L in `dtype`; f: H x L floats (any real filter, not only an
+ * SSM's); D: H floats.  Limits: L a power of two, 16 <= L <= 8192; B, H >= 1.
+ * u and y may not overlap. */
+FC_API fc_status fftconv_fwd(const void* u, const float* f, const float* D, void* y,
+                             int B, int H, int L, fc_dtype dtype, void* stream);
+
+/* ssm_conv_fwd -- ssm_kernel_gen followed by fftconv_fwd in one call (the
+ * filter is regenerated on the device every call).  workspace must hold
+ * ssm_conv_workspace(H, L) bytes (the H x L filter). */
+FC_API size_t ssm_conv_workspace(int H, int L);
+FC_API fc_status ssm_conv_fwd(const void* u, const float* dt, const float* lambda, const float* Bp,
+                              const float* Cp, const float* D, void* y, int B, int H, int L, int N,
+                              void* workspace, size_t ws_bytes, fc_dtype dtype, void* stream);
+
+/* fftconv_statepass -- FlashConv state passing for long sequences (A6-A9).
+ * H3 summary section 4 "Long-sequence computation" / "Correctness" and
+ * appendix C "State Passing"; H3 blog "The Solution, Part 2".  The sequence
+ * is split into chunks of T = `chunk`; each chunk is an FFT convolution with
+ * the length-T filter plus D u plus the initial-state term, and the state is
+ * carried between chunks:
+ *   y[cT+t] = (f_T * u_c)[t] + D u_c[t] + 2 Re sum_n C_n A_n^(t+1) x_{c-1,n}
+ *   x_c     = A^T x_{c-1} + sum_{i<T} A^(T-1-i) B u_c[i],   x_{-1} = state_in
+ * The result equals the unchunked SSM output.
+ * u, y: B x H x L in `dtype`; dt: H; lambda, Bp, Cp: H x N complex; D: H.
+ * state_in: B x H x N complex or NULL (zero state); state_out: B x H x N
+ * complex or NULL (written with x after the last chunk).  A caller can
+ * split one sequence over several calls by passing state_out as the next
+ * call's state_in.  workspace: at least fftconv_statepass_workspace(...)
+ * bytes, 256-byte aligned.  Limits: chunk a power of two, 16 <= chunk <=
+ * 8192, L % chunk == 0, 1 <= N <= 256. */
+FC_API size_t fftconv_statepass_workspace(int B, int H, int L, int N, int chunk);
+FC_API fc_status fftconv_statepass(const void* u, const float* dt, const float* lambda, const float* Bp,
+                                   const float* Cp, const float* D, void* y, int B, int H, int L, int N,
+                                   int chunk, const float* state_in, float* state_out, void* workspace,
+                                   size_t ws_bytes, fc_dtype dtype, void* stream);
+
+/* h3_mixer_fwd -- H3 layer core, projections excluded (A10-A11).
+ * H3 blog "The Solution, Part 1": O = Q (.) SSM_diag(SSM_shift(K) (.) V);
+ * H3 summary section 3 "H3 design" and appendix D.2 "H3 Complexity" (heads).
+ * Per head h (channels h*hd .. h*hd+hd-1):
+ *   k~[t,c]  = sum_{j<shift_len, j<=t} Cshift[c,j] k[t-j,c]   (tap 0 = current token)
+ *   y_ij[t]  = sum_{s<=t} f_h[t-s] k~_i[s] v_j[s] + D_h k~_i[t] v_j[t]
+ *   o_j[t]   = sum_i q_i[t] y_ij[t]
+ * with f_h the diagonal-SSM filter of head h (as ssm_kernel_gen).
+ * q, k, v, o: B x L x (heads*head_dim) in `dtype`; Cshift:
+ * (heads*head_dim) x shift_len floats; dt, D: heads floats; lambda, Bp, Cp:
+ * heads x N complex.  workspace: at least h3_mixer_workspace(...) bytes.
+ * Limits: head_dim == 64, 1 <= shift_len <= 8, 1 <= L <= 65536, 1 <= N <= 1024. */
+FC_API size_t h3_mixer_workspace(int B, int L, int heads, int head_dim, int N);
+FC_API fc_status h3_mixer_fwd(const void* q, const void* k, const void* v, const float* Cshift,
+                              const float* dt, const float* lambda, const float* Bp, const float* Cp,
+                              const float* D, void* o, int B, int L, int heads, int head_dim, int N,
+                              int shift_len, void* workspace, size_t ws_bytes, fc_dtype dtype,
+                              void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FLASHCONV_B200_H */
