@@ -4,7 +4,8 @@
 One JSON line on stdout (rank 0).  A step is one pass of the hot path over one
 batch: the headline workload is the H3-125M-layer-shaped convolution
 (B=8, H=768, L=1024, N=64, fp16 I/O, filter regenerated on the device every
-step): ssm_kernel_gen followed by the fused FFT convolution.
+step): one ssm_conv_fwd call, i.e. one kernel that generates the SSM filter
+and runs the fused FFT convolution.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                   [--others] [--impl ours|reference]
@@ -131,7 +132,7 @@ def run_ours(args, rank, world, local_rank):
     for i in range(args.steps):
         flush.zero_()
         ev[i][0].record(stream)
-        conv_fn(ev[i][1])         # records ev[i][1] between filter generation and the conv kernel
+        conv_fn(ev[i][1])         # records ev[i][1] right before the dominant launch
         ev[i][2].record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -169,7 +170,7 @@ def run_ours(args, rank, world, local_rank):
                     l2="flushed before every step (256 MiB write, outside the per-step events)",
                     parallelism=f"replicas x{world} (rows independent, no collective)"),
         roofline=dict(bound="hbm", achieved=achieved, peak=peak, unit="GB/s", frac=achieved / peak,
-                      traffic=traffic, kernel="fftconv_kernel", peak_source=peak_kind,
+                      traffic=traffic, kernel="fftconv_kernel (filter generated in-kernel)", peak_source=peak_kind,
                       algorithmic_bytes_per_launch=alg_bytes, avg_launch_ms=conv_avg),
         e2e=dict(value=e2e_val, unit="conv elements/s", h2d_bytes_per_step=e2e_bytes[0],
                  d2h_bytes_per_step=e2e_bytes[1]),
@@ -182,26 +183,29 @@ def run_ours(args, rank, world, local_rank):
 
 
 def build_step(wl, T, dev, api, lib):
-    """Return the step closures for a convolution workload."""
+    """Return the step closures for a convolution workload.  A step is one
+    ssm_conv_fwd call: the filter is regenerated on the device and the fused
+    FFT convolution runs (for L >= 1024 both happen in one kernel launch)."""
     import torch
     if not isinstance(wl, W.ConvWorkload) or wl.chunk:
         raise SystemExit("headline workload must be a fused-convolution config")
     u = T(wl.u, wl.dtype)
     dt, lam, Bp, Cp, D = T(wl.dt), T(wl.lam), T(wl.Bp), T(wl.Cp), T(wl.D)
-    f = torch.empty((wl.H, wl.L), dtype=torch.float32, device=dev)
     y = torch.empty_like(u)
+    ws = torch.empty(max(int(lib.ssm_conv_workspace(wl.H, wl.L)), 1), dtype=torch.uint8, device=dev)
     s = DT_BYTES[wl.dtype]
     units = wl.B * wl.H * wl.L
-    alg = units * 2 * s + wl.H * wl.L * 4   # u read + y write + f read, per conv launch
+    fused = wl.L >= 1024
+    # algorithmic bytes of the dominant launch: u read + y write (+ the filter
+    # read when it is generated by a separate kernel)
+    alg = units * 2 * s + (0 if fused else wl.H * wl.L * 4)
 
     def step():
-        api.ssm_kernel_gen(dt, lam, Bp, Cp, wl.L, out=f)
-        api.fftconv_fwd(u, f, D, out=y)
+        api.ssm_conv_fwd(u, dt, lam, Bp, Cp, D, workspace=ws, out=y)
 
     def conv(ev_mid):
-        api.ssm_kernel_gen(dt, lam, Bp, Cp, wl.L, out=f)
         ev_mid.record(torch.cuda.current_stream())
-        api.fftconv_fwd(u, f, D, out=y)
+        api.ssm_conv_fwd(u, dt, lam, Bp, Cp, D, workspace=ws, out=y)
 
     # e2e: pinned host inputs -> device, one ssm_conv_fwd C-ABI call, result -> pinned host
     hu = torch.empty(u.shape, dtype=u.dtype, pin_memory=True)
@@ -209,10 +213,16 @@ def build_step(wl, T, dev, api, lib):
     hp = [x.cpu().pin_memory() for x in (dt, lam, Bp, Cp, D)]
     dp = [torch.empty_like(x, device=dev) for x in hp]
     hy = torch.empty(u.shape, dtype=u.dtype, pin_memory=True)
-    ws = torch.empty(max(int(lib.ssm_conv_workspace(wl.H, wl.L)), 1), dtype=torch.uint8, device=dev)
     du = torch.empty_like(u)
     h2d = hu.numel() * hu.element_size() + sum(x.numel() * x.element_size() for x in hp)
     d2h = hy.numel() * hy.element_size()
+
+    def one():
+        du.copy_(hu, non_blocking=True)
+        for a, b in zip(dp, hp):
+            a.copy_(b, non_blocking=True)
+        api.ssm_conv_fwd(du, dp[0], dp[1], dp[2], dp[3], dp[4], workspace=ws, out=y)
+        hy.copy_(y, non_blocking=True)
 
     def e2e(n):
         for _ in range(2):
@@ -226,14 +236,7 @@ def build_step(wl, T, dev, api, lib):
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / n
 
-    def one():
-        du.copy_(hu, non_blocking=True)
-        for a, b in zip(dp, hp):
-            a.copy_(b, non_blocking=True)
-        api.ssm_conv_fwd(du, dp[0], dp[1], dp[2], dp[3], dp[4], workspace=ws, out=y)
-        hy.copy_(y, non_blocking=True)
-
-    return step, conv, units, alg, 2, e2e, (h2d, d2h)
+    return step, conv, units, alg, (1 if fused else 2), e2e, (h2d, d2h)
 
 
 def other_workloads(T, dev, api, args):
@@ -257,6 +260,16 @@ def other_workloads(T, dev, api, args):
             torch.cuda.synchronize()
             tot += a.elapsed_time(b)
         return tot / n
+
+    wl = W.make("cfg2_conv_f16_B8_H768_L1024")
+    u = T(wl.u, "f16")
+    dt, lam, Bp, Cp, D = T(wl.dt), T(wl.lam), T(wl.Bp), T(wl.Cp), T(wl.D)
+    f = torch.empty((wl.H, wl.L), dtype=torch.float32, device=dev)
+    y = torch.empty_like(u)
+    ms_gen = timeit(lambda: api.ssm_kernel_gen(dt, lam, Bp, Cp, wl.L, out=f), args.other_steps)
+    ms_conv = timeit(lambda: api.fftconv_fwd(u, f, D, out=y), args.other_steps)
+    out[wl.name + " (separate kernels)"] = dict(gen_ms=ms_gen, conv_ms=ms_conv)
+    del u, y, f
 
     wl = W.make("cfg3_conv_bf16_B4_H1024_L8192")
     u = T(wl.u, "bf16")
@@ -319,7 +332,7 @@ def profiled_traffic(workload):
 def kernel_source_sha1():
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "fft_long_convolution_flashconv_b200", "csrc")
-    for name in ("fftconv.cu", "fft_stockham.cuh", "common.cuh"):
+    for name in ("fftconv.cu", "fft_stockham.cuh", "common.cuh", "ssm_tables.cuh"):
         with open(os.path.join(csrc, name), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()

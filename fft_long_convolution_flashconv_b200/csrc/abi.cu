@@ -7,6 +7,7 @@
 #include <string.h>
 
 #include "../../include/flashconv.h"
+#include "../../include/flashconv_testing.h"
 #include "kernels.cuh"
 
 namespace {
@@ -100,7 +101,8 @@ FC_API fc_status fftconv_fwd(const void* u, const float* f, const float* D, void
   FC_REQUIRE(pow2(L) && L >= 16 && L <= 8192, FC_EUNSUPPORTED,
              "fftconv_fwd: L must be a power of two in [16, 8192] (got %d)", L);
   FC_REQUIRE((long long)B * 1 <= (1LL << 30), FC_EUNSUPPORTED, "B too large");
-  return cuda_status(fc::launch_fftconv(u, f, L, D, y, B, H, L, L, 1, dtype, (cudaStream_t)stream),
+  const fc::SsmArgs none{nullptr, nullptr, nullptr, nullptr, 0};
+  return cuda_status(fc::launch_fftconv(u, f, L, none, D, y, B, H, L, L, 1, dtype, (cudaStream_t)stream),
                      "fftconv_fwd launch");
 }
 
@@ -127,9 +129,16 @@ FC_API fc_status ssm_conv_fwd(const void* u, const float* dt, const float* lambd
              ssm_conv_workspace(H, L));
   float* f = (float*)workspace;
   cudaStream_t st = (cudaStream_t)stream;
+  const fc::SsmArgs none{nullptr, nullptr, nullptr, nullptr, 0};
+  if (L >= 1024) {  // filter generated inside the convolution kernel
+    const fc::SsmArgs sp{dt, (const float2*)lambda, (const float2*)Bp, (const float2*)Cp, N};
+    return cuda_status(fc::launch_fftconv(u, nullptr, L, sp, D, y, B, H, L, L, 1, dtype, st),
+                       "ssm_conv_fwd: fused launch");
+  }
   s = cuda_status(fc::launch_ssm_gen(dt, lambda, Bp, Cp, H, N, L, f, st), "ssm_conv_fwd: filter launch");
   if (s != FC_OK) return s;
-  return cuda_status(fc::launch_fftconv(u, f, L, D, y, B, H, L, L, 1, dtype, st), "ssm_conv_fwd: conv launch");
+  return cuda_status(fc::launch_fftconv(u, f, L, none, D, y, B, H, L, L, 1, dtype, st),
+                     "ssm_conv_fwd: conv launch");
 }
 
 // workspace layout: [f_T: H*T floats][s: B*H*C*N complex][x: B*H*C*N complex], each 256-aligned
@@ -171,7 +180,8 @@ FC_API fc_status fftconv_statepass(const void* u, const float* dt, const float* 
   cudaStream_t st = (cudaStream_t)stream;
   s = cuda_status(fc::launch_ssm_gen(dt, lambda, Bp, Cp, H, N, chunk, fT, st), "statepass: filter launch");
   if (s != FC_OK) return s;
-  s = cuda_status(fc::launch_fftconv(u, fT, chunk, D, y, B, H, L, chunk, C, dtype, st),
+  const fc::SsmArgs none{nullptr, nullptr, nullptr, nullptr, 0};
+  s = cuda_status(fc::launch_fftconv(u, fT, chunk, none, D, y, B, H, L, chunk, C, dtype, st),
                   "statepass: chunk conv launch");
   if (s != FC_OK) return s;
   return cuda_status(fc::launch_statepass_tail(u, dt, lambda, Bp, Cp, y, B, H, L, N, chunk, state_in, state_out,
@@ -219,8 +229,13 @@ FC_API fc_status h3_mixer_fwd(const void* q, const void* k, const void* v, const
   cudaStream_t st = (cudaStream_t)stream;
   s = cuda_status(fc::launch_ssm_gen(dt, lambda, Bp, Cp, heads, N, L, f, st), "h3_mixer: filter launch");
   if (s != FC_OK) return s;
+  if (dtype == FC_F16 || dtype == FC_BF16)
+    return cuda_status(fc::launch_h3_mixer_tc(q, k, v, Cshift, f, D, o, B, L, heads, shift_len, dtype, st),
+                       "h3_mixer (tensor cores) launch");
   return cuda_status(fc::launch_h3_mixer(q, k, v, Cshift, f, D, o, B, L, heads, shift_len, dtype, st),
                      "h3_mixer launch");
 }
+
+FC_TEST_API unsigned int fc_debug_tc_timeouts(void) { return fc::mixer_tc_timeouts(); }
 
 }  // extern "C"

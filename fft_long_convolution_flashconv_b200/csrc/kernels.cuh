@@ -8,12 +8,23 @@
 
 namespace fc {
 
+// Diagonal-SSM parameters for kernels that generate their filter (dt == nullptr: none).
+struct SsmArgs {
+  const float* dt;
+  const float2* lam;
+  const float2* Bp;
+  const float2* Cp;
+  int N;
+};
+
 cudaError_t launch_ssm_gen(const float* dt, const float* lam, const float* Bp, const float* Cp, int H, int N, int L,
                            float* f, cudaStream_t st);
 
 // dtype: 0 f32, 1 f16, 2 bf16.  Lc = transform half-length (chunk), C chunks per row.
-cudaError_t launch_fftconv(const void* u, const float* f, int fstride, const float* D, void* y, int B, int H,
-                           long long Lrow, int Lc, int C, int dtype, cudaStream_t st);
+// sp.dt != nullptr: generate the filter from the SSM parameters inside the
+// kernel (Lc >= 1024); otherwise read it from f (row stride fstride).
+cudaError_t launch_fftconv(const void* u, const float* f, int fstride, SsmArgs sp, const float* D, void* y, int B,
+                           int H, long long Lrow, int Lc, int C, int dtype, cudaStream_t st);
 
 cudaError_t launch_statepass_tail(const void* u, const float* dt, const float* lam, const float* Bp,
                                   const float* Cp, void* y, int B, int H, int L, int N, int T,
@@ -23,5 +34,12 @@ cudaError_t launch_statepass_tail(const void* u, const float* dt, const float* l
 cudaError_t launch_h3_mixer(const void* q, const void* k, const void* v, const float* Cshift, const float* fdiag,
                             const float* D, void* o, int B, int L, int heads, int shift_len, int dtype,
                             cudaStream_t st);
+
+// Tensor-core H3 mixer (fp16 / bf16 I/O, head_dim 64, shift_len <= 8).
+cudaError_t launch_h3_mixer_tc(const void* q, const void* k, const void* v, const float* Cshift, const float* fdiag,
+                               const float* D, void* o, int B, int L, int heads, int shift_len, int dtype,
+                               cudaStream_t st);
+// Number of tensor-core CTAs that gave up waiting for an MMA (0 in normal operation).
+unsigned int mixer_tc_timeouts();
 
 }  // namespace fc

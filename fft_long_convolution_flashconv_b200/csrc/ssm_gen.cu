@@ -2,63 +2,51 @@
 //   f[h,k] = 2 Re sum_n C[h,n] B[h,n] A[h,n]^k,  A = exp(dt * lambda)
 // (H3 blog "The Convolution Connection": f = [CB, CAB, CA^2B, ...]).
 //
-// The powers are factored A^k = A^(k0 + 64 kh) * A^(kl), k = k0 + 64 kh + kl,
-// so the N-sum is a small real contraction per channel:
-//   f[k0 + 64 kh + kl] = sum_n Re( W[kh][n] * Q[n][kl] )
-//   W[kh][n] = 2 C_n B_n A_n^(k0 + 64 kh),   Q[n][kl] = A_n^kl
-// Every table entry is an exactly phase-reduced power (fc::ssm_pow), so no
-// error builds up along k however long the filter is.
+// One CTA evaluates 2048 taps of one channel with the factored tables of
+// ssm_tables.cuh (a real contraction over the modes, blocks of 64 modes).
 #include "kernels.cuh"
+
+#include "ssm_tables.cuh"
 
 namespace fc {
 
 constexpr int kGenTile = 2048;    // taps per CTA
 constexpr int kGenThreads = 256;
-
-constexpr int kGenNB = 64;        // modes per table block
+constexpr int kGenMB = 64;        // modes per table block
+constexpr int kGenKH = kGenTile / 64;
+constexpr size_t kGenSmem = sizeof(float2) * ((size_t)kGenMB * 64 + (size_t)kGenKH * kGenMB +
+                                              (size_t)kGenMB * ssm_scratch_per_mode(kGenKH));
 
 __global__ void __launch_bounds__(kGenThreads) ssm_gen_kernel(const float* __restrict__ dt,
                                                              const float2* __restrict__ lam,
                                                              const float2* __restrict__ Bp,
                                                              const float2* __restrict__ Cp, int H, int N,
                                                              int L, float* __restrict__ f) {
-  __shared__ float2 Qt[kGenNB * 64];               // [n][kl]
-  __shared__ float2 Wt[(kGenTile / 64) * kGenNB];  // [kh][n]
+  extern __shared__ float2 gsm[];
+  float2* Q = gsm;                       // [m][64]
+  float2* W = Q + kGenMB * 64;           // [kh][kGenMB]
+  float2* X = W + kGenKH * kGenMB;       // scratch
   const int h = blockIdx.y;
-  const int k0 = blockIdx.x * kGenTile;
-  const int ntap = min(kGenTile, L - k0);
+  const long long k0 = (long long)blockIdx.x * kGenTile;
+  const int ntap = (int)min((long long)kGenTile, (long long)L - k0);
   const int KH = (ntap + 63) >> 6;
-  const float d = dt[h];
   const int kl = threadIdx.x & 63;
   const int kg = threadIdx.x >> 6;  // 0..3
-  constexpr int PER = kGenTile / 64 / (kGenThreads / 64);  // 8
+  constexpr int PER = kGenKH / (kGenThreads / 64);  // 8
   float acc[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) acc[i] = 0.f;
-  for (int n0 = 0; n0 < N; n0 += kGenNB) {
-    const int nb = min(kGenNB, N - n0);
+  for (int m0 = 0; m0 < N; m0 += kGenMB) {
+    const int mb = min(kGenMB, N - m0);
     __syncthreads();  // previous block's readers are done
-    for (int idx = threadIdx.x; idx < nb * 64; idx += blockDim.x) {
-      const int n = idx >> 6, e = idx & 63;
-      const float2 lm = lam[(size_t)h * N + n0 + n];
-      Qt[idx] = ssm_pow(d, lm.x, lm.y, (double)e);
-    }
-    for (int idx = threadIdx.x; idx < nb * KH; idx += blockDim.x) {
-      const int n = idx / KH, kh = idx - n * KH;
-      const size_t pn = (size_t)h * N + n0 + n;
-      const float2 lm = lam[pn];
-      const float2 cb = cmul(Cp[pn], Bp[pn]);
-      const float2 w = cmul(cb, ssm_pow(d, lm.x, lm.y, (double)k0 + 64.0 * kh));
-      Wt[kh * kGenNB + n] = make_float2(2.f * w.x, 2.f * w.y);
-    }
-    __syncthreads();
-    for (int n = 0; n < nb; ++n) {
-      const float2 q = Qt[n * 64 + kl];
+    ssm_fill_tables(dt, lam, Bp, Cp, h, N, m0, mb, kGenMB, k0, KH, Q, W, X, threadIdx.x, kGenThreads);
+    for (int m = 0; m < mb; ++m) {
+      const float2 q = Q[m * 64 + kl];
 #pragma unroll
       for (int i = 0; i < PER; ++i) {
         const int kh = kg + 4 * i;
         if (kh < KH) {
-          const float2 w = Wt[kh * kGenNB + n];
+          const float2 w = W[kh * kGenMB + m];
           acc[i] = fmaf(w.x, q.x, fmaf(-w.y, q.y, acc[i]));
         }
       }
@@ -74,10 +62,12 @@ __global__ void __launch_bounds__(kGenThreads) ssm_gen_kernel(const float* __res
 cudaError_t launch_ssm_gen(const float* dt, const float* lam, const float* Bp, const float* Cp, int H, int N,
                            int L, float* f, cudaStream_t st) {
   const int tiles = (L + kGenTile - 1) / kGenTile;
+  cudaError_t e = cudaFuncSetAttribute(ssm_gen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGenSmem);
+  if (e != cudaSuccess) return e;
   dim3 grid(tiles, H);
-  ssm_gen_kernel<<<grid, kGenThreads, 0, st>>>(dt, reinterpret_cast<const float2*>(lam),
-                                               reinterpret_cast<const float2*>(Bp),
-                                               reinterpret_cast<const float2*>(Cp), H, N, L, f);
+  ssm_gen_kernel<<<grid, kGenThreads, kGenSmem, st>>>(dt, reinterpret_cast<const float2*>(lam),
+                                                      reinterpret_cast<const float2*>(Bp),
+                                                      reinterpret_cast<const float2*>(Cp), H, N, L, f);
   return cudaGetLastError();
 }
 

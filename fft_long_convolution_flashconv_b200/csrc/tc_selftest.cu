@@ -1,0 +1,84 @@
+// Self-test of the tcgen05 wrappers (test hook, not part of the convolution
+// path): D[128 x N] = A[128 x K] * B[N x K]^T with fp16 or bf16 operands staged
+// into the K-major no-swizzle layout, accumulated in tensor memory, read back
+// with tcgen05.ld.  Used by the GPU tests to pin the descriptor and TMEM
+// layouts against a plain matrix product.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "../../include/flashconv_testing.h"
+#include "tc100.cuh"
+
+namespace fc {
+
+__global__ void __launch_bounds__(128, 1) umma_selftest_kernel(const uint16_t* __restrict__ A,
+                                                               const uint16_t* __restrict__ B, float* __restrict__ D,
+                                                               int* __restrict__ err, int N, int K, int bf16) {
+  extern __shared__ __align__(1024) uint8_t sm[];
+  __shared__ uint64_t mbar;
+  __shared__ uint32_t tmem_base;
+  uint8_t* sA = sm;                       // 128 x K
+  uint8_t* sB = sm + (size_t)128 * K * 2; // N x K
+  const int tid = threadIdx.x, warp = tid >> 5;
+  // stage operands (element-wise; this is a test)
+  for (int idx = tid; idx < 128 * K; idx += 128) {
+    const int r = idx / K, k = idx - r * K;
+    *reinterpret_cast<uint16_t*>(sA + tc::kmaj_off(r, k, K)) = A[idx];
+  }
+  for (int idx = tid; idx < N * K; idx += 128) {
+    const int r = idx / K, k = idx - r * K;
+    *reinterpret_cast<uint16_t*>(sB + tc::kmaj_off(r, k, K)) = B[idx];
+  }
+  uint32_t ncols = 32;
+  while (ncols < (uint32_t)N) ncols <<= 1;
+  if (warp == 0) tc::tmem_alloc(&tmem_base, ncols);
+  if (tid == 0) {
+    tc::mbar_init(&mbar, 1);
+    tc::fence_mbar_init();
+  }
+  tc::fence_smem_to_async();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = tmem_base;
+  if (tid == 0) {
+    const uint32_t idesc = tc::idesc_f16(128, N, bf16);
+    const uint32_t a0 = tc::smem_u32(sA), b0 = tc::smem_u32(sB);
+    for (int kk = 0; kk < K / 16; ++kk) {
+      const uint64_t ad = tc::desc_kmajor(a0 + kk * 256, 128, (K / 8) * 128);
+      const uint64_t bd = tc::desc_kmajor(b0 + kk * 256, 128, (K / 8) * 128);
+      tc::mma_f16(tbase, ad, bd, idesc, kk > 0 ? 1u : 0u);
+    }
+    tc::mma_commit(&mbar);
+  }
+  const bool ok = tc::mbar_wait_bounded(&mbar, 0, 1000000000ull);
+  tc::fence_after_sync();
+  if (!ok) {
+    if (tid == 0) atomicExch(err, 1);
+  } else {
+    const int row = warp * 32 + (tid & 31);
+    for (int c = 0; c < N; c += 16) {
+      float v[16];
+      tc::tmem_ld16_wait(tbase + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
+      for (int i = 0; i < 16; ++i) D[(size_t)row * N + c + i] = v[i];
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tbase, ncols);
+}
+
+}  // namespace fc
+
+extern "C" FC_TEST_API int fc_selftest_umma(const void* A, const void* B, float* D, int* err, int N, int K, int bf16,
+                                            void* stream) {
+  if (!A || !B || !D || !err) return -1;
+  if (N < 16 || N > 256 || N % 16 || K < 16 || K > 256 || K % 16 || (bf16 != 0 && bf16 != 1)) return -1;
+  const size_t smem = (size_t)(128 + N) * K * 2;
+  cudaError_t e = cudaFuncSetAttribute(fc::umma_selftest_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return -3;
+  fc::umma_selftest_kernel<<<1, 128, smem, (cudaStream_t)stream>>>((const uint16_t*)A, (const uint16_t*)B, D, err,
+                                                                   N, K, bf16);
+  return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}

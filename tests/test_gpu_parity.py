@@ -98,6 +98,20 @@ def test_fftconv_arbitrary_filter_and_impulse_alignment():
             assert np.max(np.abs(y[i, h, :s])) < 1e-5 * np.max(np.abs(f[h])) if s else True
 
 
+@pytest.mark.parametrize("L,N,dtype", [(1024, 65, "f32"), (2048, 40, "f16"), (4096, 17, "bf16"), (8192, 70, "f32"),
+                                       (512, 64, "f16")])
+def test_ssm_conv_fused_generation(L, N, dtype):
+    """ssm_conv_fwd generates the filter inside the convolution kernel for
+    L >= 1024 (several mode blocks, odd B, channels split across CTAs)."""
+    B, H = 3, 7
+    wl = W.make_conv(B=B, H=H, L=L, N=N, dtype=dtype, seed=N + L, dt_range=("loguniform", -3.0, -1.0))
+    dtt, lam, Bp, Cp, D = params(wl)
+    y = host(api.ssm_conv_fwd(dev(wl.u, dtype), dtt, lam, Bp, Cp, D))
+    f = O.ssm_filter(wl.dt, wl.lam, wl.Bp, wl.Cp, L)
+    ref = cref.causal_conv(wl.u, f, wl.D.astype(np.float64))
+    assert O.row_rel_err(y.reshape(-1, L), ref.reshape(-1, L)) < TOL[dtype]
+
+
 def test_ssm_conv_cfg1_full():
     wl = W.make("cfg1_conv_f32_B1_H4_L256")
     dtt, lam, Bp, Cp, D = params(wl)
@@ -220,13 +234,26 @@ def _head_err(o, ref, mw, rows, ts):
     return err
 
 
-@pytest.mark.parametrize("dtype,L,S", [("f32", 200, 4), ("f16", 130, 4), ("f32", 64, 1), ("bf16", 96, 3)])
-def test_h3_mixer_small(dtype, L, S):
-    mw = W.make_mixer(B=2, L=L, heads=2, head_dim=64, N=8, shift_len=S, dtype=dtype, seed=L)
+@pytest.mark.parametrize("dtype,L,S,heads", [("f32", 200, 4, 2), ("f16", 130, 4, 2), ("f32", 64, 1, 2),
+                                             ("bf16", 96, 3, 2), ("f16", 256, 8, 3), ("bf16", 129, 1, 1),
+                                             ("f16", 300, 2, 2)])
+def test_h3_mixer_small(dtype, L, S, heads):
+    """fp32 I/O runs the CUDA-core kernel, fp16/bf16 the tensor-core one
+    (128-row tiles: ragged, exact and multi-tile lengths)."""
+    mw = W.make_mixer(B=2, L=L, heads=heads, head_dim=64, N=8, shift_len=S, dtype=dtype, seed=L)
     o = _mixer_gpu(mw)
     ref = _mixer_ref(mw)
-    rows = [(b, h) for b in range(2) for h in range(2)]
+    rows = [(b, h) for b in range(2) for h in range(heads)]
     assert _head_err(o, ref, mw, rows, np.arange(L)) < TOL[dtype]
+
+
+def test_tensor_core_waits_never_timed_out():
+    import ctypes
+    from fft_long_convolution_flashconv_b200 import _lib
+    lib = _lib.load()
+    lib.fc_debug_tc_timeouts.restype = ctypes.c_uint
+    torch.cuda.synchronize()
+    assert lib.fc_debug_tc_timeouts() == 0
 
 
 def test_h3_mixer_cfg5_full_sampled():
