@@ -29,6 +29,17 @@ __host__ __device__ __forceinline__ constexpr uint32_t kmaj_off(uint32_t r, uint
   return (r >> 3) * (KT >> 3) * 128u + (k >> 3) * 128u + (r & 7u) * 16u + (k & 7u) * 2u;
 }
 
+// Byte offset of element (r, k) (r along M or N) for general leading / stride
+// byte offsets: K-major core matrices are 8 rows x 8 K-elements with K
+// contiguous; MN-major core matrices are 8 K-rows x 8 MN-elements with MN
+// contiguous.  lbo = offset between core matrices along K, sbo = along M/N.
+__host__ __device__ __forceinline__ constexpr uint32_t op_off(uint32_t r, uint32_t k, bool mn_major, uint32_t lbo,
+                                                              uint32_t sbo) {
+  return (r >> 3) * sbo + (k >> 3) * lbo + (mn_major ? ((k & 7u) * 16u + (r & 7u) * 2u) : ((r & 7u) * 16u + (k & 7u) * 2u));
+}
+
+// Descriptor of a no-swizzle operand tile (K-major or MN-major; the major-ness
+// itself is in the instruction descriptor).
 __device__ __forceinline__ uint64_t desc_kmajor(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
@@ -39,10 +50,10 @@ __device__ __forceinline__ uint64_t desc_kmajor(uint32_t saddr, uint32_t lbo_byt
 }
 
 // kind::f16 instruction descriptor: fp32 accumulator, A and B both fp16
-// (ab_bf16 = 0) or both bf16 (1), both K-major, dense.
-__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int ab_bf16) {
-  return (1u << 4) | ((uint32_t)ab_bf16 << 7) | ((uint32_t)ab_bf16 << 10) | ((uint32_t)(N >> 3) << 17) |
-         ((uint32_t)(M >> 4) << 24);
+// (ab_bf16 = 0) or both bf16 (1), dense; a_mn / b_mn select MN-major operands.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int ab_bf16, int a_mn = 0, int b_mn = 0) {
+  return (1u << 4) | ((uint32_t)ab_bf16 << 7) | ((uint32_t)ab_bf16 << 10) | ((uint32_t)a_mn << 15) |
+         ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,

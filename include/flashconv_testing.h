@@ -25,6 +25,14 @@ extern "C" {
 FC_TEST_API int fc_selftest_umma(const void* A, const void* B, float* D, int* err, int N, int K, int bf16,
                                  void* stream);
 
+/* Same product with general operand layouts: a_mn / b_mn = 1 selects an
+ * MN-major operand (core matrices of 8 K-rows x 8 contiguous MN-elements),
+ * 0 a K-major one; *_lbo / *_sbo are the byte offsets between core matrices
+ * along K / along M or N (multiples of 16, padding allowed).  Returns -1 for
+ * arguments outside those limits or a shared-memory footprint above 200 KB. */
+FC_TEST_API int fc_selftest_umma2(const void* A, const void* B, float* D, int* err, int N, int K, int bf16, int a_mn,
+                                  int b_mn, int a_lbo, int a_sbo, int b_lbo, int b_sbo, void* stream);
+
 /* Number of tensor-core CTAs (all tcgen05 kernels of the library, since load)
  * that gave up waiting for MMA completion after their bounded wait; each such
  * CTA skipped its remaining work and freed its tensor memory.  0 in normal
