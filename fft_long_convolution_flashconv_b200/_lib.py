@@ -27,6 +27,9 @@ SIGNATURES = {
     "fftconv_statepass_workspace": (_sz, [_i, _i, _i, _i, _i]),
     "fftconv_statepass": (_i, [_vp, _fp, _fp, _fp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _fp, _fp, _vp, _sz,
                                _i, _vp]),
+    "ssm_conv_fwd_noalloc": (_i, [_vp, _fp, _fp, _fp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _vp]),
+    "ssm_conv_noalloc_max_filter_floats": (_sz, []),
+    "ssm_conv_noalloc_last_error": (ctypes.c_char_p, []),
     "h3_mixer_workspace": (_sz, [_i, _i, _i, _i, _i]),
     "h3_mixer_fwd": (_i, [_vp, _vp, _vp, _fp, _fp, _fp, _fp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _i, _vp, _sz,
                           _i, _vp]),

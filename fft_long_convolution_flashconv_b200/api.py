@@ -107,6 +107,22 @@ def ssm_conv_fwd(u, dt, lam, Bp, Cp, D, workspace: Optional[torch.Tensor] = None
     return out
 
 
+def ssm_conv_fwd_noalloc(u, dt, lam, Bp, Cp, D, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """ssm_conv_fwd without a workspace: the filter goes to a fixed scratch
+    array inside the library (H * L <= ssm_conv_noalloc_max_filter_floats())."""
+    lib = _lib.load()
+    B, H, L = u.shape
+    dt, lam, Bp, Cp, D = _f32(dt), _cpx(lam), _cpx(Bp), _cpx(Cp), _f32(D)
+    N = lam.shape[1]
+    if out is None:
+        out = torch.empty_like(u)
+    st = lib.ssm_conv_fwd_noalloc(_ptr(u), _ptr(dt), _ptr(lam), _ptr(Bp), _ptr(Cp), _ptr(D), _ptr(out), B, H, L, N,
+                                  _dtype(u), _stream())
+    if st != _lib.FC_OK:
+        raise _lib.FlashConvError(st, "ssm_conv_fwd_noalloc", lib.ssm_conv_noalloc_last_error().decode())
+    return out
+
+
 def statepass_workspace_bytes(B, H, L, N, chunk) -> int:
     return int(_lib.load().fftconv_statepass_workspace(B, H, L, N, chunk))
 

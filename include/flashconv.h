@@ -139,6 +139,35 @@ FC_API fc_status h3_mixer_fwd(const void* q, const void* k, const void* v, const
                               int shift_len, void* workspace, size_t ws_bytes, fc_dtype dtype,
                               void* stream);
 
+/* ssm_conv_fwd_noalloc -- ssm_conv_fwd for callers that cannot allocate
+ * device memory.  The pages have no counterpart to this call.
+ *
+ * Some callers cannot call cudaMalloc or lend the library a workspace: code
+ * embedded in a host application whose memory manager owns every byte of
+ * device memory, or a latency-critical path where an allocation is not
+ * allowed.  This variant keeps its only scratch, the H x L float filter, in a
+ * fixed 4 MiB array compiled into the library, so it takes no workspace and
+ * allocates nothing.  Every GPU that loads the library holds one copy of that
+ * array until the process exits.
+ *  - The first call on a device looks up the array's device address with
+ *    cudaGetSymbolAddress (that device current) and caches it; make that
+ *    first call on each device before any stream capture.
+ *  - Limit: H * L <= ssm_conv_noalloc_max_filter_floats() (1,048,576);
+ *    larger sizes return FC_EUNSUPPORTED and launch nothing.
+ *  - All calls share the one array and it keeps the last call's contents.
+ *    Each call rewrites the whole filter it then reads, so nothing of an
+ *    earlier call reaches a result, but calls that can overlap on the GPU
+ *    (different streams with no ordering between them) race on the array and
+ *    must not be issued that way.
+ *  - Arguments, other limits and results as ssm_conv_fwd (the filter is
+ *    generated by a separate kernel, then convolved).  On failure the message
+ *    is in ssm_conv_noalloc_last_error() (per host thread). */
+FC_API fc_status ssm_conv_fwd_noalloc(const void* u, const float* dt, const float* lambda, const float* Bp,
+                                      const float* Cp, const float* D, void* y, int B, int H, int L, int N,
+                                      fc_dtype dtype, void* stream);
+FC_API size_t ssm_conv_noalloc_max_filter_floats(void);
+FC_API const char* ssm_conv_noalloc_last_error(void);
+
 #ifdef __cplusplus
 }
 #endif

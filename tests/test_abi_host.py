@@ -132,3 +132,14 @@ def test_error_message_is_per_call():
     assert lib.fftconv_fwd(P, P2, P3, P + (1 << 26), 2, 3, 1000, 1, None) != 0
     assert _err()
     assert lib.fc_status_string(0) == b"ok"
+
+
+def test_noalloc_rejects_oversize_before_any_launch():
+    lib = _lib.load()
+    assert lib.ssm_conv_noalloc_max_filter_floats() == 1 << 20
+    # H * L = 2^21 > the fixed scratch: refused on the host, nothing launched
+    y = P + (1 << 28)
+    assert lib.ssm_conv_fwd_noalloc(P, P2, P3, P, P2, P3, y, 1, 256, 8192, 64, 1, None) == _lib.FC_EUNSUPPORTED
+    assert b"fixed scratch" in lib.ssm_conv_noalloc_last_error()
+    assert lib.ssm_conv_fwd_noalloc(P, P2, P3, P, P2, P3, y, 1, 4, 1000, 64, 1, None) == _lib.FC_EUNSUPPORTED
+    assert lib.ssm_conv_fwd_noalloc(None, P2, P3, P, P2, P3, y, 1, 4, 1024, 64, 1, None) == _lib.FC_EINVAL
