@@ -11,7 +11,7 @@ and runs the fused FFT convolution.
                   [--others] [--impl ours|reference]
 
 Timing: W untimed warm-up steps; then K steps, each preceded by an L2 flush
-(a 256 MiB write, outside the per-step CUDA events) and bracketed by events
+(a 256 MiB write then a 256 MiB read, outside the per-step events) and bracketed by events
 on the launching stream; a barrier and a synchronize bracket the loop; the
 value is the max over ranks.  Multi-GPU runs shard nothing: every rank runs
 its own full batch (weak scaling, no data-path collective).
@@ -109,6 +109,7 @@ def run_ours(args, rank, world, local_rank):
         return torch.tensor(np.asarray(x), dtype=torch.float64).to(td).to(dev).contiguous()
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    rflush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
     res = {}
     step_fn, conv_fn, units, alg_bytes, kern_per_step, e2e_fn, e2e_bytes = build_step(wl, T, dev, api, lib)
     # warm-up
@@ -123,6 +124,16 @@ def run_ours(args, rank, world, local_rank):
         for _ in range(20):
             step_fn()
         torch.cuda.synchronize()
+    # One step = the library calls of build_step, captured once into a CUDA
+    # graph and replayed, so host-side call overhead does not leave the GPU idle
+    # inside the timed interval (the same kernels, arguments and stream order).
+    graph = None
+    if args.graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step_fn()
+        graph.replay()
+        torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -130,9 +141,13 @@ def run_ours(args, rank, world, local_rank):
            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     wall0 = time.time()
     for i in range(args.steps):
-        flush.zero_()
+        flush_l2(flush, rflush)
         ev[i][0].record(stream)
-        conv_fn(ev[i][1])         # records ev[i][1] right before the dominant launch
+        if graph is not None:
+            ev[i][1].record(stream)
+            graph.replay()
+        else:
+            conv_fn(ev[i][1])     # records ev[i][1] right before the dominant launch
         ev[i][2].record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -166,11 +181,12 @@ def run_ours(args, rank, world, local_rank):
         dtype="f32",
         data="synthetic",
         config=dict(workload=args.workload, B=wl.B, H=wl.H, L=wl.L, N=wl.N, io_dtype=wl.dtype,
+                    timing="CUDA-graph replay of the step's library calls" if args.graph else "direct calls",
                     filter="generated on device every step" if "conv" in args.workload else None,
-                    l2="flushed before every step (256 MiB write, outside the per-step events)",
+                    l2="flushed before every step (256 MiB write + 256 MiB read, outside the per-step events)",
                     parallelism=f"replicas x{world} (rows independent, no collective)"),
         roofline=dict(bound="hbm", achieved=achieved, peak=peak, unit="GB/s", frac=achieved / peak,
-                      traffic=traffic, kernel="fftconv_kernel (filter generated in-kernel)", peak_source=peak_kind,
+                      traffic=traffic, kernel="the step (filter kernel + fused conv kernel)", peak_source=peak_kind,
                       algorithmic_bytes_per_launch=alg_bytes, avg_launch_ms=conv_avg),
         e2e=dict(value=e2e_val, unit="conv elements/s", h2d_bytes_per_step=e2e_bytes[0],
                  d2h_bytes_per_step=e2e_bytes[1]),
@@ -180,6 +196,14 @@ def run_ours(args, rank, world, local_rank):
     if args.others and rank == 0:
         res["other_workloads"] = other_workloads(T, dev, api, args)
     return res
+
+
+def flush_l2(wbuf, rbuf):
+    """Outside the timed interval: write 256 MiB (evicts every cached line),
+    then read another 256 MiB so that the dirty lines are written back here and
+    L2 is left holding clean, unrelated data."""
+    wbuf.zero_()
+    rbuf.sum()
 
 
 def build_step(wl, T, dev, api, lib):
@@ -245,17 +269,23 @@ def other_workloads(T, dev, api, args):
     out = {}
     peak, _ = hbm_peak()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    rflush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
 
     def timeit(fn, n):
         for _ in range(2):
             fn()
         torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        g.replay()
+        torch.cuda.synchronize()
         tot = 0.0
         for _ in range(n):
-            flush.zero_()
+            flush_l2(flush, rflush)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
-            fn()
+            g.replay()
             b.record()
             torch.cuda.synchronize()
             tot += a.elapsed_time(b)
@@ -385,6 +415,7 @@ def run_reference(args, rank, world):
                 warmup=args.warmup, ms_per_step=tot / args.steps * 1e3, higher_is_better=True, scaling="weak",
                 vs_baseline=None, dtype="f64", data="synthetic", impl="reference",
                 config=dict(workload=args.workload, B=wl.B, H=wl.H, L=wl.L, N=wl.N, io_dtype=wl.dtype,
+                    timing="CUDA-graph replay of the step's library calls" if args.graph else "direct calls",
                             note=f"each step is a bounded sample of {rows} rows on the CPU oracle"),
                 cpu_baseline=dict(value=value, unit="conv elements/s", cores=cref.num_threads(), kind="oracle",
                                   sample=f"{rows} rows per step of {wl.name}"),
@@ -405,6 +436,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=512)
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="time direct library calls instead of a CUDA-graph replay of them")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

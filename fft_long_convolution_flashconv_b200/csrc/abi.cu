@@ -101,6 +101,9 @@ FC_API fc_status fftconv_fwd(const void* u, const float* f, const float* D, void
   FC_REQUIRE(pow2(L) && L >= 16 && L <= 8192, FC_EUNSUPPORTED,
              "fftconv_fwd: L must be a power of two in [16, 8192] (got %d)", L);
   FC_REQUIRE((long long)B * 1 <= (1LL << 30), FC_EUNSUPPORTED, "B too large");
+  if (fc::fftconv_tc_supported(L, dtype))
+    return cuda_status(fc::launch_fftconv_tc(u, f, D, y, B, H, L, dtype, (cudaStream_t)stream),
+                       "fftconv_fwd (tensor cores) launch");
   const fc::SsmArgs none{nullptr, nullptr, nullptr, nullptr, 0};
   return cuda_status(fc::launch_fftconv(u, f, L, none, D, y, B, H, L, L, 1, dtype, (cudaStream_t)stream),
                      "fftconv_fwd launch");
@@ -130,6 +133,12 @@ FC_API fc_status ssm_conv_fwd(const void* u, const float* dt, const float* lambd
   float* f = (float*)workspace;
   cudaStream_t st = (cudaStream_t)stream;
   const fc::SsmArgs none{nullptr, nullptr, nullptr, nullptr, 0};
+  if (fc::fftconv_tc_supported(L, dtype)) {  // filter kernel, then the tensor-core convolution
+    s = cuda_status(fc::launch_ssm_gen(dt, lambda, Bp, Cp, H, N, L, f, st), "ssm_conv_fwd: filter launch");
+    if (s != FC_OK) return s;
+    return cuda_status(fc::launch_fftconv_tc(u, f, D, y, B, H, L, dtype, st),
+                       "ssm_conv_fwd: tensor-core conv launch");
+  }
   if (L >= 1024) {  // filter generated inside the convolution kernel
     const fc::SsmArgs sp{dt, (const float2*)lambda, (const float2*)Bp, (const float2*)Cp, N};
     return cuda_status(fc::launch_fftconv(u, nullptr, L, sp, D, y, B, H, L, L, 1, dtype, st),
@@ -189,12 +198,11 @@ FC_API fc_status fftconv_statepass(const void* u, const float* dt, const float* 
                      "statepass: state launch");
 }
 
+// workspace layout: [f: heads*L floats][k~: B*L*heads*head_dim 16-bit elements], each 256-aligned
 FC_API size_t h3_mixer_workspace(int B, int L, int heads, int head_dim, int N) {
-  (void)B;
-  (void)head_dim;
   (void)N;
-  if (heads < 1 || L < 1) return 0;
-  return round_up((size_t)heads * L * sizeof(float), 256);
+  if (heads < 1 || L < 1 || B < 1 || head_dim < 1) return 0;
+  return round_up((size_t)heads * L * sizeof(float), 256) + round_up((size_t)B * L * heads * head_dim * 2, 256);
 }
 
 FC_API fc_status h3_mixer_fwd(const void* q, const void* k, const void* v, const float* Cshift, const float* dt,
@@ -229,13 +237,15 @@ FC_API fc_status h3_mixer_fwd(const void* q, const void* k, const void* v, const
   cudaStream_t st = (cudaStream_t)stream;
   s = cuda_status(fc::launch_ssm_gen(dt, lambda, Bp, Cp, heads, N, L, f, st), "h3_mixer: filter launch");
   if (s != FC_OK) return s;
-  if (dtype == FC_F16 || dtype == FC_BF16)
-    return cuda_status(fc::launch_h3_mixer_tc(q, k, v, Cshift, f, D, o, B, L, heads, shift_len, dtype, st),
+  if (dtype == FC_F16 || dtype == FC_BF16) {
+    void* kt = (char*)workspace + round_up((size_t)heads * L * sizeof(float), 256);
+    return cuda_status(fc::launch_h3_mixer_tc(q, k, v, Cshift, f, D, o, kt, B, L, heads, shift_len, dtype, st),
                        "h3_mixer (tensor cores) launch");
+  }
   return cuda_status(fc::launch_h3_mixer(q, k, v, Cshift, f, D, o, B, L, heads, shift_len, dtype, st),
                      "h3_mixer launch");
 }
 
-FC_TEST_API unsigned int fc_debug_tc_timeouts(void) { return fc::mixer_tc_timeouts(); }
+FC_TEST_API unsigned int fc_debug_tc_timeouts(void) { return fc::mixer_tc_timeouts() + fc::fftconv_tc_timeouts(); }
 
 }  // extern "C"

@@ -1,0 +1,331 @@
+// Fused FFT convolution with block-FFT stages on the 5th-generation tensor
+// cores (fp16 / bf16 I/O, L = 1024, i.e. M = 2L = 2048 = 128 x 16).
+//
+// H3 summary section 4 "Short-sequence computation": FFT, pointwise multiply
+// and inverse FFT fused in one kernel, with the block FFT written as matrix
+// multiplies so that it runs on the tensor cores (H3 blog, "Fused Block
+// FFTConv").  Index split n = 16 n1 + n2, k = k1 + 128 k2 (n1, k1 < 128,
+// n2, k2 < 16), w_K = exp(-2 pi i / K):
+//   stage A   (GEMM)      Y[k1,n2]  = sum_{n1<64} w_128^(n1 k1) x[16 n1 + n2]
+//                                     (n1 >= 64 is the zero padding)
+//   registers             Y'        = Y w_2048^(k1 n2);  X^[k1+128k2] = DFT16_n2(Y')
+//                         Z^        = X^ . F^ / M;       Z = IDFT16_k2(Z^) w_2048^(-k1 n2)
+//   stage A'  (GEMM)      y[16 n1 + n2] = sum_{k1} w_128^(-n1 k1) Z[k1, n2],  n1 < 64
+// Complex products are split into real GEMMs with fp32 accumulation in TMEM.
+// Two constant 128x128 matrices hold the real DFT-128 blocks,
+//   CA[k1][j] = j<64 ?  cos(2 pi k1 j/128) : sin(2 pi k1 (j-64)/128)
+//   CB[k1][j] = j<64 ? -sin(2 pi k1 j/128) : cos(2 pi k1 (j-64)/128)
+// read K-major by stage A and (the DFT matrix being symmetric) MN-major by
+// stage A':
+//   stage A : Yr = CA[:, :64] Xr + CA[:, 64:] Xi,   Yi = CA[:, :64] Xi + CB[:, :64] Xr
+//   stage A': rows j<64 give Re y[n1=j], rows j>=64 give Im y[n1=j-64]:
+//             y = CA^T Zr + CB^T Zi
+// One CTA takes one channel at a time: its filter and up to 4 row pairs (two
+// real rows packed as one complex sequence u0 + i u1; f is real, so the real
+// and imaginary outputs are the two convolutions) form one batch of
+// N = 16 x (1 + pairs) GEMM columns.  The CTA has two groups of four warps
+// (each group covers the four TMEM lane quarters, thread row k1 = tid % 128);
+// both groups transform the filter column (cheap) and keep its 16 bins per
+// row in registers for the whole channel, then split the row pairs.  Waits on
+// MMA completion are bounded; a CTA that gives up records it in a device
+// counter, skips its remaining work and frees its TMEM.
+#include "fft_stockham.cuh"
+#include "kernels.cuh"
+#include "tc100.cuh"
+
+namespace fc {
+
+static __device__ unsigned int g_fftconv_tc_timeouts;
+
+namespace {
+constexpr int kN1 = 128, kN2 = 16, kM = kN1 * kN2, kL = kM / 2;
+constexpr int kThr = 256;                  // two groups of four warps
+constexpr int kMaxPairs = 4;               // row pairs per batch
+constexpr uint32_t kTmemCols = 256;
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr uint32_t kCLbo = 128, kCSbo = (kN1 / 8) * 128;  // CA / CB K-major: 128 rows x 128 K
+constexpr uint32_t kCBytes = kN1 * kN1 * 2;
+constexpr uint32_t kXZBytes = kMaxPairs * kN2 * 2 * kN1 * 2;  // Z (the larger of X and Z): 2 x 128 x 64 x 2 B
+
+struct TcSmem {
+  uint8_t ca[kCBytes];
+  uint8_t cb[kCBytes];
+  uint8_t xz[kXZBytes];   // stage-A input X, later the stage-A' input Z
+  float2 costab[kN1];
+  uint64_t mbar;
+  uint32_t tmem_base;
+};
+
+template <typename T> struct Op;
+template <> struct Op<__half> {
+  static constexpr int bf16 = 0;
+  static __device__ __forceinline__ uint16_t bits(float x) { return __half_as_ushort(__float2half_rn(x)); }
+  static __device__ __forceinline__ uint32_t pack(float a, float b) {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+  static __device__ __forceinline__ float2 unpack(uint32_t w) {
+    return __half22float2(*reinterpret_cast<__half2*>(&w));
+  }
+};
+template <> struct Op<__nv_bfloat16> {
+  static constexpr int bf16 = 1;
+  static __device__ __forceinline__ uint16_t bits(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
+  static __device__ __forceinline__ uint32_t pack(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+  static __device__ __forceinline__ float2 unpack(uint32_t w) {
+    return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w));
+  }
+};
+}  // namespace
+
+// u, y: B x H x 1024 (T); f: H x 1024 fp32 filters; D: H.
+template <typename T>
+__global__ void __launch_bounds__(kThr, 2) fftconv_tc_kernel(const T* __restrict__ u, const float* __restrict__ f,
+                                                             const float* __restrict__ D, T* __restrict__ y, int B,
+                                                             int H) {
+  extern __shared__ __align__(1024) uint8_t smraw[];
+  TcSmem& sm = *reinterpret_cast<TcSmem*>(smraw);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int row = tid & (kN1 - 1);  // TMEM lane / frequency row k1 / output lane j
+  const int grp = tid >> 7;         // 0 or 1
+  const uint16_t* ub = reinterpret_cast<const uint16_t*>(u);
+  uint16_t* yb = reinterpret_cast<uint16_t*>(y);
+
+  if (warp == 0) tc::tmem_alloc(&sm.tmem_base, kTmemCols);
+  if (tid == 0) {
+    tc::mbar_init(&sm.mbar, 1);
+    tc::fence_mbar_init();
+  }
+  if (tid < kN1) {
+    float s, c;
+    sincospif(2.0f * (float)tid / (float)kN1, &s, &c);
+    sm.costab[tid] = make_float2(c, s);
+  }
+  __syncthreads();
+  // constant DFT-128 blocks, K-major (rows k1, K = j), 8 consecutive j per 16-byte store
+  for (int idx = tid; idx < kN1 * (kN1 / 8); idx += kThr) {
+    const int k1 = idx >> 4, j0 = (idx & 15) * 8;
+    float a[8], b[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int j = j0 + i, jj = j & 63;
+      const float2 cs = sm.costab[(k1 * jj) & 127];
+      a[i] = j < 64 ? cs.x : cs.y;
+      b[i] = j < 64 ? -cs.y : cs.x;
+    }
+    const uint32_t off = tc::kmaj_off(k1, j0, kN1);
+    *reinterpret_cast<uint4*>(sm.ca + off) =
+        make_uint4(Op<T>::pack(a[0], a[1]), Op<T>::pack(a[2], a[3]), Op<T>::pack(a[4], a[5]), Op<T>::pack(a[6], a[7]));
+    *reinterpret_cast<uint4*>(sm.cb + off) =
+        make_uint4(Op<T>::pack(b[0], b[1]), Op<T>::pack(b[2], b[3]), Op<T>::pack(b[4], b[5]), Op<T>::pack(b[6], b[7]));
+  }
+  // this thread's stage twiddles w_2048^(k1 n2), k1 = row
+  float2 tw[kN2];
+#pragma unroll
+  for (int n2 = 0; n2 < kN2; ++n2) {
+    float s, c;
+    sincospif(-2.0f * (float)(row * n2) / (float)kM, &s, &c);
+    tw[n2] = make_float2(c, s);
+  }
+  tc::fence_smem_to_async();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = sm.tmem_base;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+  const uint32_t ca = tc::smem_u32(sm.ca), cb = tc::smem_u32(sm.cb), xz = tc::smem_u32(sm.xz);
+  const int npairs = (B + 1) / 2;
+  uint32_t phase = 0;
+  bool failed = false;
+  float2 fh[kN2];
+
+  for (int h = blockIdx.x; h < H && !failed; h += gridDim.x) {
+    for (int p0 = 0; p0 < npairs && !failed; p0 += kMaxPairs) {
+      const bool with_filter = (p0 == 0);
+      const int P = min(kMaxPairs, npairs - p0);
+      const int NS = P + (with_filter ? 1 : 0);
+      const int NC = NS * kN2;                       // stage-A columns per real/imag half
+      const uint32_t lboX = (uint32_t)(NC / 8) * 128;  // X: MN-major, 64 K-rows (n1) x NC
+      const uint32_t xr = xz, xi = xz + 8 * lboX;
+      // ---- stage X: 16-byte chunks of 8 consecutive n2 at fixed (sequence, n1)
+      for (int idx = tid; idx < NS * 64 * 2; idx += kThr) {
+        const int half = idx & 1, n1 = (idx >> 1) & 63, s = idx >> 7;
+        const int n = s * kN2 + half * 8;
+        const uint32_t off = (uint32_t)(n >> 3) * 128 + (uint32_t)(n1 >> 3) * lboX + (uint32_t)(n1 & 7) * 16;
+        const int t = n1 * kN2 + half * 8;  // time index of the chunk's first element
+        uint4 re = make_uint4(0, 0, 0, 0), im = make_uint4(0, 0, 0, 0);
+        if (with_filter && s == 0) {
+          const float4* fp = reinterpret_cast<const float4*>(f + (size_t)h * kL + t);
+          float4 a = __ldg(fp);
+          const float4 b = __ldg(fp + 1);
+          if (t == 0) a.x += D[h];  // y = f * u + D u = (f + D delta) * u
+          re = make_uint4(Op<T>::pack(a.x, a.y), Op<T>::pack(a.z, a.w), Op<T>::pack(b.x, b.y),
+                          Op<T>::pack(b.z, b.w));
+        } else {
+          const int p = p0 + s - (with_filter ? 1 : 0);
+          const int b0 = 2 * p, b1 = 2 * p + 1;
+          re = *reinterpret_cast<const uint4*>(ub + ((size_t)b0 * H + h) * kL + t);
+          if (b1 < B) im = *reinterpret_cast<const uint4*>(ub + ((size_t)b1 * H + h) * kL + t);
+        }
+        *reinterpret_cast<uint4*>(sm.xz + off) = re;
+        *reinterpret_cast<uint4*>(sm.xz + 8 * lboX + off) = im;
+      }
+      tc::fence_smem_to_async();
+      tc::fence_before_sync();
+      __syncthreads();
+      tc::fence_after_sync();
+      // ---- stage A: D_re at TMEM columns [0, NC), D_im at [NC, 2 NC)
+      if (tid == 0) {
+        const uint32_t idA = tc::idesc_f16(128, NC, Op<T>::bf16, 0, 1);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc::mma_f16(tmem, tc::desc_kmajor(ca + kk * 256, kCLbo, kCSbo), tc::desc_kmajor(xr + kk * 2 * lboX, lboX, 128),
+                      idA, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc::mma_f16(tmem, tc::desc_kmajor(ca + (4 + kk) * 256, kCLbo, kCSbo),
+                      tc::desc_kmajor(xi + kk * 2 * lboX, lboX, 128), idA, 1u);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc::mma_f16(tmem + NC, tc::desc_kmajor(ca + kk * 256, kCLbo, kCSbo),
+                      tc::desc_kmajor(xi + kk * 2 * lboX, lboX, 128), idA, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc::mma_f16(tmem + NC, tc::desc_kmajor(cb + kk * 256, kCLbo, kCSbo),
+                      tc::desc_kmajor(xr + kk * 2 * lboX, lboX, 128), idA, 1u);
+        tc::mma_commit(&sm.mbar);
+      }
+      bool ok = tc::mbar_wait_bounded(&sm.mbar, phase, kWaitNs);
+      phase ^= 1u;
+      if (__syncthreads_or(!ok)) {
+        failed = true;
+        break;
+      }
+      tc::fence_after_sync();
+      // ---- register stage: twiddle, DFT-16, x filter spectrum, IDFT-16, twiddle
+      const uint32_t lboZ = (uint32_t)(P * kN2 / 8) * 128;  // Z: MN-major, 256 K-rows (re k1 | im k1) x P*16
+#pragma unroll 1
+      for (int s = 0; s < NS; ++s) {
+        const bool is_filter = with_filter && s == 0;
+        if (!is_filter && ((s - (with_filter ? 1 : 0)) & 1) != grp) continue;  // pairs alternate between groups
+        float yr[16], yi[16];
+        tc::tmem_ld16x2_wait(tmem + lane_off + (uint32_t)(s * kN2), tmem + lane_off + (uint32_t)(NC + s * kN2), yr, yi);
+        float2 v[kN2];
+#pragma unroll
+        for (int n2 = 0; n2 < kN2; ++n2) v[n2] = cmul(make_float2(yr[n2], yi[n2]), tw[n2]);
+        dft<kN2, -1>(v);
+        if (is_filter) {
+          constexpr float inv_m = 1.0f / (float)kM;
+#pragma unroll
+          for (int k2 = 0; k2 < kN2; ++k2) fh[k2] = make_float2(v[k2].x * inv_m, v[k2].y * inv_m);
+          continue;
+        }
+#pragma unroll
+        for (int k2 = 0; k2 < kN2; ++k2) v[k2] = cmul(v[k2], fh[k2]);
+        dft<kN2, +1>(v);
+#pragma unroll
+        for (int n2 = 0; n2 < kN2; ++n2) v[n2] = cmul(v[n2], cconj(tw[n2]));
+        const int pc = s - (with_filter ? 1 : 0);  // pair column block
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int n = pc * kN2 + half * 8;
+          const uint32_t offr = (uint32_t)(n >> 3) * 128 + (uint32_t)(row >> 3) * lboZ + (uint32_t)(row & 7) * 16;
+          const uint32_t offi = offr + 16 * lboZ;  // K rows 128 + k1
+          const float2* w = v + half * 8;
+          *reinterpret_cast<uint4*>(sm.xz + offr) =
+              make_uint4(Op<T>::pack(w[0].x, w[1].x), Op<T>::pack(w[2].x, w[3].x), Op<T>::pack(w[4].x, w[5].x),
+                         Op<T>::pack(w[6].x, w[7].x));
+          *reinterpret_cast<uint4*>(sm.xz + offi) =
+              make_uint4(Op<T>::pack(w[0].y, w[1].y), Op<T>::pack(w[2].y, w[3].y), Op<T>::pack(w[4].y, w[5].y),
+                         Op<T>::pack(w[6].y, w[7].y));
+        }
+      }
+      tc::fence_smem_to_async();
+      tc::fence_before_sync();
+      __syncthreads();
+      tc::fence_after_sync();
+      // ---- stage A': y = CA^T Zr + CB^T Zi into TMEM columns [0, P*16)
+      if (tid == 0) {
+        const uint32_t idB = tc::idesc_f16(128, P * kN2, Op<T>::bf16, 1, 1);
+        const uint32_t zr = xz, zi = xz + 16 * lboZ;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc::mma_f16(tmem, tc::desc_kmajor(ca + kk * 2 * kCSbo, kCSbo, kCLbo),
+                      tc::desc_kmajor(zr + kk * 2 * lboZ, lboZ, 128), idB, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc::mma_f16(tmem, tc::desc_kmajor(cb + kk * 2 * kCSbo, kCSbo, kCLbo),
+                      tc::desc_kmajor(zi + kk * 2 * lboZ, lboZ, 128), idB, 1u);
+        tc::mma_commit(&sm.mbar);
+      }
+      ok = tc::mbar_wait_bounded(&sm.mbar, phase, kWaitNs);
+      phase ^= 1u;
+      if (__syncthreads_or(!ok)) {
+        failed = true;
+        break;
+      }
+      tc::fence_after_sync();
+      // ---- epilogue: lane j -> (part c = j / 64, n1 = j % 64); the D u term rode
+      // through the transform with the filter (its tap 0 carries D)
+      const int c = row >> 6, n1 = row & 63;
+#pragma unroll 1
+      for (int p = grp; p < P; p += 2) {
+        float yv[16];
+        tc::tmem_ld16_wait(tmem + lane_off + (uint32_t)(p * kN2), yv);
+        const int brow = 2 * (p0 + p) + c;
+        if (brow < B) {
+          const size_t rbase = ((size_t)brow * H + h) * kL + (size_t)n1 * kN2;
+          uint32_t ow[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) ow[i] = Op<T>::pack(yv[2 * i], yv[2 * i + 1]);
+          *reinterpret_cast<uint4*>(yb + rbase) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+          *reinterpret_cast<uint4*>(yb + rbase + 8) = make_uint4(ow[4], ow[5], ow[6], ow[7]);
+        }
+      }
+      tc::fence_before_sync();
+      __syncthreads();
+    }
+  }
+  if (failed && tid == 0) atomicAdd(&g_fftconv_tc_timeouts, 1u);
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
+}
+
+template <typename T>
+static cudaError_t fftconv_tc_t(const void* u, const float* f, const float* D, void* y, int B, int H,
+                                cudaStream_t st) {
+  auto kern = fftconv_tc_kernel<T>;
+  const size_t smem = sizeof(TcSmem) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  static int num_sms = 0;
+  if (num_sms == 0) {
+    int dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+  }
+  const int grid = H < 2 * num_sms ? H : 2 * num_sms;
+  kern<<<grid, kThr, smem, st>>>((const T*)u, f, D, (T*)y, B, H);
+  return cudaGetLastError();
+}
+
+bool fftconv_tc_supported(int L, int dtype) { return L == kL && (dtype == 1 || dtype == 2); }
+
+cudaError_t launch_fftconv_tc(const void* u, const float* f, const float* D, void* y, int B, int H, int L, int dtype,
+                              cudaStream_t st) {
+  if (!fftconv_tc_supported(L, dtype)) return cudaErrorInvalidValue;
+  return dtype == 1 ? fftconv_tc_t<__half>(u, f, D, y, B, H, st) : fftconv_tc_t<__nv_bfloat16>(u, f, D, y, B, H, st);
+}
+
+unsigned int fftconv_tc_timeouts() {
+  unsigned int v = 0;
+  cudaMemcpyFromSymbol(&v, g_fftconv_tc_timeouts, sizeof(v));
+  return v;
+}
+
+}  // namespace fc

@@ -9,8 +9,11 @@
 //   S  = Q_t K~_s^T            tcgen05.mma, M=128 N=128 K=64, fp32 in TMEM
 //   P  = S (.) T_f(t-s)        4 warps: tcgen05.ld, scale, round, store to SMEM
 //   O += P V_s                 tcgen05.mma, M=128 N=64 K=128, fp32 in TMEM
-// The shift SSM k~[s,c] = sum_j Cshift[c,j] k[s-j,c] is applied while the K
-// tile is staged.  Operands use the K-major no-swizzle layout of tc100.cuh.
+// The shift SSM k~[s,c] = sum_j Cshift[c,j] k[s-j,c] runs once, in a small
+// elementwise kernel, into a workspace (rounded to the operand type).  Q and
+// K~ tiles are K-major with padded core-matrix offsets (LBO 144 bytes) so that
+// the row-wise 16-byte staging stores are free of bank conflicts; V is staged
+// as it lies in memory and read by the tensor cores as an MN-major operand.
 // Every wait on MMA completion is bounded; on a timeout the CTA records it in
 // a device counter, skips its remaining work and still frees its TMEM.
 #include "kernels.cuh"
@@ -28,17 +31,25 @@ constexpr int kMaxS = 8;        // shift taps
 constexpr uint32_t kTmemCols = 256;  // S: cols [0,128), O: [128,192)
 constexpr uint64_t kWaitNs = 2000000000ull;
 
+constexpr uint32_t kQLbo = 144, kQSbo = (kHD / 8) * 144;   // Q, K~: 128 rows x 64 K, padded
+constexpr uint32_t kVSbo = 144, kVLbo = (kHD / 8) * 144;   // V: MN-major, 64 N (j) x 128 K (s), padded
+constexpr uint32_t kPLbo = 128, kPSbo = (kT / 8) * 128;    // P: 128 rows x 128 K
 struct MixSmem {
-  uint8_t q[kT * kHD * 2];          // A of S-MMA  (rows t, K = i)
-  uint8_t k[kT * kHD * 2];          // B of S-MMA  (rows s, K = i)
-  uint8_t vt[kHD * kT * 2];         // B of O-MMA  (rows j, K = s)
+  uint8_t q[(kT / 8) * kQSbo];      // A of S-MMA  (rows t, K = i)
+  uint8_t k[(kT / 8) * kQSbo];      // B of S-MMA  (rows s, K = i)
+  uint8_t v[(kT / 8) * kVLbo];      // B of O-MMA  (N = j, K = s), MN-major
   uint8_t p[kT * kT * 2];           // A of O-MMA  (rows t, K = s)
-  uint16_t kraw[(kT + kMaxS) * kHD];  // raw k rows s0-S+1 .. s0+127 (row-major)
-  float cs[kHD * kMaxS];
   float fs[2 * kT];
   uint64_t mbar;
   uint32_t tmem_base;
 };
+
+__device__ __forceinline__ uint32_t qoff(int r, int c8) {
+  return (uint32_t)(r >> 3) * kQSbo + (uint32_t)(c8 >> 3) * kQLbo + (uint32_t)(r & 7) * 16;
+}
+__device__ __forceinline__ uint32_t voff(int s, int j8) {  // 8 consecutive j at time s
+  return (uint32_t)(j8 >> 3) * kVSbo + (uint32_t)(s >> 3) * kVLbo + (uint32_t)(s & 7) * 16;
+}
 }  // namespace
 
 template <typename T> struct Bits;
@@ -61,13 +72,41 @@ template <> struct Bits<__nv_bfloat16> {
   static __device__ __forceinline__ uint16_t fromf(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
 };
 
+// k~ = shift SSM of k (B x L x dm, same type as k), one thread per 8 channels.
 template <typename T>
-__global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restrict__ q, const T* __restrict__ k,
+__global__ void shift_ssm_kernel(const T* __restrict__ k, const float* __restrict__ Cshift, T* __restrict__ kt,
+                                 int B, int L, int dm, int S) {
+  const long long nvec = (long long)B * L * (dm / 8);
+  for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < nvec;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int c8 = (int)(idx % (dm / 8)) * 8;
+    const long long bt = idx / (dm / 8);
+    const int t = (int)(bt % L);
+    const uint16_t* kb = reinterpret_cast<const uint16_t*>(k);
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int j = 0; j < S && j <= t; ++j) {
+      const uint4 w = *reinterpret_cast<const uint4*>(kb + (bt - j) * dm + c8);
+      const uint16_t* e = reinterpret_cast<const uint16_t*>(&w);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = fmaf(__ldg(Cshift + (size_t)(c8 + i) * S + j), Bits<T>::tof(e[i]), acc[i]);
+    }
+    uint4 out;
+    out.x = Bits<T>::pack(acc[0], acc[1]);
+    out.y = Bits<T>::pack(acc[2], acc[3]);
+    out.z = Bits<T>::pack(acc[4], acc[5]);
+    out.w = Bits<T>::pack(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(kt) + bt * dm + c8) = out;
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restrict__ q, const T* __restrict__ kt,
                                                               const T* __restrict__ v,
-                                                              const float* __restrict__ Cshift,
                                                               const float* __restrict__ fdiag,
                                                               const float* __restrict__ D, T* __restrict__ o, int L,
-                                                              int heads, int S) {
+                                                              int heads) {
   extern __shared__ __align__(1024) uint8_t smraw[];
   MixSmem& sm = *reinterpret_cast<MixSmem*>(smraw);
   const int tt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -76,7 +115,7 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
   const int t0 = tt * kT;
   const size_t base = (size_t)b * L * dm + (size_t)h * kHD;
   const uint16_t* qb = reinterpret_cast<const uint16_t*>(q) + base;
-  const uint16_t* kb = reinterpret_cast<const uint16_t*>(k) + base;
+  const uint16_t* kb = reinterpret_cast<const uint16_t*>(kt) + base;
   const uint16_t* vb = reinterpret_cast<const uint16_t*>(v) + base;
 
   if (warp == 0) tc::tmem_alloc(&sm.tmem_base, kTmemCols);
@@ -84,14 +123,13 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
     tc::mbar_init(&sm.mbar, 1);
     tc::fence_mbar_init();
   }
-  for (int idx = tid; idx < kHD * S; idx += kThr) sm.cs[idx] = Cshift[(size_t)(h * kHD) * S + idx];
   // Q tile: rows t0..t0+127, 8-element chunks
   for (int idx = tid; idx < kT * (kHD / 8); idx += kThr) {
     const int r = idx >> 3, c8 = (idx & 7) * 8;
     const int t = t0 + r;
     uint4 val = make_uint4(0, 0, 0, 0);
     if (t < L) val = *reinterpret_cast<const uint4*>(qb + (size_t)t * dm + c8);
-    *reinterpret_cast<uint4*>(sm.q + tc::kmaj_off(r, c8, kHD)) = val;
+    *reinterpret_cast<uint4*>(sm.q + qoff(r, c8)) = val;
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -100,7 +138,7 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
   const uint32_t tS = tmem, tO = tmem + 128;
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
   const uint32_t idS = tc::idesc_f16(128, 128, Bits<T>::bf16);
-  const uint32_t idO = tc::idesc_f16(128, kHD, Bits<T>::bf16);
+  const uint32_t idO = tc::idesc_f16(128, kHD, Bits<T>::bf16, 0, 1);
   const float dh = D[h];
   const float* fh = fdiag + (size_t)h * L;
   uint32_t phase = 0;
@@ -109,48 +147,23 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
 
   for (int st = 0; st <= tt && !failed; ++st) {
     const int s0 = st * kT;
-    // ---- stage raw k rows s0-(S-1) .. s0+127, then k~ (shift SSM) into the K-major tile
-    const int nraw = kT + S - 1;
-    for (int idx = tid; idx < nraw * (kHD / 8); idx += kThr) {
-      const int r = idx >> 3, c8 = (idx & 7) * 8;
-      const int s = s0 - (S - 1) + r;
-      uint4 val = make_uint4(0, 0, 0, 0);
-      if (s >= 0 && s < L) val = *reinterpret_cast<const uint4*>(kb + (size_t)s * dm + c8);
-      *reinterpret_cast<uint4*>(&sm.kraw[r * kHD + c8]) = val;
-    }
-    // V^T tile (rows j, K = s) and the Toeplitz weights for this (t, s) tile pair
+    // ---- stage the K~ and V tiles (rows s0 .. s0+127) and the Toeplitz weights
     for (int idx = tid; idx < kT * (kHD / 8); idx += kThr) {
       const int r = idx >> 3, c8 = (idx & 7) * 8;
       const int s = s0 + r;
-      uint4 val = make_uint4(0, 0, 0, 0);
-      if (s < L) val = *reinterpret_cast<const uint4*>(vb + (size_t)s * dm + c8);
-      const uint16_t* e = reinterpret_cast<const uint16_t*>(&val);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) *reinterpret_cast<uint16_t*>(sm.vt + tc::kmaj_off(c8 + i, r, kT)) = e[i];
+      uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
+      if (s < L) {
+        kv = *reinterpret_cast<const uint4*>(kb + (size_t)s * dm + c8);
+        vv = *reinterpret_cast<const uint4*>(vb + (size_t)s * dm + c8);
+      }
+      *reinterpret_cast<uint4*>(sm.k + qoff(r, c8)) = kv;
+      *reinterpret_cast<uint4*>(sm.v + voff(r, c8)) = vv;
     }
     for (int idx = tid; idx < 2 * kT - 1; idx += kThr) {
       const int d = idx - (kT - 1) + (t0 - s0);  // t - s
       float w = (d >= 0 && d < L) ? fh[d] : 0.f;
       if (d == 0) w += dh;
       sm.fs[idx] = w;
-    }
-    __syncthreads();
-    for (int idx = tid; idx < kT * (kHD / 8); idx += kThr) {
-      const int r = idx >> 3, c8 = (idx & 7) * 8;
-      float acc[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-      for (int j = 0; j < S; ++j) {
-        const uint16_t* kr = &sm.kraw[(r + (S - 1) - j) * kHD + c8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = fmaf(sm.cs[(c8 + i) * S + j], Bits<T>::tof(kr[i]), acc[i]);
-      }
-      uint4 pk;
-      pk.x = Bits<T>::pack(acc[0], acc[1]);
-      pk.y = Bits<T>::pack(acc[2], acc[3]);
-      pk.z = Bits<T>::pack(acc[4], acc[5]);
-      pk.w = Bits<T>::pack(acc[6], acc[7]);
-      *reinterpret_cast<uint4*>(sm.k + tc::kmaj_off(r, c8, kHD)) = pk;
     }
     tc::fence_smem_to_async();
     tc::fence_before_sync();
@@ -161,8 +174,8 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
       const uint32_t qa = tc::smem_u32(sm.q), ka = tc::smem_u32(sm.k);
 #pragma unroll
       for (int kk = 0; kk < kHD / 16; ++kk)
-        tc::mma_f16(tS, tc::desc_kmajor(qa + kk * 256, 128, (kHD / 8) * 128),
-                    tc::desc_kmajor(ka + kk * 256, 128, (kHD / 8) * 128), idS, kk > 0 ? 1u : 0u);
+        tc::mma_f16(tS, tc::desc_kmajor(qa + kk * 2 * kQLbo, kQLbo, kQSbo),
+                    tc::desc_kmajor(ka + kk * 2 * kQLbo, kQLbo, kQSbo), idS, kk > 0 ? 1u : 0u);
       tc::mma_commit(&sm.mbar);
     }
     bool ok = tc::mbar_wait_bounded(&sm.mbar, phase, kWaitNs);
@@ -184,8 +197,10 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
         const float bb = sv[2 * i + 1] * sm.fs[row - (c + 2 * i + 1) + (kT - 1)];
         pw[i] = Bits<T>::pack(a, bb);
       }
-      *reinterpret_cast<uint4*>(sm.p + tc::kmaj_off(row, c, kT)) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
-      *reinterpret_cast<uint4*>(sm.p + tc::kmaj_off(row, c + 8, kT)) = make_uint4(pw[4], pw[5], pw[6], pw[7]);
+      *reinterpret_cast<uint4*>(sm.p + (uint32_t)(row >> 3) * kPSbo + (uint32_t)(c >> 3) * kPLbo + (row & 7) * 16) =
+          make_uint4(pw[0], pw[1], pw[2], pw[3]);
+      *reinterpret_cast<uint4*>(sm.p + (uint32_t)(row >> 3) * kPSbo + (uint32_t)((c + 8) >> 3) * kPLbo + (row & 7) * 16) =
+          make_uint4(pw[4], pw[5], pw[6], pw[7]);
     }
     tc::fence_smem_to_async();
     tc::fence_before_sync();
@@ -193,11 +208,11 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
     tc::fence_after_sync();
     // ---- O += P V
     if (tid == 0) {
-      const uint32_t pa = tc::smem_u32(sm.p), va = tc::smem_u32(sm.vt);
+      const uint32_t pa = tc::smem_u32(sm.p), va = tc::smem_u32(sm.v);
 #pragma unroll
       for (int kk = 0; kk < kT / 16; ++kk)
-        tc::mma_f16(tO, tc::desc_kmajor(pa + kk * 256, 128, (kT / 8) * 128),
-                    tc::desc_kmajor(va + kk * 256, 128, (kT / 8) * 128), idO, (st > 0 || kk > 0) ? 1u : 0u);
+        tc::mma_f16(tO, tc::desc_kmajor(pa + kk * 2 * kPLbo, kPLbo, kPSbo),
+                    tc::desc_kmajor(va + kk * 2 * kVLbo, kVLbo, kVSbo), idO, (st > 0 || kk > 0) ? 1u : 0u);
       tc::mma_commit(&sm.mbar);
     }
     ok = tc::mbar_wait_bounded(&sm.mbar, phase, kWaitNs);
@@ -239,23 +254,29 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
 
 template <typename T>
 static cudaError_t mixer_tc_t(const void* q, const void* k, const void* v, const float* Cs, const float* f,
-                              const float* D, void* o, int B, int L, int heads, int S, cudaStream_t st) {
+                              const float* D, void* o, void* kt, int B, int L, int heads, int S, cudaStream_t st) {
+  const int dm = heads * kHD;
+  const long long nvec = (long long)B * L * (dm / 8);
+  const int sgrid = (int)((nvec + 255) / 256 < 148 * 16 ? (nvec + 255) / 256 : 148 * 16);
+  shift_ssm_kernel<T><<<sgrid, 256, 0, st>>>((const T*)k, Cs, (T*)kt, B, L, dm, S);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   const size_t smem = sizeof(MixSmem) + 1024;
   auto kern = h3_mixer_tc_kernel<T>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((L + kT - 1) / kT, heads, B);
-  kern<<<grid, kThr, smem, st>>>((const T*)q, (const T*)k, (const T*)v, Cs, f, D, (T*)o, L, heads, S);
+  kern<<<grid, kThr, smem, st>>>((const T*)q, (const T*)kt, (const T*)v, f, D, (T*)o, L, heads);
   return cudaGetLastError();
 }
 
 cudaError_t launch_h3_mixer_tc(const void* q, const void* k, const void* v, const float* Cshift, const float* fdiag,
-                               const float* D, void* o, int B, int L, int heads, int shift_len, int dtype,
-                               cudaStream_t st) {
+                               const float* D, void* o, void* ktilde, int B, int L, int heads, int shift_len,
+                               int dtype, cudaStream_t st) {
   if (shift_len > kMaxS) return cudaErrorInvalidValue;
   switch (dtype) {
-    case 1: return mixer_tc_t<__half>(q, k, v, Cshift, fdiag, D, o, B, L, heads, shift_len, st);
-    case 2: return mixer_tc_t<__nv_bfloat16>(q, k, v, Cshift, fdiag, D, o, B, L, heads, shift_len, st);
+    case 1: return mixer_tc_t<__half>(q, k, v, Cshift, fdiag, D, o, ktilde, B, L, heads, shift_len, st);
+    case 2: return mixer_tc_t<__nv_bfloat16>(q, k, v, Cshift, fdiag, D, o, ktilde, B, L, heads, shift_len, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -36,10 +36,17 @@ cudaError_t launch_h3_mixer(const void* q, const void* k, const void* v, const f
                             cudaStream_t st);
 
 // Tensor-core H3 mixer (fp16 / bf16 I/O, head_dim 64, shift_len <= 8).
+// ktilde: scratch of B x L x (heads*64) elements of the I/O type (the shift-SSM output).
 cudaError_t launch_h3_mixer_tc(const void* q, const void* k, const void* v, const float* Cshift, const float* fdiag,
-                               const float* D, void* o, int B, int L, int heads, int shift_len, int dtype,
-                               cudaStream_t st);
+                               const float* D, void* o, void* ktilde, int B, int L, int heads, int shift_len,
+                               int dtype, cudaStream_t st);
 // Number of tensor-core CTAs that gave up waiting for an MMA (0 in normal operation).
 unsigned int mixer_tc_timeouts();
+
+// Tensor-core fused FFT convolution (block-FFT stages as tcgen05 GEMMs).
+bool fftconv_tc_supported(int L, int dtype);
+cudaError_t launch_fftconv_tc(const void* u, const float* f, const float* D, void* y, int B, int H, int L, int dtype,
+                              cudaStream_t st);
+unsigned int fftconv_tc_timeouts();
 
 }  // namespace fc

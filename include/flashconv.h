@@ -130,7 +130,8 @@ FC_API fc_status fftconv_statepass(const void* u, const float* dt, const float* 
  * with f_h the diagonal-SSM filter of head h (as ssm_kernel_gen).
  * q, k, v, o: B x L x (heads*head_dim) in `dtype`; Cshift:
  * (heads*head_dim) x shift_len floats; dt, D: heads floats; lambda, Bp, Cp:
- * heads x N complex.  workspace: at least h3_mixer_workspace(...) bytes.
+ * heads x N complex.  workspace: at least h3_mixer_workspace(...) bytes
+ * (the per-head filters and, for 16-bit I/O, the shift-SSM output k~).
  * Limits: head_dim == 64, 1 <= shift_len <= 8, 1 <= L <= 65536, 1 <= N <= 1024. */
 FC_API size_t h3_mixer_workspace(int B, int L, int heads, int head_dim, int N);
 FC_API fc_status h3_mixer_fwd(const void* q, const void* k, const void* v, const float* Cshift,

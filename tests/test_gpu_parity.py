@@ -76,6 +76,19 @@ def test_fftconv_all_sizes(L, dtype):
     assert err < TOL[dtype], err
 
 
+@pytest.mark.parametrize("B,H,dtype", [(10, 3, "f16"), (1, 4, "bf16"), (2, 300, "f16"), (7, 2, "bf16")])
+def test_fftconv_tensor_core_batches(B, H, dtype):
+    """L = 1024 fp16/bf16 runs the tensor-core block FFT: several row-pair
+    batches per channel (B = 10), a single row, more channels than resident
+    CTAs (H = 300), odd B."""
+    L = 1024
+    wl = W.make_conv(B=B, H=H, L=L, N=16, dtype=dtype, seed=B * 1000 + H, dt_range=("loguniform", -3.0, -1.0))
+    f32 = W.round_to(O.ssm_filter(wl.dt, wl.lam, wl.Bp, wl.Cp, L), "f32")
+    y = host(api.fftconv_fwd(dev(wl.u, dtype), dev(f32), dev(wl.D)))
+    ref = cref.causal_conv(wl.u, f32, wl.D.astype(np.float64))
+    assert O.row_rel_err(y.reshape(B * H, L), ref.reshape(B * H, L)) < TOL[dtype]
+
+
 def test_fftconv_arbitrary_filter_and_impulse_alignment():
     """A non-SSM filter; impulses at several offsets land exactly where the
     causal index bookkeeping says (argmax position is an integer check)."""
