@@ -31,6 +31,16 @@ cudaError_t launch_statepass_tail(const void* u, const float* dt, const float* l
                                   const float* state_in, float* state_out, float* s_ws, float* x_ws, int dtype,
                                   cudaStream_t st);
 
+// Tensor-core state passing (fp16 / bf16, T in {2048, 4096, 8192}, N <= 64):
+// end states into s_ws, and the initial-state correction added into y for
+// chunks c >= c_begin (x_ws = state entering each chunk).
+bool statepass_tc_supported(int T, int N, int dtype);
+cudaError_t launch_sp_state_tc(const void* u, const float* dt, const float* lam, const float* Bp, int B, int H, int L,
+                               int N, int T, float* s_ws, int dtype, cudaStream_t st);
+cudaError_t launch_sp_corr_tc(void* y, const float* dt, const float* lam, const float* Cp, const float* x_ws, int B,
+                              int H, int L, int N, int T, int c_begin, int dtype, cudaStream_t st);
+unsigned int statepass_tc_timeouts();
+
 cudaError_t launch_h3_mixer(const void* q, const void* k, const void* v, const float* Cshift, const float* fdiag,
                             const float* D, void* o, int B, int L, int heads, int shift_len, int dtype,
                             cudaStream_t st);

@@ -254,10 +254,29 @@ static cudaError_t sp_tail(const void* u, const float* dt, const float* lam, con
   return cudaGetLastError();
 }
 
+// Tensor-core tail: end states and corrections as tcgen05 GEMMs, the carry as above.
+static cudaError_t sp_tail_tc(const void* u, const float* dt, const float* lam, const float* Bp, const float* Cp,
+                              void* y, int B, int H, int L, int N, int Tc, const float* state_in, float* state_out,
+                              float* s_ws, float* x_ws, int dtype, cudaStream_t st) {
+  const int C = L / Tc;
+  cudaError_t e = launch_sp_state_tc(u, dt, lam, Bp, B, H, L, N, Tc, s_ws, dtype, st);
+  if (e != cudaSuccess) return e;
+  const long long nst = (long long)B * H * N;
+  sp_carry_kernel<<<(unsigned)((nst + 255) / 256), 256, 0, st>>>(dt, (const float2*)lam, (const float2*)s_ws,
+                                                                 (const float2*)state_in, (float2*)state_out,
+                                                                 (float2*)x_ws, B, H, N, C, Tc);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // with no initial state the first chunk needs no correction
+  return launch_sp_corr_tc(y, dt, lam, Cp, x_ws, B, H, L, N, Tc, state_in != nullptr ? 0 : 1, dtype, st);
+}
+
 cudaError_t launch_statepass_tail(const void* u, const float* dt, const float* lam, const float* Bp,
                                   const float* Cp, void* y, int B, int H, int L, int N, int T_,
                                   const float* state_in, float* state_out, float* s_ws, float* x_ws, int dtype,
                                   cudaStream_t st) {
+  if (statepass_tc_supported(T_, N, dtype))
+    return sp_tail_tc(u, dt, lam, Bp, Cp, y, B, H, L, N, T_, state_in, state_out, s_ws, x_ws, dtype, st);
   switch (dtype) {
     case 0: return sp_tail<float>(u, dt, lam, Bp, Cp, y, B, H, L, N, T_, state_in, state_out, s_ws, x_ws, st);
     case 1: return sp_tail<__half>(u, dt, lam, Bp, Cp, y, B, H, L, N, T_, state_in, state_out, s_ws, x_ws, st);

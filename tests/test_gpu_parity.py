@@ -177,15 +177,25 @@ def test_ssm_conv_cfg3_full_sampled_rows():
     (2, 2, 256, 256, 8, "f32"),     # chunk == L
     (1, 2, 256, 16, 8, "f32"),      # smallest chunk
     (2, 3, 2048, 512, 32, "f16"),
+    # tensor-core tail (16-bit I/O, T in {2048, 4096, 8192}, N <= 64)
     (1, 2, 16384, 8192, 64, "bf16"),
+    (2, 3, 8192, 2048, 33, "f16"),      # ragged mode count, 4 chunks
+    (1, 2, 16384, 4096, 64, "bf16"),
+    (1, 3, 2048, 2048, 1, "bf16"),      # one chunk, one mode: correction from state_in only
+    (2, 2, 8192, 2048, 64, "f16-nox0"),  # no initial state: the first chunk is not corrected
 ])
 def test_statepass_small(B, H, L, T, N, dtype):
+    with_x0 = not dtype.endswith("-nox0")
+    dtype = dtype.replace("-nox0", "")
     wl = W.make_conv(B=B, H=H, L=L, N=N, dtype=dtype, seed=L + T, dt_range=("loguniform", -3.0, -1.0))
     dtt, lam, Bp, Cp, D = params(wl)
     rng = np.random.default_rng(1)
     x0 = rng.normal(size=(B, H, N)) + 1j * rng.normal(size=(B, H, N))
+    if not with_x0:
+        x0 = np.zeros_like(x0)
     x0_t = torch.view_as_real(torch.tensor(x0.astype(np.complex64))).cuda().contiguous()
-    y, xs = api.fftconv_statepass(dev(wl.u, dtype), dtt, lam, Bp, Cp, D, T, state_in=x0_t, return_state=True)
+    y, xs = api.fftconv_statepass(dev(wl.u, dtype), dtt, lam, Bp, Cp, D, T, state_in=x0_t if with_x0 else None,
+                                  return_state=True)
     A, Bc, Cc = oracle_A(wl)
     x0_r = x0.astype(np.complex64).astype(np.complex128)
     ref, xref = cref.ssm_recurrence(wl.u, A, Bc, Cc, wl.D.astype(np.float64), x0=x0_r)
