@@ -247,7 +247,7 @@ FC_API fc_status h3_mixer_fwd(const void* q, const void* k, const void* v, const
 }
 
 FC_TEST_API unsigned int fc_debug_tc_timeouts(void) {
-  return fc::mixer_tc_timeouts() + fc::fftconv_tc_timeouts() + fc::statepass_tc_timeouts();
+  return fc::mixer_tc_timeouts() + fc::fftconv_tc_timeouts() + fc::statepass_tc_timeouts() + fc::gen_tc_timeouts();
 }
 
 }  // extern "C"

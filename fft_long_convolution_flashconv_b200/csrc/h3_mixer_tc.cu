@@ -72,32 +72,58 @@ template <> struct Bits<__nv_bfloat16> {
   static __device__ __forceinline__ uint16_t fromf(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
 };
 
-// k~ = shift SSM of k (B x L x dm, same type as k), one thread per 8 channels.
-template <typename T>
-__global__ void shift_ssm_kernel(const T* __restrict__ k, const float* __restrict__ Cshift, T* __restrict__ kt,
-                                 int B, int L, int dm, int S) {
-  const long long nvec = (long long)B * L * (dm / 8);
-  for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < nvec;
-       idx += (long long)gridDim.x * blockDim.x) {
-    const int c8 = (int)(idx % (dm / 8)) * 8;
-    const long long bt = idx / (dm / 8);
-    const int t = (int)(bt % L);
-    const uint16_t* kb = reinterpret_cast<const uint16_t*>(k);
-    float acc[8];
+// k~ = shift SSM of k (B x L x dm, same type as k).  A thread owns 8 adjacent
+// channels (their taps stay in registers) and kSeg consecutive time steps of
+// one sequence: it loads those rows plus the S - 1 rows before them once, all
+// up front, then forms the kSeg outputs from registers.  A warp covers 256
+// adjacent channels of one time step (512-byte coalesced rows).
+constexpr int kSeg = 16;
+template <typename T, int S>
+__global__ void __launch_bounds__(256) shift_ssm_kernel(const T* __restrict__ k, const float* __restrict__ Cshift,
+                                                        T* __restrict__ kt, int B, int L, int dm) {
+  const int ng = dm / 8;
+  const int nseg = (L + kSeg - 1) / kSeg;
+  const long long item = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (item >= (long long)B * nseg * ng) return;
+  const int g = (int)(item % ng);
+  const long long bs = item / ng;
+  const int seg = (int)(bs % nseg), b = (int)(bs / nseg);
+  const int c8 = g * 8;
+  const uint16_t* kb = reinterpret_cast<const uint16_t*>(k) + (size_t)b * L * dm + c8;
+  uint16_t* ob = reinterpret_cast<uint16_t*>(kt) + (size_t)b * L * dm + c8;
+  const int t0 = seg * kSeg;
+  // rows t0 - (S-1) .. t0 + kSeg - 1, all loads issued before any use (zero outside [0, L))
+  uint4 rows[kSeg + S - 1];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    for (int j = 0; j < S && j <= t; ++j) {
-      const uint4 w = *reinterpret_cast<const uint4*>(kb + (bt - j) * dm + c8);
-      const uint16_t* e = reinterpret_cast<const uint16_t*>(&w);
+  for (int i = 0; i < kSeg + S - 1; ++i) {
+    const int t = t0 - (S - 1) + i;
+    rows[i] = (t >= 0 && t < L) ? *reinterpret_cast<const uint4*>(kb + (size_t)t * dm) : make_uint4(0, 0, 0, 0);
+  }
+  float cs[S][8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = fmaf(__ldg(Cshift + (size_t)(c8 + i) * S + j), Bits<T>::tof(e[i]), acc[i]);
+  for (int j = 0; j < S; ++j)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) cs[j][i] = __ldg(Cshift + (size_t)(c8 + i) * S + j);
+#pragma unroll
+  for (int i = 0; i < kSeg; ++i) {
+    const int t = t0 + i;
+    if (t < L) {
+      float acc[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+#pragma unroll
+      for (int j = 0; j < S; ++j) {  // tap j reads row t - j
+        const uint16_t* e = reinterpret_cast<const uint16_t*>(&rows[i + S - 1 - j]);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[c] = fmaf(cs[j][c], Bits<T>::tof(e[c]), acc[c]);
+      }
+      uint4 out;
+      out.x = Bits<T>::pack(acc[0], acc[1]);
+      out.y = Bits<T>::pack(acc[2], acc[3]);
+      out.z = Bits<T>::pack(acc[4], acc[5]);
+      out.w = Bits<T>::pack(acc[6], acc[7]);
+      *reinterpret_cast<uint4*>(ob + (size_t)t * dm) = out;
     }
-    uint4 out;
-    out.x = Bits<T>::pack(acc[0], acc[1]);
-    out.y = Bits<T>::pack(acc[2], acc[3]);
-    out.z = Bits<T>::pack(acc[4], acc[5]);
-    out.w = Bits<T>::pack(acc[6], acc[7]);
-    *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(kt) + bt * dm + c8) = out;
   }
 }
 
@@ -256,9 +282,21 @@ template <typename T>
 static cudaError_t mixer_tc_t(const void* q, const void* k, const void* v, const float* Cs, const float* f,
                               const float* D, void* o, void* kt, int B, int L, int heads, int S, cudaStream_t st) {
   const int dm = heads * kHD;
-  const long long nvec = (long long)B * L * (dm / 8);
-  const int sgrid = (int)((nvec + 255) / 256 < 148 * 16 ? (nvec + 255) / 256 : 148 * 16);
-  shift_ssm_kernel<T><<<sgrid, 256, 0, st>>>((const T*)k, Cs, (T*)kt, B, L, dm, S);
+  const long long items = (long long)B * ((L + kSeg - 1) / kSeg) * (dm / 8);
+  const unsigned sg = (unsigned)((items + 255) / 256);
+  const T* kk = (const T*)k;
+  T* ko = (T*)kt;
+  switch (S) {
+    case 1: shift_ssm_kernel<T, 1><<<sg, 256, 0, st>>>(kk, Cs, ko, B, L, dm); break;
+    case 2: shift_ssm_kernel<T, 2><<<sg, 256, 0, st>>>(kk, Cs, ko, B, L, dm); break;
+    case 3: shift_ssm_kernel<T, 3><<<sg, 256, 0, st>>>(kk, Cs, ko, B, L, dm); break;
+    case 4: shift_ssm_kernel<T, 4><<<sg, 256, 0, st>>>(kk, Cs, ko, B, L, dm); break;
+    case 5: shift_ssm_kernel<T, 5><<<sg, 256, 0, st>>>(kk, Cs, ko, B, L, dm); break;
+    case 6: shift_ssm_kernel<T, 6><<<sg, 256, 0, st>>>(kk, Cs, ko, B, L, dm); break;
+    case 7: shift_ssm_kernel<T, 7><<<sg, 256, 0, st>>>(kk, Cs, ko, B, L, dm); break;
+    case 8: shift_ssm_kernel<T, 8><<<sg, 256, 0, st>>>(kk, Cs, ko, B, L, dm); break;
+    default: return cudaErrorInvalidValue;
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t smem = sizeof(MixSmem) + 1024;

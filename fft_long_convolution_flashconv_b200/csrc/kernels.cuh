@@ -58,5 +58,7 @@ bool fftconv_tc_supported(int L, int dtype);
 cudaError_t launch_fftconv_tc(const void* u, const float* f, const float* D, void* y, int B, int H, int L, int dtype,
                               cudaStream_t st);
 unsigned int fftconv_tc_timeouts();
+// Tensor-core filter generation CTAs that gave up waiting for an MMA.
+unsigned int gen_tc_timeouts();
 
 }  // namespace fc

@@ -2,11 +2,14 @@
 //   f[h,k] = 2 Re sum_n C[h,n] B[h,n] A[h,n]^k,  A = exp(dt * lambda)
 // (H3 blog "The Convolution Connection": f = [CB, CAB, CA^2B, ...]).
 //
-// One CTA evaluates 1024 taps of one channel with the factored tables of
-// ssm_tables.cuh (a real contraction over the modes, blocks of 64 modes).
+// Two kernels: for N <= 64 a tensor-core GEMM per 2048 taps (below); for
+// larger N a CUDA-core kernel in which one CTA evaluates 1024 taps of one
+// channel with the factored tables of ssm_tables.cuh (a real contraction over
+// the modes, blocks of 64 modes).
 #include "kernels.cuh"
 
 #include "ssm_tables.cuh"
+#include "tc100.cuh"
 
 namespace fc {
 
@@ -68,8 +71,211 @@ __global__ void __launch_bounds__(kGenThreads) ssm_gen_kernel(const float* __res
     }
 }
 
+// ---------------------------------------------------------------- tensor-core variant (N <= 64)
+// With t = 16 th + tl (tl < 16) the filter is one real GEMM per 2048 taps:
+//   f[16 th + tl] = sum_k AH[th][k] Q[tl][k]        (M = 128 rows th, N = 16, K = 128)
+//   AH[th][2n] + i AH[th][2n+1] = A_n^(16 th)
+//   Q[tl][2n]  - i Q[tl][2n+1]  = 2 C_n B_n A_n^tl   (scaled by a power of two)
+// Both tables are split into fp16 high and remainder parts (three MMAs,
+// about 22 significant bits).  AH[th] = A^(16 th0) A^(128 g) A^(16 m) for
+// th = th0 + 8 g + m, each factor an exactly phase-reduced power or at most
+// 7 products of one.  One CTA owns up to kGUnits consecutive 2048-tap units
+// of one channel and builds Q once.
+static __device__ unsigned int g_gen_tc_timeouts;
+
+namespace {
+constexpr int kGThr = 256;
+constexpr int kGUnits = 4;
+constexpr int kGRows = 128, kGNC = 16, kGUnitTaps = kGRows * kGNC;
+constexpr uint32_t kGLbo = 144, kGSbo = 16 * 144;  // padded K-major, K = 128
+constexpr uint32_t kGTab = (kGRows / 8) * kGSbo;
+constexpr uint32_t kGQ = (kGNC / 8) * kGSbo;
+constexpr uint64_t kGWaitNs = 2000000000ull;
+struct GenSmem {
+  uint8_t ahh[kGTab];
+  uint8_t ahl[kGTab];
+  uint8_t qh[kGQ];
+  uint8_t ql[kGQ];
+  float red[kGThr / 32];
+  uint64_t mbar;
+  uint32_t tmem_base;
+};
+__device__ __forceinline__ uint32_t gsplit(float a, float b, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(a, b);
+  const float2 hf = __half22float2(h);
+  const __half2 l = __floats2half2_rn(a - hf.x, b - hf.y);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t goff(int r, int n) {  // K elements (2n, 2n+1) of row r
+  return (uint32_t)(r >> 3) * kGSbo + (uint32_t)(n >> 2) * kGLbo + (uint32_t)(r & 7) * 16u + (uint32_t)(n & 3) * 4u;
+}
+}  // namespace
+
+__global__ void __launch_bounds__(kGThr, 2) ssm_gen_tc_kernel(const float* __restrict__ dt,
+                                                              const float2* __restrict__ lam,
+                                                              const float2* __restrict__ Bp,
+                                                              const float2* __restrict__ Cp, int H, int N, int L,
+                                                              float* __restrict__ f) {
+  extern __shared__ __align__(1024) uint8_t gtsm[];
+  GenSmem& sm = *reinterpret_cast<GenSmem*>(gtsm);
+  const int h = blockIdx.y;
+  const int units = (L + kGUnitTaps - 1) / kGUnitTaps;
+  const int u0 = blockIdx.x * kGUnits, u1 = min(units, u0 + kGUnits);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int n = tid & 63, gq = tid >> 6;  // this thread's mode and row-group phase (0..3)
+  const float d = dt[h];
+  if (warp == 0) tc::tmem_alloc(&sm.tmem_base, 32);
+  if (tid == 0) {
+    tc::mbar_init(&sm.mbar, 1);
+    tc::fence_mbar_init();
+  }
+  float2 lm = make_float2(0.f, 0.f), w = make_float2(0.f, 0.f), m8[8], G[4];
+  if (n < N) {
+    lm = lam[(size_t)h * N + n];
+    const float2 cb = cmul(Cp[(size_t)h * N + n], Bp[(size_t)h * N + n]);
+    w = make_float2(2.f * cb.x, 2.f * cb.y);
+    const float2 a16 = ssm_pow(d, lm.x, lm.y, 16.0);
+    m8[0] = make_float2(1.f, 0.f);
+#pragma unroll
+    for (int m = 1; m < 8; ++m) m8[m] = cmul(m8[m - 1], a16);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) G[r] = ssm_pow(d, lm.x, lm.y, 128.0 * (gq + 4 * r));
+  } else {
+#pragma unroll
+    for (int m = 0; m < 8; ++m) m8[m] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) G[r] = make_float2(0.f, 0.f);
+  }
+  // power-of-two scale: the largest |Re|, |Im| of any 2 C B just below 2^13
+  float mx = fmaxf(fabsf(w.x), fabsf(w.y));
+  mx = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(mx)));
+  if ((tid & 31) == 0) sm.red[warp] = mx;
+  __syncthreads();
+  mx = 0.f;
+#pragma unroll
+  for (int i = 0; i < kGThr / 32; ++i) mx = fmaxf(mx, sm.red[i]);
+  float scale = 1.f, inv = 1.f;
+  if (mx > 0.f && mx <= 3.0e38f) {
+    int ex = 0;
+    (void)frexpf(mx, &ex);
+    scale = ldexpf(1.f, 13 - ex);
+    inv = ldexpf(1.f, ex - 13);
+  }
+  // Q rows tl = 4 gq .. 4 gq + 3
+  {
+    float2 p = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+    if (n < N) {
+      a1 = ssm_pow(d, lm.x, lm.y, 1.0);
+      p = cmul(make_float2(w.x * scale, w.y * scale), ssm_pow(d, lm.x, lm.y, 4.0 * gq));
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t lo;
+      const uint32_t hi = gsplit(p.x, -p.y, lo);
+      *reinterpret_cast<uint32_t*>(sm.qh + goff(4 * gq + j, n)) = hi;
+      *reinterpret_cast<uint32_t*>(sm.ql + goff(4 * gq + j, n)) = lo;
+      p = cmul(p, a1);
+    }
+  }
+  const uint32_t idesc = tc::idesc_f16(kGRows, kGNC, 0);
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+  const bool vec_ok = (L & 3) == 0;
+  uint32_t phase = 0;
+  bool failed = false;
+  for (int u = u0; u < u1; ++u) {
+    const int th0 = u * kGRows;
+    const int rows = min(kGRows, (L - th0 * kGNC + kGNC - 1) / kGNC);
+    const float2 base = n < N ? ssm_pow(d, lm.x, lm.y, 16.0 * th0) : make_float2(0.f, 0.f);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int g = gq + 4 * r;
+      if (8 * g >= rows) continue;  // rows past the end are never stored
+      const float2 pg = cmul(base, G[r]);
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const float2 v = cmul(pg, m8[m]);
+        uint32_t lo;
+        const uint32_t hi = gsplit(v.x, v.y, lo);
+        *reinterpret_cast<uint32_t*>(sm.ahh + goff(8 * g + m, n)) = hi;
+        *reinterpret_cast<uint32_t*>(sm.ahl + goff(8 * g + m, n)) = lo;
+      }
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = sm.tmem_base;
+    if (tid == 0) {
+      const uint32_t ah = tc::smem_u32(sm.ahh), al = tc::smem_u32(sm.ahl);
+      const uint32_t qh = tc::smem_u32(sm.qh), ql = tc::smem_u32(sm.ql);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        tc::mma_f16(tmem, tc::desc_kmajor(ah + kk * 2 * kGLbo, kGLbo, kGSbo),
+                    tc::desc_kmajor(qh + kk * 2 * kGLbo, kGLbo, kGSbo), idesc, kk > 0 ? 1u : 0u);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        tc::mma_f16(tmem, tc::desc_kmajor(ah + kk * 2 * kGLbo, kGLbo, kGSbo),
+                    tc::desc_kmajor(ql + kk * 2 * kGLbo, kGLbo, kGSbo), idesc, 1u);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        tc::mma_f16(tmem, tc::desc_kmajor(al + kk * 2 * kGLbo, kGLbo, kGSbo),
+                    tc::desc_kmajor(qh + kk * 2 * kGLbo, kGLbo, kGSbo), idesc, 1u);
+      tc::mma_commit(&sm.mbar);
+    }
+    const bool ok = tc::mbar_wait_bounded(&sm.mbar, phase, kGWaitNs);
+    phase ^= 1u;
+    if (__syncthreads_or(!ok)) {
+      failed = true;
+      break;
+    }
+    tc::fence_after_sync();
+    if (warp < 4) {
+      float v[16];
+      tc::tmem_ld16_wait(tmem + lane_off, v);
+      const int r = tid;  // TMEM lane = row
+      if (r < rows) {
+        const long long t0 = (long long)(th0 + r) * kGNC;
+        float* fp = f + (size_t)h * L + t0;
+        if (vec_ok && t0 + kGNC <= L) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            reinterpret_cast<float4*>(fp)[q] =
+                make_float4(v[4 * q] * inv, v[4 * q + 1] * inv, v[4 * q + 2] * inv, v[4 * q + 3] * inv);
+        } else {
+#pragma unroll
+          for (int j = 0; j < kGNC; ++j)
+            if (t0 + j < L) fp[j] = v[j] * inv;
+        }
+      }
+    }
+  }
+  if (failed && tid == 0) atomicAdd(&g_gen_tc_timeouts, 1u);
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(sm.tmem_base, 32);
+}
+
+unsigned int gen_tc_timeouts() {
+  unsigned int v = 0;
+  cudaMemcpyFromSymbol(&v, g_gen_tc_timeouts, sizeof(v));
+  return v;
+}
+
 cudaError_t launch_ssm_gen(const float* dt, const float* lam, const float* Bp, const float* Cp, int H, int N,
                            int L, float* f, cudaStream_t st) {
+  if (N <= 64) {
+    const int units = (L + kGUnitTaps - 1) / kGUnitTaps;
+    const size_t smem = sizeof(GenSmem) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(ssm_gen_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((units + kGUnits - 1) / kGUnits, H);
+    ssm_gen_tc_kernel<<<grid, kGThr, smem, st>>>(dt, reinterpret_cast<const float2*>(lam),
+                                                  reinterpret_cast<const float2*>(Bp),
+                                                  reinterpret_cast<const float2*>(Cp), H, N, L, f);
+    return cudaGetLastError();
+  }
+
   const int tiles = (L + kGenTile - 1) / kGenTile;
   cudaError_t e = cudaFuncSetAttribute(ssm_gen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGenSmem);
   if (e != cudaSuccess) return e;

@@ -53,6 +53,8 @@ def oracle_A(wl, hs=None):
     (6, 64, 8192, ("split", (-3.0, -2.9), (-1.1, -1.0))),
     (3, 64, 65536, ("loguniform", -3.0, -2.5)),         # long, slowly decaying: phase reduction
     (2, 1, 100, ("loguniform", -1.0, -1.0)),            # N = 1 (real A for n = 0)
+    (3, 64, 1001, ("loguniform", -3.0, -1.0)),          # L % 16 != 0: ragged last row, scalar stores
+    (2, 96, 3000, ("loguniform", -3.0, -1.0)),          # N > 64: CUDA-core generator
 ])
 def test_ssm_kernel_gen(H, N, L, dt):
     wl = W.make_conv(B=1, H=H, L=8, N=N, dtype="f32", seed=7, dt_range=dt)
