@@ -102,7 +102,7 @@ FC_API fc_status fftconv_fwd(const void* u, const float* f, const float* D, void
              "fftconv_fwd: L must be a power of two in [16, 8192] (got %d)", L);
   FC_REQUIRE((long long)B * 1 <= (1LL << 30), FC_EUNSUPPORTED, "B too large");
   if (fc::fftconv_tc_supported(L, dtype))
-    return cuda_status(fc::launch_fftconv_tc(u, f, D, y, B, H, L, dtype, (cudaStream_t)stream),
+    return cuda_status(fc::launch_fftconv_tc(u, f, D, y, B, H, L, dtype, false, (cudaStream_t)stream),
                        "fftconv_fwd (tensor cores) launch");
   const fc::SsmArgs none{nullptr, nullptr, nullptr, nullptr, 0};
   return cuda_status(fc::launch_fftconv(u, f, L, none, D, y, B, H, L, L, 1, dtype, (cudaStream_t)stream),
@@ -136,7 +136,7 @@ FC_API fc_status ssm_conv_fwd(const void* u, const float* dt, const float* lambd
   if (fc::fftconv_tc_supported(L, dtype)) {  // filter kernel, then the tensor-core convolution
     s = cuda_status(fc::launch_ssm_gen(dt, lambda, Bp, Cp, H, N, L, f, st), "ssm_conv_fwd: filter launch");
     if (s != FC_OK) return s;
-    return cuda_status(fc::launch_fftconv_tc(u, f, D, y, B, H, L, dtype, st),
+    return cuda_status(fc::launch_fftconv_tc(u, f, D, y, B, H, L, dtype, true, st),
                        "ssm_conv_fwd: tensor-core conv launch");
   }
   if (L >= 1024) {  // filter generated inside the convolution kernel

@@ -46,6 +46,15 @@ constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint32_t kCLbo = 128, kCSbo = (kN1 / 8) * 128;  // CA / CB K-major: 128 rows x 128 K
 constexpr uint32_t kCBytes = kN1 * kN1 * 2;
 constexpr uint32_t kXZBytes = kMaxPairs * kN2 * 2 * kN1 * 2;  // Z (the larger of X and Z): 2 x 128 x 64 x 2 B
+// fp32 filter staging inside the X/Z buffer, past the largest X (2 planes x 64 K-rows x 80 columns)
+constexpr uint32_t kFStage = 2 * 64 * (kMaxPairs + 1) * kN2 * 2;
+static_assert(kFStage + kL * 4 <= kXZBytes, "filter staging must fit in the X/Z buffer");
+
+__device__ __forceinline__ void cp_async16(uint32_t saddr, const void* g) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(g) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 struct TcSmem {
   uint8_t ca[kCBytes];
@@ -142,153 +151,191 @@ __global__ void __launch_bounds__(kThr, 2) fftconv_tc_kernel(const T* __restrict
   bool failed = false;
   float2 fh[kN2];
 
-  for (int h = blockIdx.x; h < H && !failed; h += gridDim.x) {
-    for (int p0 = 0; p0 < npairs && !failed; p0 += kMaxPairs) {
-      const bool with_filter = (p0 == 0);
-      const int P = min(kMaxPairs, npairs - p0);
-      const int NS = P + (with_filter ? 1 : 0);
-      const int NC = NS * kN2;                       // stage-A columns per real/imag half
-      const uint32_t lboX = (uint32_t)(NC / 8) * 128;  // X: MN-major, 64 K-rows (n1) x NC
-      const uint32_t xr = xz, xi = xz + 8 * lboX;
-      // ---- stage X: 16-byte chunks of 8 consecutive n2 at fixed (sequence, n1)
-      for (int idx = tid; idx < NS * 64 * 2; idx += kThr) {
-        const int half = idx & 1, n1 = (idx >> 1) & 63, s = idx >> 7;
-        const int n = s * kN2 + half * 8;
-        const uint32_t off = (uint32_t)(n >> 3) * 128 + (uint32_t)(n1 >> 3) * lboX + (uint32_t)(n1 & 7) * 16;
-        const int t = n1 * kN2 + half * 8;  // time index of the chunk's first element
-        uint4 re = make_uint4(0, 0, 0, 0), im = make_uint4(0, 0, 0, 0);
-        if (with_filter && s == 0) {
-          const float4* fp = reinterpret_cast<const float4*>(f + (size_t)h * kL + t);
-          float4 a = __ldg(fp);
-          const float4 b = __ldg(fp + 1);
-          if (t == 0) a.x += D[h];  // y = f * u + D u = (f + D delta) * u
-          re = make_uint4(Op<T>::pack(a.x, a.y), Op<T>::pack(a.z, a.w), Op<T>::pack(b.x, b.y),
-                          Op<T>::pack(b.z, b.w));
-        } else {
-          const int p = p0 + s - (with_filter ? 1 : 0);
-          const int b0 = 2 * p, b1 = 2 * p + 1;
-          re = *reinterpret_cast<const uint4*>(ub + ((size_t)b0 * H + h) * kL + t);
-          if (b1 < B) im = *reinterpret_cast<const uint4*>(ub + ((size_t)b1 * H + h) * kL + t);
-        }
-        *reinterpret_cast<uint4*>(sm.xz + off) = re;
-        *reinterpret_cast<uint4*>(sm.xz + 8 * lboX + off) = im;
+  // Work items of this CTA, in order: channels h = blockIdx.x, + gridDim.x, ...,
+  // each in batches of up to kMaxPairs row pairs (the first batch also carries
+  // the filter).  The next item's inputs are copied into the X/Z buffer with
+  // cp.async while the current item's epilogue runs.
+  int h = blockIdx.x, p0 = 0;
+  // u rows of item (h, p0) -> X planes (zero rows written directly)
+  auto issue_u = [&](int hh, int pp0) {
+    const bool wf = (pp0 == 0);
+    const int P = min(kMaxPairs, npairs - pp0);
+    const int NS = P + (wf ? 1 : 0);
+    const uint32_t lboX = (uint32_t)(NS * kN2 / 8) * 128;
+    for (int idx = tid; idx < P * 64 * 2; idx += kThr) {
+      const int half = idx & 1, n1 = (idx >> 1) & 63, pc = idx >> 7;
+      const int s = pc + (wf ? 1 : 0);
+      const int n = s * kN2 + half * 8;
+      const uint32_t off = (uint32_t)(n >> 3) * 128 + (uint32_t)(n1 >> 3) * lboX + (uint32_t)(n1 & 7) * 16;
+      const int t = n1 * kN2 + half * 8;
+      const int b0 = 2 * (pp0 + pc), b1 = b0 + 1;
+      cp_async16(xz + off, ub + ((size_t)b0 * H + hh) * kL + t);
+      if (b1 < B)
+        cp_async16(xz + 8 * lboX + off, ub + ((size_t)b1 * H + hh) * kL + t);
+      else
+        *reinterpret_cast<uint4*>(sm.xz + 8 * lboX + off) = make_uint4(0, 0, 0, 0);
+    }
+  };
+  // fp32 filter row of channel hh -> staging area past the X planes
+  auto issue_f = [&](int hh) {
+    for (int idx = tid; idx < kL / 4; idx += kThr)
+      cp_async16(xz + kFStage + idx * 16, f + (size_t)hh * kL + idx * 4);
+  };
+  if (h < H) issue_u(h, 0);
+  // the filter is written by the preceding kernel when launched as its
+  // programmatic dependent (no-op otherwise)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (h < H) issue_f(h);
+  cp_async_commit();
+
+  while (h < H && !failed) {
+    const bool with_filter = (p0 == 0);
+    const int P = min(kMaxPairs, npairs - p0);
+    const int NS = P + (with_filter ? 1 : 0);
+    const int NC = NS * kN2;                         // stage-A columns per real/imag half
+    const uint32_t lboX = (uint32_t)(NC / 8) * 128;  // X: MN-major, 64 K-rows (n1) x NC
+    const uint32_t xr = xz, xi = xz + 8 * lboX;
+    cp_async_wait_all();  // this thread's copies; the barrier makes everyone's visible
+    __syncthreads();
+    if (with_filter) {  // filter block: fp32 staging -> operand type, D folded into tap 0
+      for (int idx = tid; idx < 64 * 2; idx += kThr) {
+        const int half = idx & 1, n1 = idx >> 1;
+        const int t = n1 * kN2 + half * 8;
+        const uint32_t off = (uint32_t)half * 128 + (uint32_t)(n1 >> 3) * lboX + (uint32_t)(n1 & 7) * 16;
+        float4 a = *reinterpret_cast<const float4*>(sm.xz + kFStage + t * 4);
+        const float4 b = *reinterpret_cast<const float4*>(sm.xz + kFStage + t * 4 + 16);
+        if (t == 0) a.x += D[h];  // y = f * u + D u = (f + D delta) * u
+        *reinterpret_cast<uint4*>(sm.xz + off) = make_uint4(Op<T>::pack(a.x, a.y), Op<T>::pack(a.z, a.w),
+                                                            Op<T>::pack(b.x, b.y), Op<T>::pack(b.z, b.w));
+        *reinterpret_cast<uint4*>(sm.xz + 8 * lboX + off) = make_uint4(0, 0, 0, 0);
       }
-      tc::fence_smem_to_async();
-      tc::fence_before_sync();
-      __syncthreads();
-      tc::fence_after_sync();
-      // ---- stage A: D_re at TMEM columns [0, NC), D_im at [NC, 2 NC)
-      if (tid == 0) {
-        const uint32_t idA = tc::idesc_f16(128, NC, Op<T>::bf16, 0, 1);
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    // ---- stage A: D_re at TMEM columns [0, NC), D_im at [NC, 2 NC)
+    if (tid == 0) {
+      const uint32_t idA = tc::idesc_f16(128, NC, Op<T>::bf16, 0, 1);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          tc::mma_f16(tmem, tc::desc_kmajor(ca + kk * 256, kCLbo, kCSbo), tc::desc_kmajor(xr + kk * 2 * lboX, lboX, 128),
-                      idA, kk > 0 ? 1u : 0u);
+      for (int kk = 0; kk < 4; ++kk)
+        tc::mma_f16(tmem, tc::desc_kmajor(ca + kk * 256, kCLbo, kCSbo), tc::desc_kmajor(xr + kk * 2 * lboX, lboX, 128),
+                    idA, kk > 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          tc::mma_f16(tmem, tc::desc_kmajor(ca + (4 + kk) * 256, kCLbo, kCSbo),
-                      tc::desc_kmajor(xi + kk * 2 * lboX, lboX, 128), idA, 1u);
+      for (int kk = 0; kk < 4; ++kk)
+        tc::mma_f16(tmem, tc::desc_kmajor(ca + (4 + kk) * 256, kCLbo, kCSbo),
+                    tc::desc_kmajor(xi + kk * 2 * lboX, lboX, 128), idA, 1u);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          tc::mma_f16(tmem + NC, tc::desc_kmajor(ca + kk * 256, kCLbo, kCSbo),
-                      tc::desc_kmajor(xi + kk * 2 * lboX, lboX, 128), idA, kk > 0 ? 1u : 0u);
+      for (int kk = 0; kk < 4; ++kk)
+        tc::mma_f16(tmem + NC, tc::desc_kmajor(ca + kk * 256, kCLbo, kCSbo),
+                    tc::desc_kmajor(xi + kk * 2 * lboX, lboX, 128), idA, kk > 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          tc::mma_f16(tmem + NC, tc::desc_kmajor(cb + kk * 256, kCLbo, kCSbo),
-                      tc::desc_kmajor(xr + kk * 2 * lboX, lboX, 128), idA, 1u);
-        tc::mma_commit(&sm.mbar);
-      }
-      bool ok = tc::mbar_wait_bounded(&sm.mbar, phase, kWaitNs);
-      phase ^= 1u;
-      if (__syncthreads_or(!ok)) {
-        failed = true;
-        break;
-      }
-      tc::fence_after_sync();
-      // ---- register stage: twiddle, DFT-16, x filter spectrum, IDFT-16, twiddle
-      const uint32_t lboZ = (uint32_t)(P * kN2 / 8) * 128;  // Z: MN-major, 256 K-rows (re k1 | im k1) x P*16
+      for (int kk = 0; kk < 4; ++kk)
+        tc::mma_f16(tmem + NC, tc::desc_kmajor(cb + kk * 256, kCLbo, kCSbo),
+                    tc::desc_kmajor(xr + kk * 2 * lboX, lboX, 128), idA, 1u);
+      tc::mma_commit(&sm.mbar);
+    }
+    bool ok = tc::mbar_wait_bounded(&sm.mbar, phase, kWaitNs);
+    phase ^= 1u;
+    if (__syncthreads_or(!ok)) {
+      failed = true;
+      break;
+    }
+    tc::fence_after_sync();
+    // ---- register stage: twiddle, DFT-16, x filter spectrum, IDFT-16, twiddle
+    const uint32_t lboZ = (uint32_t)(P * kN2 / 8) * 128;  // Z: MN-major, 256 K-rows (re k1 | im k1) x P*16
 #pragma unroll 1
-      for (int s = 0; s < NS; ++s) {
-        const bool is_filter = with_filter && s == 0;
-        if (!is_filter && ((s - (with_filter ? 1 : 0)) & 1) != grp) continue;  // pairs alternate between groups
-        float yr[16], yi[16];
-        tc::tmem_ld16x2_wait(tmem + lane_off + (uint32_t)(s * kN2), tmem + lane_off + (uint32_t)(NC + s * kN2), yr, yi);
-        float2 v[kN2];
+    for (int s = 0; s < NS; ++s) {
+      const bool is_filter = with_filter && s == 0;
+      if (!is_filter && ((s - (with_filter ? 1 : 0)) & 1) != grp) continue;  // pairs alternate between groups
+      float yr[16], yi[16];
+      tc::tmem_ld16x2_wait(tmem + lane_off + (uint32_t)(s * kN2), tmem + lane_off + (uint32_t)(NC + s * kN2), yr, yi);
+      float2 v[kN2];
 #pragma unroll
-        for (int n2 = 0; n2 < kN2; ++n2) v[n2] = cmul(make_float2(yr[n2], yi[n2]), tw[n2]);
-        dft<kN2, -1>(v);
-        if (is_filter) {
-          constexpr float inv_m = 1.0f / (float)kM;
+      for (int n2 = 0; n2 < kN2; ++n2) v[n2] = cmul(make_float2(yr[n2], yi[n2]), tw[n2]);
+      dft<kN2, -1>(v);
+      if (is_filter) {
+        constexpr float inv_m = 1.0f / (float)kM;
 #pragma unroll
-          for (int k2 = 0; k2 < kN2; ++k2) fh[k2] = make_float2(v[k2].x * inv_m, v[k2].y * inv_m);
-          continue;
-        }
-#pragma unroll
-        for (int k2 = 0; k2 < kN2; ++k2) v[k2] = cmul(v[k2], fh[k2]);
-        dft<kN2, +1>(v);
-#pragma unroll
-        for (int n2 = 0; n2 < kN2; ++n2) v[n2] = cmul(v[n2], cconj(tw[n2]));
-        const int pc = s - (with_filter ? 1 : 0);  // pair column block
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int n = pc * kN2 + half * 8;
-          const uint32_t offr = (uint32_t)(n >> 3) * 128 + (uint32_t)(row >> 3) * lboZ + (uint32_t)(row & 7) * 16;
-          const uint32_t offi = offr + 16 * lboZ;  // K rows 128 + k1
-          const float2* w = v + half * 8;
-          *reinterpret_cast<uint4*>(sm.xz + offr) =
-              make_uint4(Op<T>::pack(w[0].x, w[1].x), Op<T>::pack(w[2].x, w[3].x), Op<T>::pack(w[4].x, w[5].x),
-                         Op<T>::pack(w[6].x, w[7].x));
-          *reinterpret_cast<uint4*>(sm.xz + offi) =
-              make_uint4(Op<T>::pack(w[0].y, w[1].y), Op<T>::pack(w[2].y, w[3].y), Op<T>::pack(w[4].y, w[5].y),
-                         Op<T>::pack(w[6].y, w[7].y));
-        }
+        for (int k2 = 0; k2 < kN2; ++k2) fh[k2] = make_float2(v[k2].x * inv_m, v[k2].y * inv_m);
+        continue;
       }
-      tc::fence_smem_to_async();
-      tc::fence_before_sync();
-      __syncthreads();
-      tc::fence_after_sync();
-      // ---- stage A': y = CA^T Zr + CB^T Zi into TMEM columns [0, P*16)
-      if (tid == 0) {
-        const uint32_t idB = tc::idesc_f16(128, P * kN2, Op<T>::bf16, 1, 1);
-        const uint32_t zr = xz, zi = xz + 16 * lboZ;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          tc::mma_f16(tmem, tc::desc_kmajor(ca + kk * 2 * kCSbo, kCSbo, kCLbo),
-                      tc::desc_kmajor(zr + kk * 2 * lboZ, lboZ, 128), idB, kk > 0 ? 1u : 0u);
+      for (int k2 = 0; k2 < kN2; ++k2) v[k2] = cmul(v[k2], fh[k2]);
+      dft<kN2, +1>(v);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          tc::mma_f16(tmem, tc::desc_kmajor(cb + kk * 2 * kCSbo, kCSbo, kCLbo),
-                      tc::desc_kmajor(zi + kk * 2 * lboZ, lboZ, 128), idB, 1u);
-        tc::mma_commit(&sm.mbar);
+      for (int n2 = 0; n2 < kN2; ++n2) v[n2] = cmul(v[n2], cconj(tw[n2]));
+      const int pc = s - (with_filter ? 1 : 0);  // pair column block
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int n = pc * kN2 + half * 8;
+        const uint32_t offr = (uint32_t)(n >> 3) * 128 + (uint32_t)(row >> 3) * lboZ + (uint32_t)(row & 7) * 16;
+        const uint32_t offi = offr + 16 * lboZ;  // K rows 128 + k1
+        const float2* w = v + half * 8;
+        *reinterpret_cast<uint4*>(sm.xz + offr) =
+            make_uint4(Op<T>::pack(w[0].x, w[1].x), Op<T>::pack(w[2].x, w[3].x), Op<T>::pack(w[4].x, w[5].x),
+                       Op<T>::pack(w[6].x, w[7].x));
+        *reinterpret_cast<uint4*>(sm.xz + offi) =
+            make_uint4(Op<T>::pack(w[0].y, w[1].y), Op<T>::pack(w[2].y, w[3].y), Op<T>::pack(w[4].y, w[5].y),
+                       Op<T>::pack(w[6].y, w[7].y));
       }
-      ok = tc::mbar_wait_bounded(&sm.mbar, phase, kWaitNs);
-      phase ^= 1u;
-      if (__syncthreads_or(!ok)) {
-        failed = true;
-        break;
-      }
-      tc::fence_after_sync();
-      // ---- epilogue: lane j -> (part c = j / 64, n1 = j % 64); the D u term rode
-      // through the transform with the filter (its tap 0 carries D)
-      const int c = row >> 6, n1 = row & 63;
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    // ---- stage A': y = CA^T Zr + CB^T Zi into TMEM columns [0, P*16)
+    if (tid == 0) {
+      const uint32_t idB = tc::idesc_f16(128, P * kN2, Op<T>::bf16, 1, 1);
+      const uint32_t zr = xz, zi = xz + 16 * lboZ;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        tc::mma_f16(tmem, tc::desc_kmajor(ca + kk * 2 * kCSbo, kCSbo, kCLbo),
+                    tc::desc_kmajor(zr + kk * 2 * lboZ, lboZ, 128), idB, kk > 0 ? 1u : 0u);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        tc::mma_f16(tmem, tc::desc_kmajor(cb + kk * 2 * kCSbo, kCSbo, kCLbo),
+                    tc::desc_kmajor(zi + kk * 2 * lboZ, lboZ, 128), idB, 1u);
+      tc::mma_commit(&sm.mbar);
+    }
+    ok = tc::mbar_wait_bounded(&sm.mbar, phase, kWaitNs);
+    phase ^= 1u;
+    if (__syncthreads_or(!ok)) {
+      failed = true;
+      break;
+    }
+    tc::fence_after_sync();
+    // ---- the X/Z buffer is free: start copying the next item's inputs
+    const int h_cur = h, p0_cur = p0;
+    p0 += kMaxPairs;
+    if (p0 >= npairs) {
+      p0 = 0;
+      h += gridDim.x;
+    }
+    if (h < H) {
+      issue_u(h, p0);
+      if (p0 == 0) issue_f(h);
+    }
+    cp_async_commit();
+    // ---- epilogue: lane j -> (part c = j / 64, n1 = j % 64); the D u term rode
+    // through the transform with the filter (its tap 0 carries D)
+    const int c = row >> 6, n1 = row & 63;
 #pragma unroll 1
-      for (int p = grp; p < P; p += 2) {
-        float yv[16];
-        tc::tmem_ld16_wait(tmem + lane_off + (uint32_t)(p * kN2), yv);
-        const int brow = 2 * (p0 + p) + c;
-        if (brow < B) {
-          const size_t rbase = ((size_t)brow * H + h) * kL + (size_t)n1 * kN2;
-          uint32_t ow[8];
+    for (int p = grp; p < P; p += 2) {
+      float yv[16];
+      tc::tmem_ld16_wait(tmem + lane_off + (uint32_t)(p * kN2), yv);
+      const int brow = 2 * (p0_cur + p) + c;
+      if (brow < B) {
+        const size_t rbase = ((size_t)brow * H + h_cur) * kL + (size_t)n1 * kN2;
+        uint32_t ow[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) ow[i] = Op<T>::pack(yv[2 * i], yv[2 * i + 1]);
-          *reinterpret_cast<uint4*>(yb + rbase) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-          *reinterpret_cast<uint4*>(yb + rbase + 8) = make_uint4(ow[4], ow[5], ow[6], ow[7]);
-        }
+        for (int i = 0; i < 8; ++i) ow[i] = Op<T>::pack(yv[2 * i], yv[2 * i + 1]);
+        *reinterpret_cast<uint4*>(yb + rbase) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+        *reinterpret_cast<uint4*>(yb + rbase + 8) = make_uint4(ow[4], ow[5], ow[6], ow[7]);
       }
-      tc::fence_before_sync();
-      __syncthreads();
     }
   }
+  cp_async_wait_all();
   if (failed && tid == 0) atomicAdd(&g_fftconv_tc_timeouts, 1u);
   tc::fence_before_sync();
   __syncthreads();
@@ -296,7 +343,7 @@ __global__ void __launch_bounds__(kThr, 2) fftconv_tc_kernel(const T* __restrict
 }
 
 template <typename T>
-static cudaError_t fftconv_tc_t(const void* u, const float* f, const float* D, void* y, int B, int H,
+static cudaError_t fftconv_tc_t(const void* u, const float* f, const float* D, void* y, int B, int H, bool pdl,
                                 cudaStream_t st) {
   auto kern = fftconv_tc_kernel<T>;
   const size_t smem = sizeof(TcSmem) + 1024;
@@ -310,16 +357,26 @@ static cudaError_t fftconv_tc_t(const void* u, const float* f, const float* D, v
     if (e != cudaSuccess) return e;
   }
   const int grid = H < 2 * num_sms ? H : 2 * num_sms;
-  kern<<<grid, kThr, smem, st>>>((const T*)u, f, D, (T*)y, B, H);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThr);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, (const T*)u, f, D, (T*)y, B, H);
 }
 
 bool fftconv_tc_supported(int L, int dtype) { return L == kL && (dtype == 1 || dtype == 2); }
 
 cudaError_t launch_fftconv_tc(const void* u, const float* f, const float* D, void* y, int B, int H, int L, int dtype,
-                              cudaStream_t st) {
+                              bool after_filter_kernel, cudaStream_t st) {
   if (!fftconv_tc_supported(L, dtype)) return cudaErrorInvalidValue;
-  return dtype == 1 ? fftconv_tc_t<__half>(u, f, D, y, B, H, st) : fftconv_tc_t<__nv_bfloat16>(u, f, D, y, B, H, st);
+  return dtype == 1 ? fftconv_tc_t<__half>(u, f, D, y, B, H, after_filter_kernel, st)
+                    : fftconv_tc_t<__nv_bfloat16>(u, f, D, y, B, H, after_filter_kernel, st);
 }
 
 unsigned int fftconv_tc_timeouts() {

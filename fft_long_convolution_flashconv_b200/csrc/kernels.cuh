@@ -55,8 +55,12 @@ unsigned int mixer_tc_timeouts();
 
 // Tensor-core fused FFT convolution (block-FFT stages as tcgen05 GEMMs).
 bool fftconv_tc_supported(int L, int dtype);
+// after_filter_kernel: f is written by the kernel launched just before on the
+// same stream (ssm_gen), which lets this launch start as its programmatic
+// dependent (prologue overlapped; the filter is read only after that kernel
+// has completed).
 cudaError_t launch_fftconv_tc(const void* u, const float* f, const float* D, void* y, int B, int H, int L, int dtype,
-                              cudaStream_t st);
+                              bool after_filter_kernel, cudaStream_t st);
 unsigned int fftconv_tc_timeouts();
 // Tensor-core filter generation CTAs that gave up waiting for an MMA.
 unsigned int gen_tc_timeouts();

@@ -28,6 +28,7 @@ __global__ void __launch_bounds__(kGenThreads) ssm_gen_kernel(const float* __res
                                                              const float2* __restrict__ Bp,
                                                              const float2* __restrict__ Cp, int H, int N,
                                                              int L, float* __restrict__ f) {
+  asm volatile("griddepcontrol.launch_dependents;");  // see ssm_gen_tc_kernel
   extern __shared__ __align__(16) float2 gsm[];
   float2* Q = gsm;                       // [m][64]
   float2* Wt = Q + kGenMB * 64;          // [kh][kGenMB] as written by ssm_fill_tables
@@ -91,14 +92,18 @@ constexpr uint32_t kGLbo = 144, kGSbo = 16 * 144;  // padded K-major, K = 128
 constexpr uint32_t kGTab = (kGRows / 8) * kGSbo;
 constexpr uint32_t kGQ = (kGNC / 8) * kGSbo;
 constexpr uint64_t kGWaitNs = 2000000000ull;
-struct GenSmem {
-  uint8_t ahh[kGTab];
-  uint8_t ahl[kGTab];
-  uint8_t qh[kGQ];
-  uint8_t ql[kGQ];
-  float red[kGThr / 32];
-  uint64_t mbar;
-  uint32_t tmem_base;
+// Shared-memory layout (byte offsets).  With at most 64 rows (L <= 1024,
+// SHORT) the rows 64..127 that the M = 128 MMA reads past each AH tile are
+// never stored, so those reads may land on the next tile: the tiles then take
+// 18 KB each instead of 36 KB and four CTAs fit on an SM.  The control words
+// sit past every byte an MMA reads.
+template <bool SHORT>
+struct GenLayout {
+  static constexpr uint32_t tab = SHORT ? kGTab / 2 : kGTab;
+  static constexpr uint32_t ahh = 0, ahl = tab, qh = 2 * tab, ql = qh + kGQ;
+  static constexpr uint32_t mma_end = (ahl + kGTab > ql + kGQ) ? ahl + kGTab : ql + kGQ;
+  static constexpr uint32_t red = (mma_end + 15u) & ~15u, mbar = red + 32, tmem = mbar + 8;
+  static constexpr uint32_t bytes = tmem + 8;
 };
 __device__ __forceinline__ uint32_t gsplit(float a, float b, uint32_t& lo) {
   const __half2 h = __floats2half2_rn(a, b);
@@ -112,25 +117,40 @@ __device__ __forceinline__ uint32_t goff(int r, int n) {  // K elements (2n, 2n+
 }
 }  // namespace
 
-__global__ void __launch_bounds__(kGThr, 2) ssm_gen_tc_kernel(const float* __restrict__ dt,
-                                                              const float2* __restrict__ lam,
-                                                              const float2* __restrict__ Bp,
-                                                              const float2* __restrict__ Cp, int H, int N, int L,
-                                                              float* __restrict__ f) {
+template <bool SHORT>
+__global__ void __launch_bounds__(kGThr, SHORT ? 4 : 2) ssm_gen_tc_kernel(const float* __restrict__ dt,
+                                                                          const float2* __restrict__ lam,
+                                                                          const float2* __restrict__ Bp,
+                                                                          const float2* __restrict__ Cp, int H, int N,
+                                                                          int L, float* __restrict__ f) {
+  // a convolution launched as this kernel's programmatic dependent may start
+  // its prologue now; it reads f only after this grid has completed
+  asm volatile("griddepcontrol.launch_dependents;");
+  using LY = GenLayout<SHORT>;
+  constexpr int NG = SHORT ? 2 : 4;  // row groups g = gq + 4 r this thread may fill
   extern __shared__ __align__(1024) uint8_t gtsm[];
-  GenSmem& sm = *reinterpret_cast<GenSmem*>(gtsm);
+  struct {
+    uint8_t* ahh;
+    uint8_t* ahl;
+    uint8_t* qh;
+    uint8_t* ql;
+    float* red;
+    uint64_t* mbar;
+    uint32_t* tmem_p;
+  } sm{gtsm + LY::ahh, gtsm + LY::ahl, gtsm + LY::qh, gtsm + LY::ql, reinterpret_cast<float*>(gtsm + LY::red),
+       reinterpret_cast<uint64_t*>(gtsm + LY::mbar), reinterpret_cast<uint32_t*>(gtsm + LY::tmem)};
   const int h = blockIdx.y;
   const int units = (L + kGUnitTaps - 1) / kGUnitTaps;
   const int u0 = blockIdx.x * kGUnits, u1 = min(units, u0 + kGUnits);
   const int tid = threadIdx.x, warp = tid >> 5;
   const int n = tid & 63, gq = tid >> 6;  // this thread's mode and row-group phase (0..3)
   const float d = dt[h];
-  if (warp == 0) tc::tmem_alloc(&sm.tmem_base, 32);
+  if (warp == 0) tc::tmem_alloc(sm.tmem_p, 32);
   if (tid == 0) {
-    tc::mbar_init(&sm.mbar, 1);
+    tc::mbar_init(sm.mbar, 1);
     tc::fence_mbar_init();
   }
-  float2 lm = make_float2(0.f, 0.f), w = make_float2(0.f, 0.f), m8[8], G[4];
+  float2 lm = make_float2(0.f, 0.f), w = make_float2(0.f, 0.f), m8[8], G[NG];
   if (n < N) {
     lm = lam[(size_t)h * N + n];
     const float2 cb = cmul(Cp[(size_t)h * N + n], Bp[(size_t)h * N + n]);
@@ -140,12 +160,12 @@ __global__ void __launch_bounds__(kGThr, 2) ssm_gen_tc_kernel(const float* __res
 #pragma unroll
     for (int m = 1; m < 8; ++m) m8[m] = cmul(m8[m - 1], a16);
 #pragma unroll
-    for (int r = 0; r < 4; ++r) G[r] = ssm_pow(d, lm.x, lm.y, 128.0 * (gq + 4 * r));
+    for (int r = 0; r < NG; ++r) G[r] = ssm_pow(d, lm.x, lm.y, 128.0 * (gq + 4 * r));
   } else {
 #pragma unroll
     for (int m = 0; m < 8; ++m) m8[m] = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int r = 0; r < 4; ++r) G[r] = make_float2(0.f, 0.f);
+    for (int r = 0; r < NG; ++r) G[r] = make_float2(0.f, 0.f);
   }
   // power-of-two scale: the largest |Re|, |Im| of any 2 C B just below 2^13
   float mx = fmaxf(fabsf(w.x), fabsf(w.y));
@@ -188,7 +208,7 @@ __global__ void __launch_bounds__(kGThr, 2) ssm_gen_tc_kernel(const float* __res
     const int rows = min(kGRows, (L - th0 * kGNC + kGNC - 1) / kGNC);
     const float2 base = n < N ? ssm_pow(d, lm.x, lm.y, 16.0 * th0) : make_float2(0.f, 0.f);
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
+    for (int r = 0; r < NG; ++r) {
       const int g = gq + 4 * r;
       if (8 * g >= rows) continue;  // rows past the end are never stored
       const float2 pg = cmul(base, G[r]);
@@ -205,7 +225,7 @@ __global__ void __launch_bounds__(kGThr, 2) ssm_gen_tc_kernel(const float* __res
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    const uint32_t tmem = sm.tmem_base;
+    const uint32_t tmem = *sm.tmem_p;
     if (tid == 0) {
       const uint32_t ah = tc::smem_u32(sm.ahh), al = tc::smem_u32(sm.ahl);
       const uint32_t qh = tc::smem_u32(sm.qh), ql = tc::smem_u32(sm.ql);
@@ -221,9 +241,9 @@ __global__ void __launch_bounds__(kGThr, 2) ssm_gen_tc_kernel(const float* __res
       for (int kk = 0; kk < 8; ++kk)
         tc::mma_f16(tmem, tc::desc_kmajor(al + kk * 2 * kGLbo, kGLbo, kGSbo),
                     tc::desc_kmajor(qh + kk * 2 * kGLbo, kGLbo, kGSbo), idesc, 1u);
-      tc::mma_commit(&sm.mbar);
+      tc::mma_commit(sm.mbar);
     }
-    const bool ok = tc::mbar_wait_bounded(&sm.mbar, phase, kGWaitNs);
+    const bool ok = tc::mbar_wait_bounded(sm.mbar, phase, kGWaitNs);
     phase ^= 1u;
     if (__syncthreads_or(!ok)) {
       failed = true;
@@ -253,7 +273,7 @@ __global__ void __launch_bounds__(kGThr, 2) ssm_gen_tc_kernel(const float* __res
   if (failed && tid == 0) atomicAdd(&g_gen_tc_timeouts, 1u);
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 0) tc::tmem_dealloc(sm.tmem_base, 32);
+  if (warp == 0) tc::tmem_dealloc(*sm.tmem_p, 32);
 }
 
 unsigned int gen_tc_timeouts() {
@@ -266,13 +286,14 @@ cudaError_t launch_ssm_gen(const float* dt, const float* lam, const float* Bp, c
                            int L, float* f, cudaStream_t st) {
   if (N <= 64) {
     const int units = (L + kGUnitTaps - 1) / kGUnitTaps;
-    const size_t smem = sizeof(GenSmem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(ssm_gen_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const bool short_rows = L <= kGUnitTaps / 2;
+    auto kern = short_rows ? ssm_gen_tc_kernel<true> : ssm_gen_tc_kernel<false>;
+    const size_t smem = short_rows ? GenLayout<true>::bytes : GenLayout<false>::bytes;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((units + kGUnits - 1) / kGUnits, H);
-    ssm_gen_tc_kernel<<<grid, kGThr, smem, st>>>(dt, reinterpret_cast<const float2*>(lam),
-                                                  reinterpret_cast<const float2*>(Bp),
-                                                  reinterpret_cast<const float2*>(Cp), H, N, L, f);
+    kern<<<grid, kGThr, smem, st>>>(dt, reinterpret_cast<const float2*>(lam), reinterpret_cast<const float2*>(Bp),
+                                    reinterpret_cast<const float2*>(Cp), H, N, L, f);
     return cudaGetLastError();
   }
 
