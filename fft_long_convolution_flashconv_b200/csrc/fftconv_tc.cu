@@ -6,13 +6,17 @@
 // multiplies so that it runs on the tensor cores (H3 blog, "Fused Block
 // FFTConv").  Index split n = 16 n1 + n2, k = k1 + 128 k2 (n1, k1 < 128,
 // n2, k2 < 16), w_K = exp(-2 pi i / K):
-//   stage A   (GEMM)      Y[k1,n2]  = sum_{n1<64} w_128^(n1 k1) x[16 n1 + n2]
-//                                     (n1 >= 64 is the zero padding)
-//   registers             Y'        = Y w_2048^(k1 n2);  X^[k1+128k2] = DFT16_n2(Y')
-//                         Z^        = X^ . F^ / M;       Z = IDFT16_k2(Z^) w_2048^(-k1 n2)
-//   stage A'  (GEMM)      y[16 n1 + n2] = sum_{k1} w_128^(-n1 k1) Z[k1, n2],  n1 < 64
-// Complex products are split into real GEMMs with fp32 accumulation in TMEM.
-// Two constant 128x128 matrices hold the real DFT-128 blocks,
+//   stage A   (GEMM)  Y[k1,n2]  = sum_{n1<64} w_128^(n1 k1) x[16 n1 + n2]   (n1 >= 64: zero padding)
+//   registers         Y'        = Y w_2048^(k1 n2) / 32                      (fp16 tile, K = re|im n2)
+//   stage B   (GEMM)  X^[k1,k2] = sum_n2 w_16^(n2 k2) Y'[k1,n2]              (32 x 32 real DFT-16 block)
+//   registers         V         = X^ . 32 F^ / M                             (fp16 tile, K = re|im k2)
+//   stage B'  (GEMM)  W[k1,n2]  = sum_k2 w_16^(-n2 k2) V[k1,k2]
+//   registers         Z         = W w_2048^(-k1 n2)
+//   stage A'  (GEMM)  y[16 n1 + n2] = sum_{k1} w_128^(-n1 k1) Z[k1, n2],      n1 < 64
+// (X^[k1 + 128 k2] is the 2048-point transform; F^ that of the filter, which
+// goes through stages A and B as one more sequence.)  Complex products are
+// split into real GEMMs with fp32 accumulation in TMEM.  Two constant 128x128
+// matrices hold the real DFT-128 blocks,
 //   CA[k1][j] = j<64 ?  cos(2 pi k1 j/128) : sin(2 pi k1 (j-64)/128)
 //   CB[k1][j] = j<64 ? -sin(2 pi k1 j/128) : cos(2 pi k1 (j-64)/128)
 // read K-major by stage A and (the DFT matrix being symmetric) MN-major by
@@ -20,15 +24,19 @@
 //   stage A : Yr = CA[:, :64] Xr + CA[:, 64:] Xi,   Yi = CA[:, :64] Xi + CB[:, :64] Xr
 //   stage A': rows j<64 give Re y[n1=j], rows j>=64 give Im y[n1=j-64]:
 //             y = CA^T Zr + CB^T Zi
+// and two 32x32 fp16 blocks the forward and inverse DFT-16 (stages B, B').
+// Stage-B operands are always fp16 (scaled by 1/32 so that |Y'| <= 2 max|u|);
+// stages A and A' use the I/O type.
 // One CTA takes one channel at a time: its filter and up to 4 row pairs (two
 // real rows packed as one complex sequence u0 + i u1; f is real, so the real
 // and imaginary outputs are the two convolutions) form one batch of
-// N = 16 x (1 + pairs) GEMM columns.  The CTA has two groups of four warps
+// N = 16 x (1 + pairs) stage-A columns.  The CTA has two groups of four warps
 // (each group covers the four TMEM lane quarters, thread row k1 = tid % 128);
-// both groups transform the filter column (cheap) and keep its 16 bins per
-// row in registers for the whole channel, then split the row pairs.  Waits on
-// MMA completion are bounded; a CTA that gives up records it in a device
-// counter, skips its remaining work and frees its TMEM.
+// the register passes alternate sequences between the groups, and every
+// thread keeps its row's 16 filter bins in registers for the whole channel.
+// The next work item's inputs are copied in with cp.async during the
+// epilogue.  Waits on MMA completion are bounded; a CTA that gives up records
+// it in a device counter, skips its remaining work and frees its TMEM.
 #include "fft_stockham.cuh"
 #include "kernels.cuh"
 #include "tc100.cuh"
@@ -45,7 +53,11 @@ constexpr uint32_t kTmemCols = 256;
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint32_t kCLbo = 128, kCSbo = (kN1 / 8) * 128;  // CA / CB K-major: 128 rows x 128 K
 constexpr uint32_t kCBytes = kN1 * kN1 * 2;
-constexpr uint32_t kXZBytes = kMaxPairs * kN2 * 2 * kN1 * 2;  // Z (the larger of X and Z): 2 x 128 x 64 x 2 B
+// Stage-B tiles: per sequence a K-major 128 (k1) x 32 (re n2 | im n2) fp16 tile
+constexpr uint32_t kYLbo = 128, kYSbo = 4 * 128, kYTile = kN1 * 32 * 2;
+// X (stage A input), the stage-B tiles, then Z (stage A' input) share one buffer
+constexpr uint32_t kXZBytes = (kMaxPairs + 1) * kYTile;
+static_assert(kXZBytes >= kMaxPairs * kN2 * 2 * kN1 * 2, "Z must fit");
 // fp32 filter staging inside the X/Z buffer, past the largest X (2 planes x 64 K-rows x 80 columns)
 constexpr uint32_t kFStage = 2 * 64 * (kMaxPairs + 1) * kN2 * 2;
 static_assert(kFStage + kL * 4 <= kXZBytes, "filter staging must fit in the X/Z buffer");
@@ -59,7 +71,9 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 struct TcSmem {
   uint8_t ca[kCBytes];
   uint8_t cb[kCBytes];
-  uint8_t xz[kXZBytes];   // stage-A input X, later the stage-A' input Z
+  uint8_t xz[kXZBytes];   // stage-A input X, then the stage-B tiles, then the stage-A' input Z
+  uint8_t wf[32 * 32 * 2];  // DFT-16 as a real 32 x 32 block (B operand, rows = output re/im k2)
+  uint8_t wi[32 * 32 * 2];  // inverse DFT-16
   float2 costab[kN1];
   uint64_t mbar;
   uint32_t tmem_base;
@@ -131,13 +145,36 @@ __global__ void __launch_bounds__(kThr, 2) fftconv_tc_kernel(const T* __restrict
     *reinterpret_cast<uint4*>(sm.cb + off) =
         make_uint4(Op<T>::pack(b[0], b[1]), Op<T>::pack(b[2], b[3]), Op<T>::pack(b[4], b[5]), Op<T>::pack(b[6], b[7]));
   }
-  // this thread's stage twiddles w_2048^(k1 n2), k1 = row
-  float2 tw[kN2];
+  // DFT-16 blocks (fp16, K-major 32 x 32): row c = output (k2 = c % 16, imaginary part if c >= 16),
+  // column j = input (n2 = j % 16, imaginary part if j >= 16); angle 2 pi n2 k2 / 16
+  for (int idx = tid; idx < 32 * 4; idx += kThr) {
+    const int c = idx >> 2, j0 = (idx & 3) * 8;
+    float a[8], b[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int j = j0 + i;
+      const float2 cs = sm.costab[(8 * (j & 15) * (c & 15)) & 127];
+      const bool oim = c >= 16, iim = j >= 16;
+      // forward (e^{-i theta}): Re += xr cos + xi sin, Im += xi cos - xr sin; inverse flips sin
+      const float fw = (oim == iim) ? cs.x : (iim ? cs.y : -cs.y);
+      a[i] = fw;
+      b[i] = (oim == iim) ? cs.x : -fw;
+    }
+    const uint32_t off = (uint32_t)(c >> 3) * kYSbo + (uint32_t)(j0 >> 3) * kYLbo + (uint32_t)(c & 7) * 16;
+    *reinterpret_cast<uint4*>(sm.wf + off) = make_uint4(Op<__half>::pack(a[0], a[1]), Op<__half>::pack(a[2], a[3]),
+                                                        Op<__half>::pack(a[4], a[5]), Op<__half>::pack(a[6], a[7]));
+    *reinterpret_cast<uint4*>(sm.wi + off) = make_uint4(Op<__half>::pack(b[0], b[1]), Op<__half>::pack(b[2], b[3]),
+                                                        Op<__half>::pack(b[4], b[5]), Op<__half>::pack(b[6], b[7]));
+  }
+  // this thread's stage twiddles w_2048^(k1 n2) / 32, k1 = row: the 1/32 keeps the
+  // fp16 stage-B tile at |Y| / 32 <= 2 max|u|; the filter bins carry the factor 32
+  // back, and the inverse twiddle is 32 conj(tws).
+  float2 tws[kN2];
 #pragma unroll
   for (int n2 = 0; n2 < kN2; ++n2) {
     float s, c;
     sincospif(-2.0f * (float)(row * n2) / (float)kM, &s, &c);
-    tw[n2] = make_float2(c, s);
+    tws[n2] = make_float2(c * (1.f / 32.f), s * (1.f / 32.f));
   }
   tc::fence_smem_to_async();
   tc::fence_before_sync();
@@ -242,33 +279,114 @@ __global__ void __launch_bounds__(kThr, 2) fftconv_tc_kernel(const T* __restrict
       break;
     }
     tc::fence_after_sync();
-    // ---- register stage: twiddle, DFT-16, x filter spectrum, IDFT-16, twiddle
-    const uint32_t lboZ = (uint32_t)(P * kN2 / 8) * 128;  // Z: MN-major, 256 K-rows (re k1 | im k1) x P*16
+    // ---- 2a: Y' = twiddled stage-A output / 32 as fp16 stage-B tiles (sequences alternate between groups)
 #pragma unroll 1
-    for (int s = 0; s < NS; ++s) {
-      const bool is_filter = with_filter && s == 0;
-      if (!is_filter && ((s - (with_filter ? 1 : 0)) & 1) != grp) continue;  // pairs alternate between groups
+    for (int s = grp; s < NS; s += 2) {
       float yr[16], yi[16];
       tc::tmem_ld16x2_wait(tmem + lane_off + (uint32_t)(s * kN2), tmem + lane_off + (uint32_t)(NC + s * kN2), yr, yi);
+      uint32_t pr[8], pi[8];
+#pragma unroll
+      for (int n2 = 0; n2 < kN2; n2 += 2) {
+        const float2 a = cmul(make_float2(yr[n2], yi[n2]), tws[n2]);
+        const float2 b = cmul(make_float2(yr[n2 + 1], yi[n2 + 1]), tws[n2 + 1]);
+        pr[n2 / 2] = Op<__half>::pack(a.x, b.x);
+        pi[n2 / 2] = Op<__half>::pack(a.y, b.y);
+      }
+      uint8_t* tile = sm.xz + (uint32_t)s * kYTile + (uint32_t)(row >> 3) * kYSbo + (uint32_t)(row & 7) * 16;
+      *reinterpret_cast<uint4*>(tile) = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+      *reinterpret_cast<uint4*>(tile + kYLbo) = make_uint4(pr[4], pr[5], pr[6], pr[7]);
+      *reinterpret_cast<uint4*>(tile + 2 * kYLbo) = make_uint4(pi[0], pi[1], pi[2], pi[3]);
+      *reinterpret_cast<uint4*>(tile + 3 * kYLbo) = make_uint4(pi[4], pi[5], pi[6], pi[7]);
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    // ---- stage B: X^ = DFT16(Y') per sequence into TMEM columns [32 s, 32 s + 32) (re k2 | im k2)
+    const uint32_t idY = tc::idesc_f16(128, 32, 0);
+    if (tid == 0) {
+      const uint32_t wfa = tc::smem_u32(sm.wf);
+      for (int s = 0; s < NS; ++s) {
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk)
+          tc::mma_f16(tmem + (uint32_t)(32 * s), tc::desc_kmajor(xz + s * kYTile + kk * 2 * kYLbo, kYLbo, kYSbo),
+                      tc::desc_kmajor(wfa + kk * 2 * kYLbo, kYLbo, kYSbo), idY, kk > 0 ? 1u : 0u);
+      }
+      tc::mma_commit(&sm.mbar);
+    }
+    ok = tc::mbar_wait_bounded(&sm.mbar, phase, kWaitNs);
+    phase ^= 1u;
+    if (__syncthreads_or(!ok)) {
+      failed = true;
+      break;
+    }
+    tc::fence_after_sync();
+    // ---- 2c: filter bins 32 f^/M (every thread keeps its row's 16), then V = X^ . f^ / M
+    // (X^ here is 1/32 of the transform) for this group's pairs
+    if (with_filter) {
+      float xr[16], xi[16];
+      tc::tmem_ld16x2_wait(tmem + lane_off, tmem + lane_off + 16u, xr, xi);
+      constexpr float sc = 32.0f * 32.0f / (float)kM;  // undo the 1/32 of stage B, x32 for the pairs, 1/M
+#pragma unroll
+      for (int k2 = 0; k2 < kN2; ++k2) fh[k2] = make_float2(xr[k2] * sc, xi[k2] * sc);
+    }
+#pragma unroll 1
+    for (int p = grp; p < P; p += 2) {
+      const int s = p + (with_filter ? 1 : 0);
+      float xr[16], xi[16];
+      tc::tmem_ld16x2_wait(tmem + lane_off + (uint32_t)(32 * s), tmem + lane_off + (uint32_t)(32 * s + 16), xr, xi);
+      uint32_t pr[8], pi[8];
+#pragma unroll
+      for (int k2 = 0; k2 < kN2; k2 += 2) {
+        const float2 a = cmul(make_float2(xr[k2], xi[k2]), fh[k2]);
+        const float2 b = cmul(make_float2(xr[k2 + 1], xi[k2 + 1]), fh[k2 + 1]);
+        pr[k2 / 2] = Op<__half>::pack(a.x, b.x);
+        pi[k2 / 2] = Op<__half>::pack(a.y, b.y);
+      }
+      uint8_t* tile = sm.xz + (uint32_t)s * kYTile + (uint32_t)(row >> 3) * kYSbo + (uint32_t)(row & 7) * 16;
+      *reinterpret_cast<uint4*>(tile) = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+      *reinterpret_cast<uint4*>(tile + kYLbo) = make_uint4(pr[4], pr[5], pr[6], pr[7]);
+      *reinterpret_cast<uint4*>(tile + 2 * kYLbo) = make_uint4(pi[0], pi[1], pi[2], pi[3]);
+      *reinterpret_cast<uint4*>(tile + 3 * kYLbo) = make_uint4(pi[4], pi[5], pi[6], pi[7]);
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    // ---- stage B': IDFT16(V) per pair into TMEM columns [32 p, 32 p + 32)
+    if (tid == 0) {
+      const uint32_t wia = tc::smem_u32(sm.wi);
+      for (int p = 0; p < P; ++p) {
+        const int s = p + (with_filter ? 1 : 0);
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk)
+          tc::mma_f16(tmem + (uint32_t)(32 * p), tc::desc_kmajor(xz + s * kYTile + kk * 2 * kYLbo, kYLbo, kYSbo),
+                      tc::desc_kmajor(wia + kk * 2 * kYLbo, kYLbo, kYSbo), idY, kk > 0 ? 1u : 0u);
+      }
+      tc::mma_commit(&sm.mbar);
+    }
+    ok = tc::mbar_wait_bounded(&sm.mbar, phase, kWaitNs);
+    phase ^= 1u;
+    if (__syncthreads_or(!ok)) {
+      failed = true;
+      break;
+    }
+    tc::fence_after_sync();
+    // ---- 2d: Z = stage-B' output x conj twiddle, MN-major (K rows re k1 | im k1) for stage A'
+    const uint32_t lboZ = (uint32_t)(P * kN2 / 8) * 128;  // Z: MN-major, 256 K-rows (re k1 | im k1) x P*16
+#pragma unroll 1
+    for (int p = grp; p < P; p += 2) {
+      float zr[16], zi[16];
+      tc::tmem_ld16x2_wait(tmem + lane_off + (uint32_t)(32 * p), tmem + lane_off + (uint32_t)(32 * p + 16), zr, zi);
       float2 v[kN2];
 #pragma unroll
-      for (int n2 = 0; n2 < kN2; ++n2) v[n2] = cmul(make_float2(yr[n2], yi[n2]), tw[n2]);
-      dft<kN2, -1>(v);
-      if (is_filter) {
-        constexpr float inv_m = 1.0f / (float)kM;
-#pragma unroll
-        for (int k2 = 0; k2 < kN2; ++k2) fh[k2] = make_float2(v[k2].x * inv_m, v[k2].y * inv_m);
-        continue;
+      for (int n2 = 0; n2 < kN2; ++n2) {
+        const float2 z = cmul(make_float2(zr[n2], zi[n2]), cconj(tws[n2]));
+        v[n2] = make_float2(32.f * z.x, 32.f * z.y);
       }
 #pragma unroll
-      for (int k2 = 0; k2 < kN2; ++k2) v[k2] = cmul(v[k2], fh[k2]);
-      dft<kN2, +1>(v);
-#pragma unroll
-      for (int n2 = 0; n2 < kN2; ++n2) v[n2] = cmul(v[n2], cconj(tw[n2]));
-      const int pc = s - (with_filter ? 1 : 0);  // pair column block
-#pragma unroll
       for (int half = 0; half < 2; ++half) {
-        const int n = pc * kN2 + half * 8;
+        const int n = p * kN2 + half * 8;
         const uint32_t offr = (uint32_t)(n >> 3) * 128 + (uint32_t)(row >> 3) * lboZ + (uint32_t)(row & 7) * 16;
         const uint32_t offi = offr + 16 * lboZ;  // K rows 128 + k1
         const float2* w = v + half * 8;
@@ -346,7 +464,7 @@ template <typename T>
 static cudaError_t fftconv_tc_t(const void* u, const float* f, const float* D, void* y, int B, int H, bool pdl,
                                 cudaStream_t st) {
   auto kern = fftconv_tc_kernel<T>;
-  const size_t smem = sizeof(TcSmem) + 1024;
+  const size_t smem = sizeof(TcSmem);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   static int num_sms = 0;

@@ -79,8 +79,8 @@ __global__ void __launch_bounds__(kGenThreads) ssm_gen_kernel(const float* __res
 //   Q[tl][2n]  - i Q[tl][2n+1]  = 2 C_n B_n A_n^tl   (scaled by a power of two)
 // Both tables are split into fp16 high and remainder parts (three MMAs,
 // about 22 significant bits).  AH[th] = A^(16 th0) A^(128 g) A^(16 m) for
-// th = th0 + 8 g + m, each factor an exactly phase-reduced power or at most
-// 7 products of one.  One CTA owns up to kGUnits consecutive 2048-tap units
+// th = th0 + 8 g + m; A^(16 th0) is an exactly phase-reduced power, the other
+// factors at most 7 products of the exact powers A, A^4, A^16, A^128, A^512.  One CTA owns up to kGUnits consecutive 2048-tap units
 // of one channel and builds Q once.
 static __device__ unsigned int g_gen_tc_timeouts;
 
@@ -102,8 +102,11 @@ struct GenLayout {
   static constexpr uint32_t tab = SHORT ? kGTab / 2 : kGTab;
   static constexpr uint32_t ahh = 0, ahl = tab, qh = 2 * tab, ql = qh + kGQ;
   static constexpr uint32_t mma_end = (ahl + kGTab > ql + kGQ) ? ahl + kGTab : ql + kGQ;
-  static constexpr uint32_t red = (mma_end + 15u) & ~15u, mbar = red + 32, tmem = mbar + 8;
-  static constexpr uint32_t bytes = tmem + 8;
+  // exact powers A, A^4, A^16, A^128, A^512 per mode; in SHORT they sit in the
+  // stretch that only feeds never-stored rows
+  static constexpr uint32_t pw = SHORT ? ql + kGQ : mma_end;
+  static constexpr uint32_t red = pw + 64 * 5 * 8, mbar = red + 32, tmem = mbar + 8;
+  static constexpr uint32_t bytes = (tmem + 8 > mma_end) ? tmem + 8 : mma_end;
 };
 __device__ __forceinline__ uint32_t gsplit(float a, float b, uint32_t& lo) {
   const __half2 h = __floats2half2_rn(a, b);
@@ -134,11 +137,13 @@ __global__ void __launch_bounds__(kGThr, SHORT ? 4 : 2) ssm_gen_tc_kernel(const 
     uint8_t* ahl;
     uint8_t* qh;
     uint8_t* ql;
+    float2* pw;
     float* red;
     uint64_t* mbar;
     uint32_t* tmem_p;
-  } sm{gtsm + LY::ahh, gtsm + LY::ahl, gtsm + LY::qh, gtsm + LY::ql, reinterpret_cast<float*>(gtsm + LY::red),
-       reinterpret_cast<uint64_t*>(gtsm + LY::mbar), reinterpret_cast<uint32_t*>(gtsm + LY::tmem)};
+  } sm{gtsm + LY::ahh, gtsm + LY::ahl, gtsm + LY::qh, gtsm + LY::ql, reinterpret_cast<float2*>(gtsm + LY::pw),
+       reinterpret_cast<float*>(gtsm + LY::red), reinterpret_cast<uint64_t*>(gtsm + LY::mbar),
+       reinterpret_cast<uint32_t*>(gtsm + LY::tmem)};
   const int h = blockIdx.y;
   const int units = (L + kGUnitTaps - 1) / kGUnitTaps;
   const int u0 = blockIdx.x * kGUnits, u1 = min(units, u0 + kGUnits);
@@ -150,22 +155,21 @@ __global__ void __launch_bounds__(kGThr, SHORT ? 4 : 2) ssm_gen_tc_kernel(const 
     tc::mbar_init(sm.mbar, 1);
     tc::fence_mbar_init();
   }
-  float2 lm = make_float2(0.f, 0.f), w = make_float2(0.f, 0.f), m8[8], G[NG];
+  // exact powers, five per mode, spread over the CTA
+  for (int idx = tid; idx < 64 * 5; idx += kGThr) {
+    const int m = idx / 5, e = idx - 5 * m;
+    float2 v = make_float2(0.f, 0.f);
+    if (m < N) {
+      const float2 l = lam[(size_t)h * N + m];
+      v = ssm_pow(d, l.x, l.y, e == 0 ? 1.0 : e == 1 ? 4.0 : e == 2 ? 16.0 : e == 3 ? 128.0 : 512.0);
+    }
+    sm.pw[idx] = v;
+  }
+  float2 lm = make_float2(0.f, 0.f), w = make_float2(0.f, 0.f);
   if (n < N) {
     lm = lam[(size_t)h * N + n];
     const float2 cb = cmul(Cp[(size_t)h * N + n], Bp[(size_t)h * N + n]);
     w = make_float2(2.f * cb.x, 2.f * cb.y);
-    const float2 a16 = ssm_pow(d, lm.x, lm.y, 16.0);
-    m8[0] = make_float2(1.f, 0.f);
-#pragma unroll
-    for (int m = 1; m < 8; ++m) m8[m] = cmul(m8[m - 1], a16);
-#pragma unroll
-    for (int r = 0; r < NG; ++r) G[r] = ssm_pow(d, lm.x, lm.y, 128.0 * (gq + 4 * r));
-  } else {
-#pragma unroll
-    for (int m = 0; m < 8; ++m) m8[m] = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int r = 0; r < NG; ++r) G[r] = make_float2(0.f, 0.f);
   }
   // power-of-two scale: the largest |Re|, |Im| of any 2 C B just below 2^13
   float mx = fmaxf(fabsf(w.x), fabsf(w.y));
@@ -182,13 +186,28 @@ __global__ void __launch_bounds__(kGThr, SHORT ? 4 : 2) ssm_gen_tc_kernel(const 
     scale = ldexpf(1.f, 13 - ex);
     inv = ldexpf(1.f, ex - 13);
   }
+  // this thread's factors: A^(16 m) (m < 8), A^(128 (gq + 4 r)), A^(4 gq); each at
+  // most 7 products of exact powers (zero for padding modes)
+  const float2 a1 = sm.pw[n * 5 + 0], a4 = sm.pw[n * 5 + 1], a16 = sm.pw[n * 5 + 2];
+  const float2 a128 = sm.pw[n * 5 + 3], a512 = sm.pw[n * 5 + 4];
+  const float2 one = n < N ? make_float2(1.f, 0.f) : make_float2(0.f, 0.f);
+  float2 m8[8], G[NG];
+  m8[0] = one;
+#pragma unroll
+  for (int m = 1; m < 8; ++m) m8[m] = cmul(m8[m - 1], a16);
+  float2 g128 = one, p4 = one;
+#pragma unroll
+  for (int i = 0; i < 3; ++i)
+    if (i < gq) {
+      g128 = cmul(g128, a128);
+      p4 = cmul(p4, a4);
+    }
+  G[0] = g128;
+#pragma unroll
+  for (int r = 1; r < NG; ++r) G[r] = cmul(G[r - 1], a512);
   // Q rows tl = 4 gq .. 4 gq + 3
   {
-    float2 p = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
-    if (n < N) {
-      a1 = ssm_pow(d, lm.x, lm.y, 1.0);
-      p = cmul(make_float2(w.x * scale, w.y * scale), ssm_pow(d, lm.x, lm.y, 4.0 * gq));
-    }
+    float2 p = cmul(make_float2(w.x * scale, w.y * scale), p4);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       uint32_t lo;
@@ -206,7 +225,8 @@ __global__ void __launch_bounds__(kGThr, SHORT ? 4 : 2) ssm_gen_tc_kernel(const 
   for (int u = u0; u < u1; ++u) {
     const int th0 = u * kGRows;
     const int rows = min(kGRows, (L - th0 * kGNC + kGNC - 1) / kGNC);
-    const float2 base = n < N ? ssm_pow(d, lm.x, lm.y, 16.0 * th0) : make_float2(0.f, 0.f);
+    const float2 base = n >= N ? make_float2(0.f, 0.f)
+                        : th0 == 0 ? make_float2(1.f, 0.f) : ssm_pow(d, lm.x, lm.y, 16.0 * th0);
 #pragma unroll
     for (int r = 0; r < NG; ++r) {
       const int g = gq + 4 * r;
