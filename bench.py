@@ -4,8 +4,9 @@
 One JSON line on stdout (rank 0).  A step is one pass of the hot path over one
 batch: the headline workload is the H3-125M-layer-shaped convolution
 (B=8, H=768, L=1024, N=64, fp16 I/O, filter regenerated on the device every
-step): one ssm_conv_fwd call, i.e. one kernel that generates the SSM filter
-and runs the fused FFT convolution.
+step): one ssm_conv_fwd call, i.e. the filter-generation kernel followed by
+the fused tensor-core FFT convolution kernel.  The roofline object describes
+the dominant kernel, the fused convolution, timed on its own in the same run.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                   [--others] [--impl ours|reference]
@@ -111,7 +112,7 @@ def run_ours(args, rank, world, local_rank):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     rflush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
     res = {}
-    step_fn, conv_fn, units, alg_bytes, kern_per_step, e2e_fn, e2e_bytes = build_step(wl, T, dev, api, lib)
+    step_fn, conv_fn, units, alg_bytes, kern_per_step, e2e_fn, e2e_bytes, dom_fn = build_step(wl, T, dev, api, lib)
     # warm-up
     for _ in range(args.warmup):
         step_fn()
@@ -155,9 +156,26 @@ def run_ours(args, rank, world, local_rank):
     wall = time.time() - wall0
     clocks = sampler.stop()
     step_ms = [a.elapsed_time(c) for a, b, c in ev]
-    conv_ms = [b.elapsed_time(c) for a, b, c in ev]
     tot_ms = sum(step_ms)
-    conv_avg = sum(conv_ms) / len(conv_ms)
+    # the dominant kernel on its own: graph-replayed, L2 flushed before each launch
+    for _ in range(3):
+        dom_fn()
+    torch.cuda.synchronize()
+    dgraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(dgraph):
+        dom_fn()
+    dgraph.replay()
+    torch.cuda.synchronize()
+    dom_ms = []
+    for i in range(args.steps):
+        flush_l2(flush, rflush)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        dgraph.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        dom_ms.append(a.elapsed_time(b))
+    conv_avg = sum(dom_ms) / len(dom_ms)
     t = torch.tensor([tot_ms, conv_avg], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -178,16 +196,19 @@ def run_ours(args, rank, world, local_rank):
     res.update(dict(
         metric=METRIC, value=value, unit="conv elements/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
         ms_per_step=ms_per_step, higher_is_better=True, scaling="weak", vs_baseline=None,
-        dtype="f32",
+        dtype="f16" if wl.dtype == "f16" else ("bf16" if wl.dtype == "bf16" else "f32"),
         data="synthetic",
         config=dict(workload=args.workload, B=wl.B, H=wl.H, L=wl.L, N=wl.N, io_dtype=wl.dtype,
                     timing="CUDA-graph replay of the step's library calls" if args.graph else "direct calls",
                     filter="generated on device every step" if "conv" in args.workload else None,
+                    arithmetic="tensor-core operands in the I/O type or fp16, fp32 accumulation; "
+                               "fp32 register arithmetic and fp32 filter",
                     l2="flushed before every step (256 MiB write + 256 MiB read, outside the per-step events)",
                     parallelism=f"replicas x{world} (rows independent, no collective)"),
         roofline=dict(bound="hbm", achieved=achieved, peak=peak, unit="GB/s", frac=achieved / peak,
-                      traffic=traffic, kernel="the step (filter kernel + fused conv kernel)", peak_source=peak_kind,
-                      algorithmic_bytes_per_launch=alg_bytes, avg_launch_ms=conv_avg),
+                      traffic=traffic, kernel=dominant_kernel_name(wl), peak_source=peak_kind,
+                      algorithmic_bytes_per_launch=alg_bytes, avg_launch_ms=conv_avg,
+                      step_achieved_gbs=units * 2 * DT_BYTES[wl.dtype] / (ms_per_step / 1e3) / 1e9),
         e2e=dict(value=e2e_val, unit="conv elements/s", h2d_bytes_per_step=e2e_bytes[0],
                  d2h_bytes_per_step=e2e_bytes[1]),
         gpu_launches=kern_per_step * args.steps,
@@ -219,10 +240,14 @@ def build_step(wl, T, dev, api, lib):
     ws = torch.empty(max(int(lib.ssm_conv_workspace(wl.H, wl.L)), 1), dtype=torch.uint8, device=dev)
     s = DT_BYTES[wl.dtype]
     units = wl.B * wl.H * wl.L
-    fused = wl.L >= 1024
-    # algorithmic bytes of the dominant launch: u read + y write (+ the filter
-    # read when it is generated by a separate kernel)
-    alg = units * 2 * s + (0 if fused else wl.H * wl.L * 4)
+    # kernels per ssm_conv_fwd call: L = 1024 with 16-bit I/O runs the filter
+    # kernel then the tensor-core convolution; other L >= 1024 generate the
+    # filter inside the convolution kernel; shorter L use two kernels
+    launches = 2 if (wl.L == 1024 and wl.dtype != "f32") or wl.L < 1024 else 1
+    # algorithmic bytes of the dominant kernel (the convolution on a given
+    # filter): u read + y write + the fp32 filter read
+    alg = units * 2 * s + wl.H * wl.L * 4
+    f_given = torch.empty((wl.H, wl.L), dtype=torch.float32, device=dev)
 
     def step():
         api.ssm_conv_fwd(u, dt, lam, Bp, Cp, D, workspace=ws, out=y)
@@ -230,6 +255,11 @@ def build_step(wl, T, dev, api, lib):
     def conv(ev_mid):
         ev_mid.record(torch.cuda.current_stream())
         api.ssm_conv_fwd(u, dt, lam, Bp, Cp, D, workspace=ws, out=y)
+
+    def dominant():
+        api.fftconv_fwd(u, f_given, D, out=y)
+
+    api.ssm_kernel_gen(dt, lam, Bp, Cp, wl.L, out=f_given)
 
     # e2e: pinned host inputs -> device, one ssm_conv_fwd C-ABI call, result -> pinned host
     hu = torch.empty(u.shape, dtype=u.dtype, pin_memory=True)
@@ -260,7 +290,7 @@ def build_step(wl, T, dev, api, lib):
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / n
 
-    return step, conv, units, alg, (1 if fused else 2), e2e, (h2d, d2h)
+    return step, conv, units, alg, launches, e2e, (h2d, d2h), dominant
 
 
 def other_workloads(T, dev, api, args):
@@ -359,10 +389,16 @@ def profiled_traffic(workload):
     return d.get("dram_bytes_per_launch")
 
 
+def dominant_kernel_name(wl):
+    if wl.L == 1024 and wl.dtype != "f32":
+        return "fftconv_tc_kernel (tensor-core fused FFT conv, given filter)"
+    return "fftconv_kernel (CUDA-core fused FFT conv, given filter)"
+
+
 def kernel_source_sha1():
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "fft_long_convolution_flashconv_b200", "csrc")
-    for name in ("fftconv.cu", "fft_stockham.cuh", "common.cuh", "ssm_tables.cuh"):
+    for name in ("fftconv_tc.cu", "fftconv.cu", "fft_stockham.cuh", "common.cuh", "tc100.cuh"):
         with open(os.path.join(csrc, name), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
