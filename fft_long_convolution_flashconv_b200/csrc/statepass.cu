@@ -19,7 +19,9 @@
 //        y[e-1]   += sum_n Re( G[eh][n] Q[n][el] ),
 //        G[eh][n]  = 2 C_n x_n A_n^(BL eh),  Q[n][el] = A_n^el
 // One CTA owns one (b, h) row and walks its chunks; modes are processed in
-// blocks of 64.
+// blocks of 64.  These CUDA-core kernels serve fp32 I/O, chunks other than
+// 2048/4096/8192 and N > 64; the other cases run the same contractions as
+// tcgen05 GEMMs (statepass_tc.cu) with this file's carry kernel.
 #include "kernels.cuh"
 
 namespace fc {
