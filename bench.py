@@ -240,10 +240,11 @@ def build_step(wl, T, dev, api, lib):
     ws = torch.empty(max(int(lib.ssm_conv_workspace(wl.H, wl.L)), 1), dtype=torch.uint8, device=dev)
     s = DT_BYTES[wl.dtype]
     units = wl.B * wl.H * wl.L
-    # kernels per ssm_conv_fwd call: L = 1024 with 16-bit I/O runs the filter
-    # kernel then the tensor-core convolution; other L >= 1024 generate the
-    # filter inside the convolution kernel; shorter L use two kernels
-    launches = 2 if (wl.L == 1024 and wl.dtype != "f32") or wl.L < 1024 else 1
+    # kernels per ssm_conv_fwd call: the filter kernel then the convolution,
+    # except for L >= 1024 with N > 64 (and no tensor-core conv), where the
+    # convolution kernel generates the filter itself
+    tc_conv = wl.L == 1024 and wl.dtype != "f32"
+    launches = 1 if (wl.L >= 1024 and wl.N > 64 and not tc_conv) else 2
     # algorithmic bytes of the dominant kernel (the convolution on a given
     # filter): u read + y write + the fp32 filter read
     alg = units * 2 * s + wl.H * wl.L * 4
@@ -261,32 +262,60 @@ def build_step(wl, T, dev, api, lib):
 
     api.ssm_kernel_gen(dt, lam, Bp, Cp, wl.L, out=f_given)
 
-    # e2e: pinned host inputs -> device, one ssm_conv_fwd C-ABI call, result -> pinned host
+    # e2e: pinned host inputs -> device, one ssm_conv_fwd C-ABI call, result -> pinned host,
+    # every step.  Steps are pipelined the way a serving loop runs them: step i's inputs go
+    # up on a copy stream while step i-1 computes, and its result comes back on another
+    # copy stream while step i+1 computes (device inputs, parameters, outputs and host
+    # outputs double-buffered; events order every reuse of a buffer).
     hu = torch.empty(u.shape, dtype=u.dtype, pin_memory=True)
     hu.copy_(u.cpu())
     hp = [x.cpu().pin_memory() for x in (dt, lam, Bp, Cp, D)]
-    dp = [torch.empty_like(x, device=dev) for x in hp]
-    hy = torch.empty(u.shape, dtype=u.dtype, pin_memory=True)
-    du = torch.empty_like(u)
+    dps = [[torch.empty_like(x, device=dev) for x in hp] for _ in range(2)]
+    hys = [torch.empty(u.shape, dtype=u.dtype, pin_memory=True) for _ in range(2)]
+    dus = [torch.empty_like(u) for _ in range(2)]
+    dys = [torch.empty_like(u) for _ in range(2)]
     h2d = hu.numel() * hu.element_size() + sum(x.numel() * x.element_size() for x in hp)
-    d2h = hy.numel() * hy.element_size()
-
-    def one():
-        du.copy_(hu, non_blocking=True)
-        for a, b in zip(dp, hp):
-            a.copy_(b, non_blocking=True)
-        api.ssm_conv_fwd(du, dp[0], dp[1], dp[2], dp[3], dp[4], workspace=ws, out=y)
-        hy.copy_(y, non_blocking=True)
+    d2h = hys[0].numel() * hys[0].element_size()
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
 
     def e2e(n):
-        for _ in range(2):
-            one()
+        cur = torch.cuda.current_stream()
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_comp = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+
+        def run(steps, t0=None):
+            if t0 is not None:
+                t0.record(cur)
+            s_in.wait_stream(cur)
+            s_out.wait_stream(cur)
+            for i in range(steps):
+                b = i % 2
+                with torch.cuda.stream(s_in):
+                    if i >= 2:
+                        s_in.wait_event(ev_comp[b])  # step i-2 has finished reading dus[b], dps[b]
+                    dus[b].copy_(hu, non_blocking=True)
+                    for a, h in zip(dps[b], hp):
+                        a.copy_(h, non_blocking=True)
+                    ev_in[b].record(s_in)
+                cur.wait_event(ev_in[b])
+                if i >= 2:
+                    cur.wait_event(ev_out[b])  # step i-2's result has left dys[b]
+                p = dps[b]
+                api.ssm_conv_fwd(dus[b], p[0], p[1], p[2], p[3], p[4], workspace=ws, out=dys[b])
+                ev_comp[b].record(cur)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev_comp[b])
+                    hys[b].copy_(dys[b], non_blocking=True)
+                    ev_out[b].record(s_out)
+            cur.wait_stream(s_in)
+            cur.wait_stream(s_out)
+
+        run(4)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(n):
-            one()
-        e1.record()
+        run(n, e0)
+        e1.record(cur)
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / n
 

@@ -139,7 +139,7 @@ FC_API fc_status ssm_conv_fwd(const void* u, const float* dt, const float* lambd
     return cuda_status(fc::launch_fftconv_tc(u, f, D, y, B, H, L, dtype, true, st),
                        "ssm_conv_fwd: tensor-core conv launch");
   }
-  if (L >= 1024) {  // filter generated inside the convolution kernel
+  if (L >= 1024 && N > 64) {  // filter generated inside the convolution kernel (no tensor-core generator)
     const fc::SsmArgs sp{dt, (const float2*)lambda, (const float2*)Bp, (const float2*)Cp, N};
     return cuda_status(fc::launch_fftconv(u, nullptr, L, sp, D, y, B, H, L, L, 1, dtype, st),
                        "ssm_conv_fwd: fused launch");

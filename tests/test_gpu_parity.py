@@ -116,8 +116,9 @@ def test_fftconv_arbitrary_filter_and_impulse_alignment():
 @pytest.mark.parametrize("L,N,dtype", [(1024, 65, "f32"), (2048, 40, "f16"), (4096, 17, "bf16"), (8192, 70, "f32"),
                                        (512, 64, "f16")])
 def test_ssm_conv_fused_generation(L, N, dtype):
-    """ssm_conv_fwd generates the filter inside the convolution kernel for
-    L >= 1024 (several mode blocks, odd B, channels split across CTAs)."""
+    """ssm_conv_fwd: for L >= 1024 and N > 64 the filter is generated inside
+    the convolution kernel (several mode blocks, odd B, channels split across
+    CTAs); otherwise the tensor-core generator runs first."""
     B, H = 3, 7
     wl = W.make_conv(B=B, H=H, L=L, N=N, dtype=dtype, seed=N + L, dt_range=("loguniform", -3.0, -1.0))
     dtt, lam, Bp, Cp, D = params(wl)
