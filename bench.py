@@ -480,7 +480,7 @@ def run_reference(args, rank, world):
                 warmup=args.warmup, ms_per_step=tot / args.steps * 1e3, higher_is_better=True, scaling="weak",
                 vs_baseline=None, dtype="f64", data="synthetic", impl="reference",
                 config=dict(workload=args.workload, B=wl.B, H=wl.H, L=wl.L, N=wl.N, io_dtype=wl.dtype,
-                    timing="CUDA-graph replay of the step's library calls" if args.graph else "direct calls",
+                            timing="host wall clock around each oracle sample (the oracle runs on the CPU)",
                             note=f"each step is a bounded sample of {rows} rows on the CPU oracle"),
                 cpu_baseline=dict(value=value, unit="conv elements/s", cores=cref.num_threads(), kind="oracle",
                                   sample=f"{rows} rows per step of {wl.name}"),
