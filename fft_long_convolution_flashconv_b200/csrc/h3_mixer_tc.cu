@@ -12,8 +12,11 @@
 // The shift SSM k~[s,c] = sum_j Cshift[c,j] k[s-j,c] runs once, in a small
 // elementwise kernel, into a workspace (rounded to the operand type).  Q and
 // K~ tiles are K-major with padded core-matrix offsets (LBO 144 bytes) so that
-// the row-wise 16-byte staging stores are free of bank conflicts; V is staged
+// the row-wise 16-byte staging copies are free of bank conflicts; V is staged
 // as it lies in memory and read by the tensor cores as an MN-major operand.
+// The next s tile's K~ and V are copied in with cp.async while the current
+// tile is processed (K~ once the S-MMA has read the current one; V into a
+// second buffer).
 // Every wait on MMA completion is bounded; on a timeout the CTA records it in
 // a device counter, skips its remaining work and still frees its TMEM.
 #include "kernels.cuh"
@@ -37,7 +40,7 @@ constexpr uint32_t kPLbo = 128, kPSbo = (kT / 8) * 128;    // P: 128 rows x 128 
 struct MixSmem {
   uint8_t q[(kT / 8) * kQSbo];      // A of S-MMA  (rows t, K = i)
   uint8_t k[(kT / 8) * kQSbo];      // B of S-MMA  (rows s, K = i)
-  uint8_t v[(kT / 8) * kVLbo];      // B of O-MMA  (N = j, K = s), MN-major
+  uint8_t v[2][(kT / 8) * kVLbo];   // B of O-MMA  (N = j, K = s), MN-major, double-buffered
   uint8_t p[kT * kT * 2];           // A of O-MMA  (rows t, K = s)
   float fs[2 * kT];
   uint64_t mbar;
@@ -47,6 +50,11 @@ struct MixSmem {
 __device__ __forceinline__ uint32_t qoff(int r, int c8) {
   return (uint32_t)(r >> 3) * kQSbo + (uint32_t)(c8 >> 3) * kQLbo + (uint32_t)(r & 7) * 16;
 }
+__device__ __forceinline__ void cp_async16(uint32_t saddr, const void* g) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(g) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ uint32_t voff(int s, int j8) {  // 8 consecutive j at time s
   return (uint32_t)(j8 >> 3) * kVSbo + (uint32_t)(s >> 3) * kVLbo + (uint32_t)(s & 7) * 16;
 }
@@ -170,21 +178,38 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
   uint32_t phase = 0;
   bool failed = false;
   const int row = tid;  // TMEM lane / tile row owned by this thread
-
-  for (int st = 0; st <= tt && !failed; ++st) {
-    const int s0 = st * kT;
-    // ---- stage the K~ and V tiles (rows s0 .. s0+127) and the Toeplitz weights
+  // K~ / V tile of rows s0 .. s0+127 -> shared memory with cp.async (rows past L zeroed)
+  auto issue_k = [&](int s0) {
+    const uint32_t ka = tc::smem_u32(sm.k);
     for (int idx = tid; idx < kT * (kHD / 8); idx += kThr) {
       const int r = idx >> 3, c8 = (idx & 7) * 8;
       const int s = s0 + r;
-      uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
-      if (s < L) {
-        kv = *reinterpret_cast<const uint4*>(kb + (size_t)s * dm + c8);
-        vv = *reinterpret_cast<const uint4*>(vb + (size_t)s * dm + c8);
-      }
-      *reinterpret_cast<uint4*>(sm.k + qoff(r, c8)) = kv;
-      *reinterpret_cast<uint4*>(sm.v + voff(r, c8)) = vv;
+      if (s < L)
+        cp_async16(ka + qoff(r, c8), kb + (size_t)s * dm + c8);
+      else
+        *reinterpret_cast<uint4*>(sm.k + qoff(r, c8)) = make_uint4(0, 0, 0, 0);
     }
+  };
+  auto issue_v = [&](int s0, int buf) {
+    const uint32_t va = tc::smem_u32(sm.v[buf]);
+    for (int idx = tid; idx < kT * (kHD / 8); idx += kThr) {
+      const int r = idx >> 3, c8 = (idx & 7) * 8;
+      const int s = s0 + r;
+      if (s < L)
+        cp_async16(va + voff(r, c8), vb + (size_t)s * dm + c8);
+      else
+        *reinterpret_cast<uint4*>(sm.v[buf] + voff(r, c8)) = make_uint4(0, 0, 0, 0);
+    }
+  };
+  issue_k(0);
+  issue_v(0, 0);
+  cp_async_commit();
+
+  for (int st = 0; st <= tt && !failed; ++st) {
+    const int s0 = st * kT;
+    // ---- this tile's K~ and V have been copied (issued during the previous tile);
+    // the Toeplitz weights for (t0, s0)
+    cp_async_wait_all();
     for (int idx = tid; idx < 2 * kT - 1; idx += kThr) {
       const int d = idx - (kT - 1) + (t0 - s0);  // t - s
       float w = (d >= 0 && d < L) ? fh[d] : 0.f;
@@ -195,6 +220,10 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
+    // ---- the next tile's V goes to the other buffer (its last reader, the O-MMA of
+    // tile st - 1, has completed)
+    if (st + 1 <= tt) issue_v(s0 + kT, (st + 1) & 1);
+    cp_async_commit();
     // ---- S = Q K~^T
     if (tid == 0) {
       const uint32_t qa = tc::smem_u32(sm.q), ka = tc::smem_u32(sm.k);
@@ -211,6 +240,9 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
       break;
     }
     tc::fence_after_sync();
+    // ---- the S-MMA has read K~: the next tile's K~ can come in now
+    if (st + 1 <= tt) issue_k(s0 + kT);
+    cp_async_commit();
     // ---- P = S (.) Toeplitz weights, rounded to the operand type, into the K-major A tile
 #pragma unroll 1
     for (int c = 0; c < kT; c += 16) {
@@ -234,7 +266,7 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
     tc::fence_after_sync();
     // ---- O += P V
     if (tid == 0) {
-      const uint32_t pa = tc::smem_u32(sm.p), va = tc::smem_u32(sm.v);
+      const uint32_t pa = tc::smem_u32(sm.p), va = tc::smem_u32(sm.v[st & 1]);
 #pragma unroll
       for (int kk = 0; kk < kT / 16; ++kk)
         tc::mma_f16(tO, tc::desc_kmajor(pa + kk * 2 * kPLbo, kPLbo, kPSbo),
@@ -249,6 +281,7 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
     }
     tc::fence_after_sync();
   }
+  cp_async_wait_all();
   if (!failed) {
     const int t = t0 + row;
 #pragma unroll 1
