@@ -7,6 +7,9 @@ batch: the headline workload is the H3-125M-layer-shaped convolution
 step): one ssm_conv_fwd call, i.e. the filter-generation kernel followed by
 the fused tensor-core FFT convolution kernel.  The roofline object describes
 the dominant kernel, the fused convolution, timed on its own in the same run.
+Rank 0 also times the rest of the metric's range by default ("configs"): the
+L = 8192 fused conv, L = 65536 state passing and the H3 mixer, each with its
+own roofline and clocks.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                   [--others] [--impl ours|reference]
@@ -38,6 +41,7 @@ from fft_long_convolution_flashconv_b200 import workloads as W  # noqa: E402
 HEADLINE = "cfg2_conv_f16_B8_H768_L1024"
 METRIC = "conv elements/s (B·H·L per sec) and achieved HBM GB/s fraction, L=1K–64K"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 DT_BYTES = {"f32": 4, "f16": 2, "bf16": 2}
 
 
@@ -214,8 +218,10 @@ def run_ours(args, rank, world, local_rank):
         gpu_launches=kern_per_step * args.steps,
         clocks=clocks, wall_s=wall,
     ))
+    if not args.headline_only and rank == 0:
+        res["configs"] = secondary_configs(T, dev, api, args, local_rank)
     if args.others and rank == 0:
-        res["other_workloads"] = other_workloads(T, dev, api, args)
+        res["headline_split"] = split_headline(T, dev, api, args)
     return res
 
 
@@ -322,86 +328,150 @@ def build_step(wl, T, dev, api, lib):
     return step, conv, units, alg, launches, e2e, (h2d, d2h), dominant
 
 
-def other_workloads(T, dev, api, args):
-    """Secondary numbers: the long fused regime, state passing, the H3 mixer."""
+def tensor_peak():
+    """Dense 16-bit tensor-core peak in TFLOP/s: the measured burst figure (the
+    mixer is timed in isolation), else the fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as fh:
+            return float(json.load(fh)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def graph_time(fn, n, flush, rflush, stream):
+    """Average CUDA-event time of one call of fn, captured once in a CUDA graph
+    and replayed n times, the L2 flushed before every replay (outside the
+    events).  Returns (avg_ms, list_of_ms)."""
+    import torch
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    g.replay()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(n):
+        flush_l2(flush, rflush)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms.append(a.elapsed_time(b))
+    del g
+    return sum(ms) / len(ms), ms
+
+
+def secondary_configs(T, dev, api, args, local_rank):
+    """The other workloads of the metric's range (L = 8K fused, L = 64K state
+    passing, the H3 mixer), each timed on the device with CUDA events (graph
+    replay, L2 flushed before every call), each with its own roofline and the
+    clocks sampled while it ran.  The headline line's value stays the L = 1K
+    workload."""
     import torch
     out = {}
-    peak, _ = hbm_peak()
+    peak, peak_kind = hbm_peak()
+    tpeak, tpeak_kind = tensor_peak()
+    stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     rflush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+    n = max(3, args.other_steps)
 
-    def timeit(fn, n):
-        for _ in range(2):
-            fn()
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            fn()
-        g.replay()
-        torch.cuda.synchronize()
-        tot = 0.0
-        for _ in range(n):
-            flush_l2(flush, rflush)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            g.replay()
-            b.record()
-            torch.cuda.synchronize()
-            tot += a.elapsed_time(b)
-        return tot / n
+    def hbm_roof(kernel, nbytes, ms, note):
+        a = nbytes / (ms / 1e3) / 1e9
+        return dict(bound="hbm", achieved=a, peak=peak, unit="GB/s", frac=a / peak, traffic=None,
+                    kernel=kernel, peak_source=peak_kind, algorithmic_bytes_per_launch=nbytes,
+                    avg_launch_ms=ms, bytes_note=note)
 
-    wl = W.make("cfg2_conv_f16_B8_H768_L1024")
-    u = T(wl.u, "f16")
-    dt, lam, Bp, Cp, D = T(wl.dt), T(wl.lam), T(wl.Bp), T(wl.Cp), T(wl.D)
-    f = torch.empty((wl.H, wl.L), dtype=torch.float32, device=dev)
-    y = torch.empty_like(u)
-    ms_gen = timeit(lambda: api.ssm_kernel_gen(dt, lam, Bp, Cp, wl.L, out=f), args.other_steps)
-    ms_conv = timeit(lambda: api.fftconv_fwd(u, f, D, out=y), args.other_steps)
-    out[wl.name + " (separate kernels)"] = dict(gen_ms=ms_gen, conv_ms=ms_conv)
-    del u, y, f
-
+    # ---- L = 8192 fused block-FFT regime (bf16, B=4, H=1024)
     wl = W.make("cfg3_conv_bf16_B4_H1024_L8192")
     u = T(wl.u, "bf16")
     dt, lam, Bp, Cp, D = T(wl.dt), T(wl.lam), T(wl.Bp), T(wl.Cp), T(wl.D)
     f = torch.empty((wl.H, wl.L), dtype=torch.float32, device=dev)
     y = torch.empty_like(u)
+    ws = torch.empty(api.ssm_conv_workspace_bytes(wl.H, wl.L), dtype=torch.uint8, device=dev)
     api.ssm_kernel_gen(dt, lam, Bp, Cp, wl.L, out=f)
-    ms = timeit(lambda: api.fftconv_fwd(u, f, D, out=y), args.other_steps)
     units = wl.B * wl.H * wl.L
-    gb = (units * 4 + wl.H * wl.L * 4) / 1e9
-    out[wl.name] = dict(conv_ms=ms, elems_per_s=units / (ms / 1e3), hbm_frac=gb / (ms / 1e3) / peak)
-    ms_full = timeit(lambda: (api.ssm_kernel_gen(dt, lam, Bp, Cp, wl.L, out=f), api.fftconv_fwd(u, f, D, out=y)),
-                     args.other_steps)
-    out[wl.name]["step_ms_with_filter_gen"] = ms_full
-    cfg3_ns_per_elem = ms * 1e6 / units
-    del u, y, f
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    ms_conv, _ = graph_time(lambda: api.fftconv_fwd(u, f, D, out=y), n, flush, rflush, stream)
+    ms_step, _ = graph_time(lambda: api.ssm_conv_fwd(u, dt, lam, Bp, Cp, D, workspace=ws, out=y), n, flush,
+                            rflush, stream)
+    clocks = sampler.stop()
+    out[wl.name] = dict(
+        step="ssm_conv_fwd (filter generated on the device, then the fused conv)",
+        step_ms=ms_step, value=units / (ms_step / 1e3), unit="conv elements/s",
+        roofline=hbm_roof(dominant_kernel_name(wl), units * 4 + wl.H * wl.L * 4, ms_conv,
+                          "u read + y written (bf16) + fp32 filter read, conv on a given filter"),
+        clocks=clocks)
+    cfg3_ns_per_elem = ms_conv * 1e6 / units
+    del u, y, f, ws
 
+    # ---- L = 65536 state passing (fp16, B=1, H=2560, chunk 8192)
     wl = W.make("cfg4_statepass_f16_B1_H2560_L65536_T8192")
     u = T(wl.u, "f16")
     dt, lam, Bp, Cp, D = T(wl.dt), T(wl.lam), T(wl.Bp), T(wl.Cp), T(wl.D)
     y = torch.empty_like(u)
     ws = torch.empty(api.statepass_workspace_bytes(wl.B, wl.H, wl.L, wl.N, wl.chunk), dtype=torch.uint8,
                      device=dev)
-    ms = timeit(lambda: api.fftconv_statepass(u, dt, lam, Bp, Cp, D, wl.chunk, workspace=ws, out=y),
-                max(2, args.other_steps // 4))
     units = wl.B * wl.H * wl.L
-    out[wl.name] = dict(step_ms=ms, elems_per_s=units / (ms / 1e3),
-                        hbm_frac=(units * 4) / 1e9 / (ms / 1e3) / peak,
-                        per_elem_vs_cfg3=(ms * 1e6 / units) / cfg3_ns_per_elem)
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    ms, _ = graph_time(lambda: api.fftconv_statepass(u, dt, lam, Bp, Cp, D, wl.chunk, workspace=ws, out=y),
+                       max(3, n // 2), flush, rflush, stream)
+    clocks = sampler.stop()
+    out[wl.name] = dict(
+        step="fftconv_statepass (chunk filter, chunk convs, end states, carry, initial-state term)",
+        step_ms=ms, value=units / (ms / 1e3), unit="conv elements/s",
+        roofline=hbm_roof("the whole state-passing step", units * 4, ms, "u read + y written (fp16)"),
+        per_elem_vs_L8192_conv=(ms * 1e6 / units) / cfg3_ns_per_elem,
+        clocks=clocks)
     del u, y, ws
 
+    # ---- H3 mixer (fp16, B=8, L=2048, 12 heads x 64)
     mw = W.make("cfg5_h3mixer_f16_B8_L2048_d768")
     q, k, v = T(mw.q, "f16"), T(mw.k, "f16"), T(mw.v, "f16")
     Cs, dt, lam, Bp, Cp, D = T(mw.Cshift), T(mw.dt), T(mw.lam), T(mw.Bp), T(mw.Cp), T(mw.D)
     o = torch.empty_like(q)
     ws = torch.empty(api.h3_mixer_workspace_bytes(mw.B, mw.L, mw.heads, mw.head_dim, mw.N), dtype=torch.uint8,
                      device=dev)
-    ms = timeit(lambda: api.h3_mixer_fwd(q, k, v, Cs, dt, lam, Bp, Cp, D, mw.heads, workspace=ws, out=o),
-                max(2, args.other_steps // 4))
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    ms, _ = graph_time(lambda: api.h3_mixer_fwd(q, k, v, Cs, dt, lam, Bp, Cp, D, mw.heads, workspace=ws, out=o),
+                       n, flush, rflush, stream)
+    clocks = sampler.stop()
     flops = 2.0 * 2.0 * mw.B * mw.heads * (mw.L * (mw.L + 1) / 2) * mw.head_dim
-    out[mw.name] = dict(step_ms=ms, toeplitz_tflops=flops / (ms / 1e3) / 1e12,
-                        hbm_frac=(4 * mw.B * mw.L * mw.heads * mw.head_dim * 2) / 1e9 / (ms / 1e3) / peak)
+    units = mw.B * mw.L * mw.heads * mw.head_dim
+    tf = flops / (ms / 1e3) / 1e12
+    out[mw.name] = dict(
+        step="h3_mixer_fwd (filters, shift SSM, Toeplitz-form mixer)", step_ms=ms,
+        value=units / (ms / 1e3), unit="output elements/s",
+        roofline=dict(bound="tensor", achieved=tf, peak=tpeak, unit="TFLOP/s", frac=tf / tpeak, traffic=None,
+                      kernel="the whole mixer call", peak_source=tpeak_kind, algorithmic_flops=flops,
+                      avg_launch_ms=ms, flops_note="causal half of S = Q K~^T and O = P V per (b, head)"),
+        hbm_frac=(4 * units * 2) / 1e9 / (ms / 1e3) / peak,
+        clocks=clocks)
     return out
+
+
+def split_headline(T, dev, api, args):
+    """The headline step's two kernels timed separately (filter, then conv)."""
+    import torch
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    rflush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+    wl = W.make(HEADLINE)
+    u = T(wl.u, "f16")
+    dt, lam, Bp, Cp, D = T(wl.dt), T(wl.lam), T(wl.Bp), T(wl.Cp), T(wl.D)
+    f = torch.empty((wl.H, wl.L), dtype=torch.float32, device=dev)
+    y = torch.empty_like(u)
+    ms_gen, _ = graph_time(lambda: api.ssm_kernel_gen(dt, lam, Bp, Cp, wl.L, out=f), args.other_steps, flush,
+                           rflush, stream)
+    ms_conv, _ = graph_time(lambda: api.fftconv_fwd(u, f, D, out=y), args.other_steps, flush, rflush, stream)
+    return {wl.name + " (separate kernels)": dict(gen_ms=ms_gen, conv_ms=ms_conv)}
 
 
 def profiled_traffic(workload):
@@ -494,8 +564,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=HEADLINE)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--others", action="store_true", help="also time the other workloads (rank 0)")
-    ap.add_argument("--other-steps", type=int, default=20)
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the L=8K, L=64K and mixer workloads (rank 0 times them by default)")
+    ap.add_argument("--others", action="store_true", help="also time the headline's two kernels separately")
+    ap.add_argument("--other-steps", type=int, default=10)
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--load-seconds", type=float, default=1.5)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

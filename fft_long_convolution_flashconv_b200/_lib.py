@@ -20,6 +20,7 @@ SIGNATURES = {
     "fc_version": (ctypes.c_int, []),
     "fc_status_string": (ctypes.c_char_p, [_i]),
     "fc_last_error": (ctypes.c_char_p, []),
+    "fc_tc_timeouts": (ctypes.c_uint, []),
     "ssm_kernel_gen": (_i, [_fp, _fp, _fp, _fp, _i, _i, _i, _fp, _vp]),
     "fftconv_fwd": (_i, [_vp, _fp, _fp, _vp, _i, _i, _i, _i, _vp]),
     "ssm_conv_workspace": (_sz, [_i, _i]),

@@ -61,6 +61,12 @@ def _alloc_ws(nbytes: int, device) -> torch.Tensor:
     return torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
 
 
+def tc_timeouts() -> int:
+    """Tensor-core blocks that gave up waiting on a matrix-multiply completion
+    (their part of an output is unwritten); 0 in normal operation."""
+    return int(_lib.load().fc_tc_timeouts())
+
+
 def ssm_kernel_gen(dt, lam, Bp, Cp, L: int, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """f[h, k] = 2 Re sum_n C B A^k, A = exp(dt lambda); returns H x L float32."""
     lib = _lib.load()

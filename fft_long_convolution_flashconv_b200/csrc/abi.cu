@@ -48,6 +48,30 @@ fc_status check_params(const float* dt, const float* lambda, const float* Bp, co
 
 }  // namespace
 
+namespace fc {
+// Filter generation then the fused convolution; f is H x L floats of scratch
+// (unused when the convolution kernel generates the filter itself).  Shared by
+// ssm_conv_fwd (caller workspace) and ssm_conv_fwd_noalloc (library array).
+cudaError_t run_ssm_conv(const void* u, const float* dt, const float* lambda, const float* Bp, const float* Cp,
+                         const float* D, void* y, int B, int H, int L, int N, float* f, int dtype,
+                         cudaStream_t st) {
+  const SsmArgs none{nullptr, nullptr, nullptr, nullptr, 0};
+  cudaError_t e;
+  if (fftconv_tc_supported(L, dtype)) {  // filter kernel, then the tensor-core convolution
+    e = launch_ssm_gen(dt, lambda, Bp, Cp, H, N, L, f, st);
+    if (e != cudaSuccess) return e;
+    return launch_fftconv_tc(u, f, D, y, B, H, L, dtype, true, st);
+  }
+  if (L >= 1024 && N > 64) {  // filter generated inside the convolution kernel (no tensor-core generator)
+    const SsmArgs sp{dt, (const float2*)lambda, (const float2*)Bp, (const float2*)Cp, N};
+    return launch_fftconv(u, nullptr, L, sp, D, y, B, H, L, L, 1, dtype, st);
+  }
+  e = launch_ssm_gen(dt, lambda, Bp, Cp, H, N, L, f, st);
+  if (e != cudaSuccess) return e;
+  return launch_fftconv(u, f, L, none, D, y, B, H, L, L, 1, dtype, st);
+}
+}  // namespace fc
+
 extern "C" {
 
 FC_API int fc_version(void) { return 100; }
@@ -82,6 +106,7 @@ FC_API fc_status ssm_kernel_gen(const float* dt, const float* lambda, const floa
 static fc_status check_conv_io(const void* u, const void* y, int B, int H, long long L, int dtype) {
   FC_REQUIRE(dtype_ok(dtype), FC_EINVAL, "unknown dtype %d", dtype);
   FC_REQUIRE(B >= 1 && H >= 1, FC_EINVAL, "B, H must be >= 1 (got %d, %d)", B, H);
+  FC_REQUIRE(B <= (1 << 30), FC_EUNSUPPORTED, "B = %d > 2^30", B);
   FC_REQUIRE(u && y, FC_EINVAL, "null u or y");
   FC_REQUIRE(aligned(u, 16) && aligned(y, 16), FC_EINVAL, "u and y must be 16-byte aligned");
   const size_t bytes = (size_t)B * H * (size_t)L * dtype_size(dtype);
@@ -100,7 +125,6 @@ FC_API fc_status fftconv_fwd(const void* u, const float* f, const float* D, void
   FC_REQUIRE(aligned(f, 16) && aligned(D, 4), FC_EINVAL, "f must be 16-byte aligned, D 4-byte aligned");
   FC_REQUIRE(pow2(L) && L >= 16 && L <= 8192, FC_EUNSUPPORTED,
              "fftconv_fwd: L must be a power of two in [16, 8192] (got %d)", L);
-  FC_REQUIRE((long long)B * 1 <= (1LL << 30), FC_EUNSUPPORTED, "B too large");
   if (fc::fftconv_tc_supported(L, dtype))
     return cuda_status(fc::launch_fftconv_tc(u, f, D, y, B, H, L, dtype, false, (cudaStream_t)stream),
                        "fftconv_fwd (tensor cores) launch");
@@ -130,24 +154,9 @@ FC_API fc_status ssm_conv_fwd(const void* u, const float* dt, const float* lambd
   FC_REQUIRE(workspace && aligned(workspace, 256), FC_EINVAL, "workspace must be non-null and 256-byte aligned");
   FC_REQUIRE(ws_bytes >= ssm_conv_workspace(H, L), FC_EINVAL, "workspace too small: %zu < %zu bytes", ws_bytes,
              ssm_conv_workspace(H, L));
-  float* f = (float*)workspace;
-  cudaStream_t st = (cudaStream_t)stream;
-  const fc::SsmArgs none{nullptr, nullptr, nullptr, nullptr, 0};
-  if (fc::fftconv_tc_supported(L, dtype)) {  // filter kernel, then the tensor-core convolution
-    s = cuda_status(fc::launch_ssm_gen(dt, lambda, Bp, Cp, H, N, L, f, st), "ssm_conv_fwd: filter launch");
-    if (s != FC_OK) return s;
-    return cuda_status(fc::launch_fftconv_tc(u, f, D, y, B, H, L, dtype, true, st),
-                       "ssm_conv_fwd: tensor-core conv launch");
-  }
-  if (L >= 1024 && N > 64) {  // filter generated inside the convolution kernel (no tensor-core generator)
-    const fc::SsmArgs sp{dt, (const float2*)lambda, (const float2*)Bp, (const float2*)Cp, N};
-    return cuda_status(fc::launch_fftconv(u, nullptr, L, sp, D, y, B, H, L, L, 1, dtype, st),
-                       "ssm_conv_fwd: fused launch");
-  }
-  s = cuda_status(fc::launch_ssm_gen(dt, lambda, Bp, Cp, H, N, L, f, st), "ssm_conv_fwd: filter launch");
-  if (s != FC_OK) return s;
-  return cuda_status(fc::launch_fftconv(u, f, L, none, D, y, B, H, L, L, 1, dtype, st),
-                     "ssm_conv_fwd: conv launch");
+  return cuda_status(fc::run_ssm_conv(u, dt, lambda, Bp, Cp, D, y, B, H, L, N, (float*)workspace, dtype,
+                                       (cudaStream_t)stream),
+                     "ssm_conv_fwd launch");
 }
 
 // workspace layout: [f_T: H*T floats][s: B*H*C*N complex][x: B*H*C*N complex], each 256-aligned
@@ -246,8 +255,10 @@ FC_API fc_status h3_mixer_fwd(const void* q, const void* k, const void* v, const
                      "h3_mixer launch");
 }
 
-FC_TEST_API unsigned int fc_debug_tc_timeouts(void) {
+FC_API unsigned int fc_tc_timeouts(void) {
   return fc::mixer_tc_timeouts() + fc::fftconv_tc_timeouts() + fc::statepass_tc_timeouts() + fc::gen_tc_timeouts();
 }
+
+FC_TEST_API unsigned int fc_debug_tc_timeouts(void) { return fc_tc_timeouts(); }
 
 }  // extern "C"

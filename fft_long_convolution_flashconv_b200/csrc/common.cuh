@@ -7,7 +7,50 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace fc {
+
+// ---- per-device launch setup, cached so that repeated calls do not repeat
+// runtime queries.  Devices with an ordinal >= 64 are served uncached.
+inline int current_device() {
+  int d = 0;
+  cudaGetDevice(&d);
+  return d;
+}
+
+// Number of SMs of the current device.
+inline int num_sms() {
+  static std::atomic<int> cache[64];
+  const int d = current_device();
+  if (d >= 0 && d < 64) {
+    const int c = cache[d].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || n < 1) n = 1;
+  if (d >= 0 && d < 64) cache[d].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+// Opt the kernel Kern in to `bytes` of dynamic shared memory once per device
+// (one cache per kernel instantiation; requests are monotone per kernel).
+template <auto Kern>
+cudaError_t smem_optin(size_t bytes) {
+  static std::atomic<unsigned long long> done{0};
+  static std::atomic<size_t> max_bytes[64];
+  const int d = current_device();
+  const bool cacheable = d >= 0 && d < 64;
+  if (cacheable && (done.load(std::memory_order_acquire) >> d & 1ull) &&
+      max_bytes[d].load(std::memory_order_relaxed) >= bytes)
+    return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess && cacheable) {
+    max_bytes[d].store(bytes, std::memory_order_relaxed);
+    done.fetch_or(1ull << d, std::memory_order_release);
+  }
+  return e;
+}
 
 // Debug-build bounds checks (-DFC_CHECK): a failed check records
 // (site << 48 | index) in a per-file device word and the access is skipped.

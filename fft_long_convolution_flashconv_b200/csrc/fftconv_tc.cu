@@ -465,16 +465,10 @@ static cudaError_t fftconv_tc_t(const void* u, const float* f, const float* D, v
                                 cudaStream_t st) {
   auto kern = fftconv_tc_kernel<T>;
   const size_t smem = sizeof(TcSmem);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = smem_optin<fftconv_tc_kernel<T>>(smem);
   if (e != cudaSuccess) return e;
-  static int num_sms = 0;
-  if (num_sms == 0) {
-    int dev = 0;
-    e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-  }
-  const int grid = H < 2 * num_sms ? H : 2 * num_sms;
+  const int sms = num_sms();
+  const int grid = H < 2 * sms ? H : 2 * sms;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThr);

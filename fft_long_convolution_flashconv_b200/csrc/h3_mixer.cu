@@ -133,7 +133,7 @@ static cudaError_t mixer_t(const void* q, const void* k, const void* v, const fl
                            const float* D, void* o, int B, int L, int heads, int S, cudaStream_t st) {
   const size_t smem = sizeof(float) * ((size_t)2 * kMixHD * kMixLd + (size_t)2 * kMixT * kMixLd + 2 * kMixT);
   auto kern = h3_mixer_kernel<T>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = smem_optin<h3_mixer_kernel<T>>(smem);
   if (e != cudaSuccess) return e;
   dim3 grid((L + kMixT - 1) / kMixT, heads, B);
   kern<<<grid, kMixThreads, smem, st>>>((const T*)q, (const T*)k, (const T*)v, Cs, f, D, (T*)o, L, heads, S);

@@ -334,7 +334,7 @@ static cudaError_t mixer_tc_t(const void* q, const void* k, const void* v, const
   if (e != cudaSuccess) return e;
   const size_t smem = sizeof(MixSmem) + 1024;
   auto kern = h3_mixer_tc_kernel<T>;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = smem_optin<h3_mixer_tc_kernel<T>>(smem);
   if (e != cudaSuccess) return e;
   dim3 grid((L + kT - 1) / kT, heads, B);
   kern<<<grid, kThr, smem, st>>>((const T*)q, (const T*)kt, (const T*)v, f, D, (T*)o, L, heads);

@@ -17,6 +17,12 @@ struct SsmArgs {
   int N;
 };
 
+// ssm_conv_fwd's dispatch: filter generation into f (H x L floats of scratch),
+// then the fused convolution (tensor cores where supported).
+cudaError_t run_ssm_conv(const void* u, const float* dt, const float* lambda, const float* Bp, const float* Cp,
+                         const float* D, void* y, int B, int H, int L, int N, float* f, int dtype,
+                         cudaStream_t st);
+
 cudaError_t launch_ssm_gen(const float* dt, const float* lam, const float* Bp, const float* Cp, int H, int N, int L,
                            float* f, cudaStream_t st);
 

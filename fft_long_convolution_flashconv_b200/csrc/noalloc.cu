@@ -69,6 +69,7 @@ FC_API fc_status ssm_conv_fwd_noalloc(const void* u, const float* dt, const floa
   if (L < 16 || L > 8192 || (L & (L - 1)) != 0)
     return na_fail(FC_EUNSUPPORTED, "L must be a power of two in [16, 8192]");
   if (N > 1024 || H > 65535) return na_fail(FC_EUNSUPPORTED, "N must be <= 1024 and H <= 65535");
+  if (B > (1 << 30)) return na_fail(FC_EUNSUPPORTED, "B must be <= 2^30");
   if ((size_t)H * (size_t)L > kNoAllocFilterFloats)
     return na_fail(FC_EUNSUPPORTED,
                    "H * L exceeds the fixed scratch of ssm_conv_fwd_noalloc (1,048,576 filter values); "
@@ -80,13 +81,11 @@ FC_API fc_status ssm_conv_fwd_noalloc(const void* u, const float* dt, const floa
   float* f = nullptr;
   cudaError_t e = noalloc_scratch(&f);
   if (e != cudaSuccess) return na_fail(FC_ECUDA, "could not resolve the scratch array on this device");
-  cudaStream_t st = (cudaStream_t)stream;
-  // the whole H x L filter is rewritten before it is read: nothing needs clearing
-  e = fc::launch_ssm_gen(dt, lambda, Bp, Cp, H, N, L, f, st);
-  if (e != cudaSuccess) return na_fail(FC_ECUDA, "filter launch failed");
-  const fc::SsmArgs none{nullptr, nullptr, nullptr, nullptr, 0};
-  e = fc::launch_fftconv(u, f, L, none, D, y, B, H, L, L, 1, dtype, st);
-  if (e != cudaSuccess) return na_fail(FC_ECUDA, "convolution launch failed");
+  // the same kernels as ssm_conv_fwd, with the library array as the filter
+  // scratch; the whole H x L filter is rewritten before it is read, so nothing
+  // needs clearing
+  e = fc::run_ssm_conv(u, dt, lambda, Bp, Cp, D, y, B, H, L, N, f, dtype, (cudaStream_t)stream);
+  if (e != cudaSuccess) return na_fail(FC_ECUDA, "launch failed");
   return FC_OK;
 }
 

@@ -309,7 +309,7 @@ cudaError_t launch_ssm_gen(const float* dt, const float* lam, const float* Bp, c
     const bool short_rows = L <= kGUnitTaps / 2;
     auto kern = short_rows ? ssm_gen_tc_kernel<true> : ssm_gen_tc_kernel<false>;
     const size_t smem = short_rows ? GenLayout<true>::bytes : GenLayout<false>::bytes;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = short_rows ? smem_optin<ssm_gen_tc_kernel<true>>(smem) : smem_optin<ssm_gen_tc_kernel<false>>(smem);
     if (e != cudaSuccess) return e;
     dim3 grid((units + kGUnits - 1) / kGUnits, H);
     kern<<<grid, kGThr, smem, st>>>(dt, reinterpret_cast<const float2*>(lam), reinterpret_cast<const float2*>(Bp),
@@ -318,7 +318,7 @@ cudaError_t launch_ssm_gen(const float* dt, const float* lam, const float* Bp, c
   }
 
   const int tiles = (L + kGenTile - 1) / kGenTile;
-  cudaError_t e = cudaFuncSetAttribute(ssm_gen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGenSmem);
+  cudaError_t e = smem_optin<ssm_gen_kernel>(kGenSmem);
   if (e != cudaSuccess) return e;
   dim3 grid(tiles, H);
   ssm_gen_kernel<<<grid, kGenThreads, kGenSmem, st>>>(dt, reinterpret_cast<const float2*>(lam),

@@ -236,7 +236,7 @@ static cudaError_t sp_tail(const void* u, const float* dt, const float* lam, con
   if (Tc > kSpMaxT || Tc < 1) return cudaErrorInvalidValue;
   const int C = L / Tc;
   const size_t smem1 = sizeof(float) * kSpMaxT + sizeof(float2) * (kSpBL * kSpNB + 4 * kSpNB);
-  cudaError_t e = cudaFuncSetAttribute(sp_state_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
+  cudaError_t e = smem_optin<sp_state_kernel<T>>(smem1);
   if (e != cudaSuccess) return e;
   sp_state_kernel<T><<<dim3(H, B), kSpThr, smem1, st>>>((const T*)u, dt, (const float2*)lam, (const float2*)Bp, H,
                                                          L, N, Tc, (float2*)s_ws);
@@ -249,7 +249,7 @@ static cudaError_t sp_tail(const void* u, const float* dt, const float* lam, con
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t smem3 = sizeof(float2) * ((size_t)kSpNB * kSpBL + 2 * (size_t)(kSpMaxNH + 1) * kSpNB);
-  e = cudaFuncSetAttribute(sp_corr_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3);
+  e = smem_optin<sp_corr_kernel<T>>(smem3);
   if (e != cudaSuccess) return e;
   sp_corr_kernel<T><<<dim3(H, B), kSpThr, smem3, st>>>((T*)y, dt, (const float2*)lam, (const float2*)Cp,
                                                         (const float2*)x_ws, H, L, N, Tc);

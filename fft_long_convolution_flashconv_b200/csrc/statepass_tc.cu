@@ -417,13 +417,13 @@ static cudaError_t sp_tc_t(const void* u, void* y, const float* dt, const float*
   if (!corr) {
     const size_t smem = sizeof(StateSmem<NC>) + 1024;
     auto kern = sp_state_tc_kernel<T, NC>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = smem_optin<sp_state_tc_kernel<T, NC>>(smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, kThr, smem, st>>>((const T*)u, dt, (const float2*)lam, (const float2*)Bp, H, L, N, (float2*)s_ws);
   } else {
     const size_t smem = sizeof(CorrSmem<NC>) + 1024;
     auto kern = sp_corr_tc_kernel<T, NC>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = smem_optin<sp_corr_tc_kernel<T, NC>>(smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, kThr, smem, st>>>((T*)y, dt, (const float2*)lam, (const float2*)Cp, (const float2*)x_ws, H, L, N,
                                    c_begin);

@@ -11,24 +11,35 @@
  * --------------------------------------
  *  - Every array pointer is caller-owned DEVICE memory on the current CUDA
  *    device, unless a comment says otherwise.  The library never allocates
- *    device memory; scratch space is passed in as `workspace`.
+ *    device memory; scratch space is passed in as `workspace`.  The one
+ *    exception is ssm_conv_fwd_noalloc (below), whose scratch is a fixed
+ *    array compiled into the library.
  *  - Sequences are row-major B x H x L (t contiguous); the H3 mixer's q, k, v,
  *    o are B x L x (heads*head_dim) (channel contiguous).
  *  - Complex arrays are interleaved (re, im) float32 pairs.
  *  - SSM parameters and filters are float32 whatever the I/O dtype.
- *  - I/O dtype: FC_F32, FC_F16 or FC_BF16 (u, y, q, k, v, o).  Arithmetic is
- *    float32 throughout (fp32 accumulate); the one rounding to a 16-bit I/O
- *    dtype is round-to-nearest-even at the store.
+ *  - I/O dtype: FC_F32, FC_F16 or FC_BF16 (u, y, q, k, v, o).  Accumulation
+ *    is float32 everywhere.  With FC_F32 I/O every step runs in float32 on
+ *    the CUDA cores and the output is rounded once.  With 16-bit I/O some
+ *    intermediates are rounded to 16-bit tensor-core operands; each entry
+ *    point states which.  All 16-bit outputs are rounded to nearest even.
  *  - u/y/q/k/v/o and filter pointers must be 16-byte aligned; parameter
  *    arrays 4-byte aligned (8-byte for complex).
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
- *    stream).  Calls are asynchronous on that stream, stateless, and safe to
- *    issue from several host threads.
+ *    stream).  Calls are asynchronous on that stream, keep no state between
+ *    calls (except ssm_conv_fwd_noalloc's shared array), and may be issued
+ *    from several host threads.
  *  - Return value: FC_OK, or a negative fc_status.  Argument errors are found
  *    on the host before anything is launched (nothing is written).  Launch
  *    errors come back as FC_ECUDA; faults during execution surface at the
  *    caller's next synchronisation.  fc_last_error() gives a message for the
  *    last failure on the calling host thread.
+ *  - Tensor-core kernels wait on their own matrix-multiply completions with a
+ *    bound of two seconds.  A block whose wait runs out (never seen in
+ *    normal operation) stops, frees its tensor memory and leaves its part of
+ *    the output unwritten; the call has already returned FC_OK.  Such events
+ *    are counted on the device; fc_tc_timeouts() reads the count (after the
+ *    caller's synchronisation), so a caller can detect an incomplete result.
  */
 #ifndef FLASHCONV_B200_H
 #define FLASHCONV_B200_H
@@ -64,6 +75,13 @@ FC_API const char* fc_status_string(int status);
 /* Message describing the last failing call on this host thread ("" if none). */
 FC_API const char* fc_last_error(void);
 
+/* Number of tensor-core blocks, over every kernel of the library on the
+ * current device since it was loaded, that gave up waiting for a
+ * matrix-multiply completion and left their part of an output unwritten
+ * (see the conventions above).  0 in normal operation.  Synchronises with
+ * the device (it reads a device counter). */
+FC_API unsigned int fc_tc_timeouts(void);
+
 /* ssm_kernel_gen -- diagonal-SSM convolution filter (A1).
  * H3 blog "The Convolution Connection": unrolling the recurrence gives the
  * filter f = [CB, CAB, CA^2B, ...]; H3 summary section 2 "Convolutional view".
@@ -73,7 +91,11 @@ FC_API const char* fc_last_error(void);
  * Arguments: dt (H floats); lambda, Bp, Cp (H x N complex); f_out (H x L
  * floats, written).  Limits: H >= 1, 1 <= N <= 1024, 1 <= L <= 1048576.
  * A^k is evaluated with its phase k*dt*Im(lambda) reduced modulo 2 pi in
- * double precision, so long, slowly decaying filters keep their phase. */
+ * double precision, so long, slowly decaying filters keep their phase.
+ * Precision: for N <= 64 the sum over modes is a tensor-core GEMM whose
+ * operands (tables of powers and of 2 C B A^k) are each split into a 16-bit
+ * high part and a 16-bit remainder (about 22 significant bits), summed in
+ * float32; for N > 64 it is float32 on the CUDA cores. */
 FC_API fc_status ssm_kernel_gen(const float* dt, const float* lambda, const float* Bp, const float* Cp,
                                 int H, int N, int L, float* f_out, void* stream);
 
@@ -86,13 +108,22 @@ FC_API fc_status ssm_kernel_gen(const float* dt, const float* lambda, const floa
  * evaluated as IFFT_{2L}(FFT_{2L}(pad u) * FFT_{2L}(pad f)) cropped to t < L.
  * u, y: B x H x L in `dtype`; f: H x L floats (any real filter, not only an
  * SSM's); D: H floats.  Limits: L a power of two, 16 <= L <= 8192; B, H >= 1.
- * u and y may not overlap. */
+ * u and y may not overlap.
+ * Precision: FC_F32 and every L without a tensor-core kernel: float32
+ * FFTs on the CUDA cores, one rounding at the store.  16-bit I/O at
+ * L = 1024 runs the block-FFT stages on the tensor cores: the filter (with D
+ * added to its tap 0) is rounded to the I/O type; the DFT-128 stages take
+ * their data operand in the I/O type (exact for u); the DFT-16 stages take
+ * float16 operands scaled by 1/32, which stay finite for |u| <= 32752; the
+ * inverse stage's input is rounded to the I/O type; accumulation is float32
+ * and y is rounded once at the store. */
 FC_API fc_status fftconv_fwd(const void* u, const float* f, const float* D, void* y,
                              int B, int H, int L, fc_dtype dtype, void* stream);
 
 /* ssm_conv_fwd -- ssm_kernel_gen followed by fftconv_fwd in one call (the
  * filter is regenerated on the device every call).  workspace must hold
- * ssm_conv_workspace(H, L) bytes (the H x L filter). */
+ * ssm_conv_workspace(H, L) bytes (the H x L filter).  Precision: that of
+ * ssm_kernel_gen followed by that of fftconv_fwd. */
 FC_API size_t ssm_conv_workspace(int H, int L);
 FC_API fc_status ssm_conv_fwd(const void* u, const float* dt, const float* lambda, const float* Bp,
                               const float* Cp, const float* D, void* y, int B, int H, int L, int N,
@@ -113,7 +144,14 @@ FC_API fc_status ssm_conv_fwd(const void* u, const float* dt, const float* lambd
  * split one sequence over several calls by passing state_out as the next
  * call's state_in.  workspace: at least fftconv_statepass_workspace(...)
  * bytes, 256-byte aligned.  Limits: chunk a power of two, 16 <= chunk <=
- * 8192, L % chunk == 0, 1 <= N <= 256. */
+ * 8192, L % chunk == 0, 1 <= N <= 256.
+ * Precision: the chunk convolutions run on the CUDA cores in float32 and are
+ * stored in the I/O type; the initial-state term is then added to the stored
+ * values and the sum rounded again (two roundings for chunks after the
+ * first).  With 16-bit I/O, chunk in {2048, 4096, 8192} and N <= 64, the end
+ * states and the initial-state term are tensor-core GEMMs against tables
+ * split hi/lo into 16-bit parts (about 22 significant bits; 16 for the
+ * bfloat16 u-side table), with u as an exact 16-bit operand. */
 FC_API size_t fftconv_statepass_workspace(int B, int H, int L, int N, int chunk);
 FC_API fc_status fftconv_statepass(const void* u, const float* dt, const float* lambda, const float* Bp,
                                    const float* Cp, const float* D, void* y, int B, int H, int L, int N,
@@ -132,7 +170,11 @@ FC_API fc_status fftconv_statepass(const void* u, const float* dt, const float* 
  * (heads*head_dim) x shift_len floats; dt, D: heads floats; lambda, Bp, Cp:
  * heads x N complex.  workspace: at least h3_mixer_workspace(...) bytes
  * (the per-head filters and, for 16-bit I/O, the shift-SSM output k~).
- * Limits: head_dim == 64, 1 <= shift_len <= 8, 1 <= L <= 65536, 1 <= N <= 1024. */
+ * Limits: head_dim == 64, 1 <= shift_len <= 8, 1 <= L <= 65536, 1 <= N <= 1024.
+ * Precision: FC_F32 runs in float32 on the CUDA cores.  16-bit I/O runs the
+ * two GEMMs per tile on the tensor cores: k~ is stored in the I/O type, the
+ * Toeplitz-weighted scores (f[t-s] + D [s == t]) (q_t . k~_s) are rounded to
+ * the I/O type before they multiply v; accumulation is float32. */
 FC_API size_t h3_mixer_workspace(int B, int L, int heads, int head_dim, int N);
 FC_API fc_status h3_mixer_fwd(const void* q, const void* k, const void* v, const float* Cshift,
                               const float* dt, const float* lambda, const float* Bp, const float* Cp,
@@ -160,9 +202,14 @@ FC_API fc_status h3_mixer_fwd(const void* q, const void* k, const void* v, const
  *    earlier call reaches a result, but calls that can overlap on the GPU
  *    (different streams with no ordering between them) race on the array and
  *    must not be issued that way.
- *  - Arguments, other limits and results as ssm_conv_fwd (the filter is
- *    generated by a separate kernel, then convolved).  On failure the message
- *    is in ssm_conv_noalloc_last_error() (per host thread). */
+ *  - Arguments, other limits, kernels and results as ssm_conv_fwd: the same
+ *    filter kernel and the same convolution kernel (the tensor-core one for
+ *    16-bit I/O at L = 1024, as in ssm_conv_fwd), so the two entry points
+ *    return identical bits.  On failure the message is in
+ *    ssm_conv_noalloc_last_error() (per host thread).
+ *  - Like every tensor-core call, a block whose completion wait runs out
+ *    leaves its part of y unwritten (fc_tc_timeouts() counts it); such a y
+ *    may then hold an earlier call's values. */
 FC_API fc_status ssm_conv_fwd_noalloc(const void* u, const float* dt, const float* lambda, const float* Bp,
                                       const float* Cp, const float* D, void* y, int B, int H, int L, int N,
                                       fc_dtype dtype, void* stream);

@@ -263,6 +263,41 @@ def test_mixer_delta_filter():
         assert np.max(np.abs(o[:, :, sl] - want)) < 1e-13 * np.max(np.abs(want))
 
 
+# ---------------------------------------------------------------- parity metric
+def test_golden_row_rel_err(golden):
+    """The parity metric against hand-worked values: per-row max-norm, max over rows."""
+    g = golden("hand_worked_row_rel_err.txt")
+    ref = np.array(g["ref"]).reshape(3, 3)
+    y = np.array(g["y"]).reshape(3, 3)
+    for r in range(3):
+        assert O.row_rel_err(y[r:r + 1], ref[r:r + 1]) == pytest.approx(g["row_err"][r], rel=1e-15)
+    assert O.row_rel_err(y, ref) == pytest.approx(g["metric"][0], rel=1e-15)
+    assert O.row_rel_err(y[2:], ref[2:]) == pytest.approx(g["zero_row_only"][0], rel=1e-15)
+    # 3-d arrays (B x H x L) reduce along the last axis the same way
+    assert O.row_rel_err(y.reshape(1, 3, 3), ref.reshape(1, 3, 3)) == pytest.approx(g["metric"][0], rel=1e-15)
+    # a tolerance check built on it must separate the rows: scaling one row's error up
+    # by 10x moves the metric, scaling the quiet row does not
+    y2 = y.copy()
+    y2[1, 1] = 20.0
+    assert O.row_rel_err(y2, ref) == pytest.approx(0.2, rel=1e-15)
+
+
+def test_row_rel_err_planted_mistakes(golden):
+    """Plausible mistakes in the metric (made here, on copies) must miss the golden value."""
+    g = golden("hand_worked_row_rel_err.txt")
+    ref = np.array(g["ref"]).reshape(3, 3)
+    y = np.array(g["y"]).reshape(3, 3)
+    want = g["metric"][0]
+    global_den = float(np.max(np.abs(y - ref)) / np.max(np.abs(ref)))
+    wrong_axis = float(np.max(np.max(np.abs(y - ref), axis=0) / np.maximum(np.max(np.abs(ref), axis=0), 1e-300)))
+    per_row = np.max(np.abs(y - ref), axis=-1) / np.where(np.max(np.abs(ref), axis=-1) == 0, 1.0,
+                                                         np.max(np.abs(ref), axis=-1))
+    mean_rows = float(np.mean(per_row))
+    for bad in (global_den, wrong_axis, mean_rows):
+        assert abs(bad - want) > 1e-3, bad
+    assert O.row_rel_err(y, ref) == pytest.approx(want, rel=1e-15)
+
+
 # ---------------------------------------------------------------- planted mistakes
 def test_pins_catch_planted_mistakes(golden):
     """Mutated copies of oracle steps (made here, on the CPU) must fail a pin."""
