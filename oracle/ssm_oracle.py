@@ -38,6 +38,7 @@ __all__ = [
     "as_complex", "discretize", "ssm_powers", "ssm_filter", "ssm_filter_from_A",
     "causal_conv_direct", "ssm_recurrence", "statepass_chunked",
     "shift_ssm", "h3_mixer_outer", "h3_mixer_toeplitz", "row_rel_err",
+    "causal_conv_bwd", "h3_mixer_recurrent",
 ]
 
 
@@ -281,3 +282,77 @@ def row_rel_err(y, ref, axis=-1) -> float:
     den = np.max(np.abs(ref), axis=axis)
     den = np.where(den == 0, 1.0, den)
     return float(np.max(num / den))
+
+
+def causal_conv_bwd(dy, u, f, D):
+    """Gradients of the causal convolution y = f * u + D u (all fp64).
+
+    H3 summary, appendix C.1 "Backward Pass": the backward pass of the FFT
+    convolution is again a convolution (with the conjugate transform), plus
+    the gradient of the D u term.  For a loss whose gradient with respect to
+    y is dy, differentiating y[b,h,t] = sum_{s<=t} f[h,t-s] u[b,h,s] + D[h]
+    u[b,h,t] term by term gives
+      du[b,h,s] = sum_{t>=s} f[h,t-s] dy[b,h,t] + D[h] dy[b,h,s]   (anti-causal)
+      df[h,k]   = sum_b sum_{t>=k} dy[b,h,t] u[b,h,t-k]             (k < L)
+      dD[h]     = sum_b sum_t dy[b,h,t] u[b,h,t]
+    written out here as the plain sums (numpy.correlate is the direct sum).
+    Returns (du, df, dD).
+    """
+    dy = np.asarray(dy, dtype=np.float64)
+    u = np.asarray(u, dtype=np.float64)
+    f = np.asarray(f, dtype=np.float64)
+    D = np.asarray(D, dtype=np.float64)
+    B, H, L = u.shape
+    du = np.empty_like(u)
+    df = np.zeros((H, L), dtype=np.float64)
+    dD = np.zeros(H, dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            # du[s] = sum_k f[k] dy[s + k]  (k = t - s >= 0, s + k < L)
+            du[b, h] = np.correlate(dy[b, h], f[h, :L], mode="full")[L - 1:] + D[h] * dy[b, h]
+            # df[k] = sum_t dy[t] u[t - k]
+            df[h] += np.correlate(dy[b, h], u[b, h], mode="full")[L - 1:]
+            dD[h] += float(np.dot(dy[b, h], u[b, h]))
+    return du, df, dD
+
+
+def h3_mixer_recurrent(q, k, v, Cshift, A, Bc, Cc, D, heads: int) -> np.ndarray:
+    """H3 mixer evaluated token by token in its recurrent form (tiny shapes).
+
+    H3 summary, section 2 "Recurrent view" (each output from the current state;
+    generation runs step by step) with the H3 layer of the H3 blog, "The
+    Solution, Part 1".  Per token t, per head h, channels i, j < hd:
+      k~_t      = sum_{j<S} Cshift[:, j] k_{t-j}          (shift SSM: its state is
+                                                          the last S-1 inputs)
+      X_ij,t    = A_h X_ij,t-1 + B_h k~_i,t v_j,t          (N complex modes)
+      y_ij,t    = 2 Re(sum_n C_h,n X_ij,t,n) + D_h k~_i,t v_j,t
+      o_j,t     = sum_i q_i,t y_ij,t
+    A, Bc, Cc: (heads, N) complex; D: (heads,).  Returns o (B, L, heads*hd).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    Cs = np.asarray(Cshift, dtype=np.float64)
+    A = np.asarray(A, dtype=np.complex128)
+    Bc = np.asarray(Bc, dtype=np.complex128)
+    Cc = np.asarray(Cc, dtype=np.complex128)
+    D = np.asarray(D, dtype=np.float64)
+    Bn, L, dm = q.shape
+    hd = dm // heads
+    S = Cs.shape[1]
+    N = A.shape[1]
+    o = np.zeros_like(q)
+    for b in range(Bn):
+        hist = np.zeros((S, dm))                      # hist[j] = k_{t-j}
+        X = np.zeros((heads, hd, hd, N), dtype=np.complex128)
+        for t in range(L):
+            hist = np.roll(hist, 1, axis=0)
+            hist[0] = k[b, t]
+            kt = np.sum(Cs.T * hist, axis=0)          # sum_j Cs[c, j] k_{t-j}[c]
+            for h in range(heads):
+                sl = slice(h * hd, (h + 1) * hd)
+                kv = np.outer(kt[sl], v[b, t, sl])    # kv[i, j]
+                X[h] = A[h][None, None, :] * X[h] + Bc[h][None, None, :] * kv[:, :, None]
+                y = 2.0 * np.real(np.sum(Cc[h][None, None, :] * X[h], axis=2)) + D[h] * kv
+                o[b, t, sl] = q[b, t, sl] @ y
+    return o

@@ -298,6 +298,107 @@ def test_row_rel_err_planted_mistakes(golden):
     assert O.row_rel_err(y, ref) == pytest.approx(want, rel=1e-15)
 
 
+# ---------------------------------------------------------------- backward pass
+def test_golden_conv_bwd(golden):
+    g = golden("hand_worked_conv_bwd.txt")
+    u = np.array(g["u"]).reshape(1, 1, -1)
+    f = np.array(g["f"]).reshape(1, -1)
+    D = np.array(g["D"])
+    dy = np.array(g["dy"]).reshape(1, 1, -1)
+    assert np.allclose(O.causal_conv_direct(u, f, D)[0, 0], g["y"], rtol=0, atol=1e-15)
+    du, df, dD = O.causal_conv_bwd(dy, u, f, D)
+    assert np.array_equal(du[0, 0], np.array(g["du"]))
+    assert np.array_equal(df[0], np.array(g["df"]))
+    assert dD[0] == g["dD"][0]
+
+
+def test_conv_bwd_by_linearity_brute_force():
+    """y is linear in u and jointly linear in (f, D), so each gradient entry is
+    exactly <dy, y(basis vector)>: brute force over every entry on a tiny case."""
+    rng = np.random.default_rng(11)
+    B, H, L = 2, 2, 7
+    u = rng.normal(size=(B, H, L))
+    f = rng.normal(size=(H, L))
+    D = rng.normal(size=H)
+    dy = rng.normal(size=(B, H, L))
+    du, df, dD = O.causal_conv_bwd(dy, u, f, D)
+    for b in range(B):
+        for h in range(H):
+            for s in range(L):
+                e = np.zeros_like(u)
+                e[b, h, s] = 1.0
+                assert abs(np.sum(dy * O.causal_conv_direct(e, f, D)) - du[b, h, s]) < 1e-12
+    for h in range(H):
+        for k in range(L):
+            e = np.zeros_like(f)
+            e[h, k] = 1.0
+            assert abs(np.sum(dy * O.causal_conv_direct(u, e, np.zeros(H))) - df[h, k]) < 1e-12
+        e = np.zeros(H)
+        e[h] = 1.0
+        assert abs(np.sum(dy * O.causal_conv_direct(u, np.zeros_like(f), e)) - dD[h]) < 1e-12
+
+
+def test_conv_bwd_adjoint_and_fft_route():
+    rng = np.random.default_rng(12)
+    B, H, L = 3, 4, 64
+    u = rng.normal(size=(B, H, L))
+    f = rng.normal(size=(H, L)) * np.exp(-np.arange(L) / 9.0)
+    D = rng.normal(size=H)
+    dy = rng.normal(size=(B, H, L))
+    du, df, dD = O.causal_conv_bwd(dy, u, f, D)
+    lhs = np.sum(dy * O.causal_conv_direct(u, f, D))
+    assert abs(lhs - np.sum(du * u)) < 1e-10 * abs(lhs)
+    assert abs(lhs - (np.sum(df * f) + np.sum(dD * D))) < 1e-10 * abs(lhs)
+    # library route: with 2L zero padding, du is the circular correlation
+    # irfft(conj(F) DY) and df the batch sum of irfft(DY conj(U)), cropped to L
+    M = 2 * L
+    F = np.fft.rfft(f, M)
+    U = np.fft.rfft(u, M)
+    DY = np.fft.rfft(dy, M)
+    du_fft = np.fft.irfft(np.conj(F)[None] * DY, M)[..., :L] + D[None, :, None] * dy
+    df_fft = np.sum(np.fft.irfft(DY * np.conj(U), M)[..., :L], axis=0)
+    assert np.max(np.abs(du_fft - du)) < 1e-12 * np.max(np.abs(du))
+    assert np.max(np.abs(df_fft - df)) < 1e-12 * np.max(np.abs(df))
+
+
+def test_conv_bwd_planted_mistakes(golden):
+    g = golden("hand_worked_conv_bwd.txt")
+    u = np.array(g["u"])
+    f = np.array(g["f"])
+    dy = np.array(g["dy"])
+    D = g["D"][0]
+    L = len(u)
+    # causal instead of anti-causal du
+    du_causal = np.convolve(dy, f)[:L] + D * dy
+    assert not np.allclose(du_causal, g["du"])
+    # D term dropped from du
+    du_noD = np.correlate(dy, f, mode="full")[L - 1:]
+    assert not np.allclose(du_noD, g["du"])
+    # df with the lag sign flipped (u leading dy)
+    df_flip = np.correlate(u, dy, mode="full")[L - 1:]
+    assert not np.allclose(df_flip, g["df"])
+
+
+def test_mixer_recurrent_equals_outer_form():
+    """The token-by-token recurrent mixer (the decode path) equals the
+    convolutional outer-product form, whose filter is f = 2 Re(C A^k B)."""
+    rng = np.random.default_rng(13)
+    Bn, L, heads, hd, N, S = 2, 9, 2, 3, 4, 3
+    q, k, v = (rng.normal(size=(Bn, L, heads * hd)) for _ in range(3))
+    Cs = rng.normal(size=(heads * hd, S))
+    A = 0.9 * np.exp(1j * rng.uniform(0, np.pi, size=(heads, N)))
+    Bc = rng.normal(size=(heads, N)) + 1j * rng.normal(size=(heads, N))
+    Cc = rng.normal(size=(heads, N)) + 1j * rng.normal(size=(heads, N))
+    D = rng.normal(size=heads)
+    o_rec = O.h3_mixer_recurrent(q, k, v, Cs, A, Bc, Cc, D, heads)
+    f = O.ssm_filter_from_A(A, Bc, Cc, L)
+    o_conv = O.h3_mixer_outer(q, k, v, Cs, f, D, heads)
+    assert np.max(np.abs(o_rec - o_conv)) < 1e-12 * np.max(np.abs(o_conv))
+    # planted: read the output before the state update (x_{t-1} instead of x_t)
+    o_lag = O.h3_mixer_outer(q, k, v, Cs, np.concatenate([np.zeros((heads, 1)), f[:, :-1]], 1), D, heads)
+    assert np.max(np.abs(o_lag - o_conv)) > 1e-3 * np.max(np.abs(o_conv))
+
+
 # ---------------------------------------------------------------- planted mistakes
 def test_pins_catch_planted_mistakes(golden):
     """Mutated copies of oracle steps (made here, on the CPU) must fail a pin."""
