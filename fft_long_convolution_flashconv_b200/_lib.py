@@ -23,7 +23,12 @@ SIGNATURES = {
     "fc_tc_timeouts": (ctypes.c_uint, []),
     "ssm_kernel_gen": (_i, [_fp, _fp, _fp, _fp, _i, _i, _i, _fp, _vp]),
     "fftconv_fwd": (_i, [_vp, _fp, _fp, _vp, _i, _i, _i, _i, _vp]),
+    "fftconv_bwd": (_i, [_vp, _vp, _fp, _fp, _vp, _fp, _fp, _i, _i, _i, _i, _vp]),
     "ssm_conv_workspace": (_sz, [_i, _i]),
+    "ssm_decode_step": (_i, [_vp, _fp, _fp, _fp, _fp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _vp]),
+    "h3_decode_state_bytes": (_sz, [_i, _i, _i, _i]),
+    "h3_mixer_decode_step": (_i, [_vp, _vp, _vp, _vp, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _vp, _i, _i, _i, _i, _i,
+                                  ctypes.c_longlong, _i, _vp]),
     "ssm_conv_fwd": (_i, [_vp, _fp, _fp, _fp, _fp, _fp, _vp, _i, _i, _i, _i, _vp, _sz, _i, _vp]),
     "fftconv_statepass_workspace": (_sz, [_i, _i, _i, _i, _i]),
     "fftconv_statepass": (_i, [_vp, _fp, _fp, _fp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _fp, _fp, _vp, _sz,

@@ -91,6 +91,59 @@ def fftconv_fwd(u: torch.Tensor, f: torch.Tensor, D: torch.Tensor,
     return out
 
 
+def fftconv_bwd(dy: torch.Tensor, u: torch.Tensor, f: torch.Tensor, D: torch.Tensor, need_du: bool = True,
+                need_dfilter: bool = True):
+    """Gradients of y = causal_conv(u, f) + D u given dy; returns (du, df, dD)
+    (None for the parts not requested)."""
+    lib = _lib.load()
+    B, H, L = dy.shape
+    f, D = _f32(f), _f32(D)
+    du = torch.empty_like(dy) if need_du else None
+    df = torch.empty((H, L), dtype=torch.float32, device=dy.device) if need_dfilter else None
+    dD = torch.empty((H,), dtype=torch.float32, device=dy.device) if need_dfilter else None
+    check(lib.fftconv_bwd(_ptr(dy), _ptr(u), _ptr(f), _ptr(D), _ptr(du), _ptr(df), _ptr(dD), B, H, L, _dtype(dy),
+                          _stream()), "fftconv_bwd")
+    return du, df, dD
+
+
+def ssm_decode_step(u, x, dt, lam, Bp, Cp, D, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """T tokens of the recurrent view; u: B x H x T; x: B x H x N x 2 float32
+    state, updated in place.  Returns y (B x H x T)."""
+    lib = _lib.load()
+    B, H, Tn = u.shape
+    dt, lam, Bp, Cp, D = _f32(dt), _cpx(lam), _cpx(Bp), _cpx(Cp), _f32(D)
+    N = lam.shape[1]
+    if x.dtype != torch.float32 or tuple(x.shape) != (B, H, N, 2) or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float32 B x H x N x 2 tensor")
+    if out is None:
+        out = torch.empty_like(u)
+    check(lib.ssm_decode_step(_ptr(u), _ptr(x), _ptr(dt), _ptr(lam), _ptr(Bp), _ptr(Cp), _ptr(D), _ptr(out), B, H,
+                              N, Tn, _dtype(u), _stream()), "ssm_decode_step")
+    return out
+
+
+def h3_decode_state(B, heads, head_dim, N, device) -> torch.Tensor:
+    """Zeroed recurrent state of the H3 mixer (B x heads x hd x hd x N x 2 float32)."""
+    return torch.zeros((B, heads, head_dim, head_dim, N, 2), dtype=torch.float32, device=device)
+
+
+def h3_mixer_decode_step(q, k, v, kring, state, Cshift, dt, lam, Bp, Cp, D, heads: int, pos: int,
+                         out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One token (q, k, v: B x d_model) of the H3 mixer in recurrent form."""
+    lib = _lib.load()
+    B, dm = q.shape
+    hd = dm // heads
+    Cshift, dt, lam, Bp, Cp, D = _f32(Cshift), _f32(dt), _cpx(lam), _cpx(Bp), _cpx(Cp), _f32(D)
+    N = lam.shape[1]
+    S = Cshift.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    check(lib.h3_mixer_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(kring), _ptr(state), _ptr(Cshift), _ptr(dt),
+                                   _ptr(lam), _ptr(Bp), _ptr(Cp), _ptr(D), _ptr(out), B, heads, hd, N, S, pos,
+                                   _dtype(q), _stream()), "h3_mixer_decode_step")
+    return out
+
+
 def ssm_conv_workspace_bytes(H: int, L: int) -> int:
     return int(_lib.load().ssm_conv_workspace(H, L))
 

@@ -62,6 +62,11 @@ cudaError_t run_ssm_conv(const void* u, const float* dt, const float* lambda, co
     if (e != cudaSuccess) return e;
     return launch_fftconv_tc(u, f, D, y, B, H, L, dtype, true, st);
   }
+  if (fftconv_tcl_supported(L, dtype)) {
+    e = launch_ssm_gen(dt, lambda, Bp, Cp, H, N, L, f, st);
+    if (e != cudaSuccess) return e;
+    return launch_fftconv_tcl(u, f, L, D, y, B, H, L, L, 1, dtype, true, false, st);
+  }
   if (L >= 1024 && N > 64) {  // filter generated inside the convolution kernel (no tensor-core generator)
     const SsmArgs sp{dt, (const float2*)lambda, (const float2*)Bp, (const float2*)Cp, N};
     return launch_fftconv(u, nullptr, L, sp, D, y, B, H, L, L, 1, dtype, st);
@@ -128,9 +133,53 @@ FC_API fc_status fftconv_fwd(const void* u, const float* f, const float* D, void
   if (fc::fftconv_tc_supported(L, dtype))
     return cuda_status(fc::launch_fftconv_tc(u, f, D, y, B, H, L, dtype, false, (cudaStream_t)stream),
                        "fftconv_fwd (tensor cores) launch");
+  if (fc::fftconv_tcl_supported(L, dtype))
+    return cuda_status(fc::launch_fftconv_tcl(u, f, L, D, y, B, H, L, L, 1, dtype, false, false, (cudaStream_t)stream),
+                       "fftconv_fwd (tensor cores) launch");
   const fc::SsmArgs none{nullptr, nullptr, nullptr, nullptr, 0};
   return cuda_status(fc::launch_fftconv(u, f, L, none, D, y, B, H, L, L, 1, dtype, (cudaStream_t)stream),
                      "fftconv_fwd launch");
+}
+
+FC_API fc_status fftconv_bwd(const void* dy, const void* u, const float* f, const float* D, void* du, float* df,
+                             float* dD, int B, int H, int L, fc_dtype dtype, void* stream) {
+  g_err[0] = 0;
+  FC_REQUIRE(du || (df && dD), FC_EINVAL, "nothing to compute: du is null and df / dD are null");
+  FC_REQUIRE(L >= 1, FC_EINVAL, "L must be >= 1");
+  FC_REQUIRE((df == nullptr) == (dD == nullptr), FC_EINVAL, "df and dD must both be given or both be null");
+  FC_REQUIRE(dtype_ok(dtype), FC_EINVAL, "unknown dtype %d", dtype);
+  FC_REQUIRE(B >= 1 && H >= 1, FC_EINVAL, "B, H must be >= 1 (got %d, %d)", B, H);
+  FC_REQUIRE(B <= (1 << 30), FC_EUNSUPPORTED, "B = %d > 2^30", B);
+  FC_REQUIRE(dy && aligned(dy, 16), FC_EINVAL, "dy must be non-null and 16-byte aligned");
+  fc_status s = FC_OK;
+  if (du) {  // du may not overlap dy
+    s = check_conv_io(dy, du, B, H, L, dtype);
+    if (s != FC_OK) return s;
+  }
+  FC_REQUIRE(pow2(L) && L >= 16 && L <= 8192, FC_EUNSUPPORTED,
+             "fftconv_bwd: L must be a power of two in [16, 8192] (got %d)", L);
+  FC_REQUIRE(H <= 65535, FC_EUNSUPPORTED, "H = %d > 65535", H);
+  if (du) FC_REQUIRE(f && D && aligned(f, 16) && aligned(D, 4), FC_EINVAL, "du needs f (16-byte aligned) and D");
+  if (df)
+    FC_REQUIRE(u && aligned(u, 16) && aligned(df, 4) && aligned(dD, 4), FC_EINVAL,
+               "df needs u (16-byte aligned); df, dD 4-byte aligned");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (du) {
+    s = fc::fftconv_tc_supported(L, dtype)
+            ? cuda_status(fc::launch_fftconv_tc(dy, f, D, du, B, H, L, dtype, false, st, true),
+                          "fftconv_bwd: du (tensor cores) launch")
+        : fc::fftconv_tcl_supported(L, dtype)
+            ? cuda_status(fc::launch_fftconv_tcl(dy, f, L, D, du, B, H, L, L, 1, dtype, false, true, st),
+                          "fftconv_bwd: du (tensor cores) launch")
+            : cuda_status(fc::launch_fftconv(dy, f, L, fc::SsmArgs{nullptr, nullptr, nullptr, nullptr, 0}, D, du, B,
+                                             H, L, L, 1, dtype, st, 1),
+                          "fftconv_bwd: du launch");
+    if (s != FC_OK) return s;
+  }
+  if (df) {
+    s = cuda_status(fc::launch_fftconv_dfilter(dy, u, df, dD, B, H, L, dtype, st), "fftconv_bwd: df launch");
+  }
+  return s;
 }
 
 FC_API size_t ssm_conv_workspace(int H, int L) {
@@ -199,8 +248,11 @@ FC_API fc_status fftconv_statepass(const void* u, const float* dt, const float* 
   s = cuda_status(fc::launch_ssm_gen(dt, lambda, Bp, Cp, H, N, chunk, fT, st), "statepass: filter launch");
   if (s != FC_OK) return s;
   const fc::SsmArgs none{nullptr, nullptr, nullptr, nullptr, 0};
-  s = cuda_status(fc::launch_fftconv(u, fT, chunk, none, D, y, B, H, L, chunk, C, dtype, st),
-                  "statepass: chunk conv launch");
+  s = fc::fftconv_tcl_supported(chunk, dtype)
+          ? cuda_status(fc::launch_fftconv_tcl(u, fT, chunk, D, y, B, H, L, chunk, C, dtype, true, false, st),
+                        "statepass: chunk conv (tensor cores) launch")
+          : cuda_status(fc::launch_fftconv(u, fT, chunk, none, D, y, B, H, L, chunk, C, dtype, st),
+                        "statepass: chunk conv launch");
   if (s != FC_OK) return s;
   return cuda_status(fc::launch_statepass_tail(u, dt, lambda, Bp, Cp, y, B, H, L, N, chunk, state_in, state_out,
                                                s_ws, x_ws, dtype, st),
@@ -255,8 +307,54 @@ FC_API fc_status h3_mixer_fwd(const void* q, const void* k, const void* v, const
                      "h3_mixer launch");
 }
 
+FC_API fc_status ssm_decode_step(const void* u, float* x, const float* dt, const float* lambda, const float* Bp,
+                                 const float* Cp, const float* D, void* y, int B, int H, int N, int T,
+                                 fc_dtype dtype, void* stream) {
+  g_err[0] = 0;
+  FC_REQUIRE(T >= 1, FC_EINVAL, "T must be >= 1 (got %d)", T);
+  fc_status s = check_conv_io(u, y, B, H, T, dtype);
+  if (s != FC_OK) return s;
+  s = check_params(dt, lambda, Bp, Cp);
+  if (s != FC_OK) return s;
+  FC_REQUIRE(D && aligned(D, 4), FC_EINVAL, "null or misaligned D");
+  FC_REQUIRE(x && aligned(x, 8), FC_EINVAL, "x must be non-null and 8-byte aligned");
+  FC_REQUIRE(N >= 1 && N <= 1024, FC_EUNSUPPORTED, "N must be in [1, 1024] (got %d)", N);
+  FC_REQUIRE(H <= 65535, FC_EUNSUPPORTED, "H = %d > 65535", H);
+  return cuda_status(fc::launch_ssm_decode(u, x, dt, lambda, Bp, Cp, D, y, B, H, N, T, dtype, (cudaStream_t)stream),
+                     "ssm_decode_step launch");
+}
+
+FC_API size_t h3_decode_state_bytes(int B, int heads, int head_dim, int N) {
+  if (B < 1 || heads < 1 || head_dim < 1 || N < 1) return 0;
+  return (size_t)B * heads * head_dim * head_dim * N * 2 * sizeof(float);
+}
+
+FC_API fc_status h3_mixer_decode_step(const void* q, const void* k, const void* v, void* kring, float* state,
+                                      const float* Cshift, const float* dt, const float* lambda, const float* Bp,
+                                      const float* Cp, const float* D, void* o, int B, int heads, int head_dim,
+                                      int N, int shift_len, long long pos, fc_dtype dtype, void* stream) {
+  g_err[0] = 0;
+  FC_REQUIRE(dtype_ok(dtype), FC_EINVAL, "unknown dtype %d", dtype);
+  FC_REQUIRE(q && k && v && o && state, FC_EINVAL, "null q, k, v, o or state");
+  FC_REQUIRE(aligned(q, 16) && aligned(k, 16) && aligned(v, 16) && aligned(o, 16) && aligned(state, 8), FC_EINVAL,
+             "q, k, v, o must be 16-byte aligned, state 8-byte aligned");
+  FC_REQUIRE(Cshift && D && aligned(Cshift, 4) && aligned(D, 4), FC_EINVAL, "null or misaligned Cshift / D");
+  fc_status s = check_params(dt, lambda, Bp, Cp);
+  if (s != FC_OK) return s;
+  FC_REQUIRE(B >= 1 && heads >= 1 && pos >= 0, FC_EINVAL, "B, heads must be >= 1 and pos >= 0");
+  FC_REQUIRE(head_dim >= 1 && head_dim <= 64, FC_EUNSUPPORTED, "head_dim must be in [1, 64] (got %d)", head_dim);
+  FC_REQUIRE(shift_len >= 1 && shift_len <= 8, FC_EUNSUPPORTED, "shift_len must be in [1, 8] (got %d)", shift_len);
+  FC_REQUIRE(shift_len == 1 || (kring && aligned(kring, 16)), FC_EINVAL, "kring must be non-null and 16-byte aligned");
+  FC_REQUIRE(N >= 1 && N <= 1024, FC_EUNSUPPORTED, "N must be in [1, 1024]");
+  FC_REQUIRE(heads <= 65535 && B <= 65535, FC_EUNSUPPORTED, "B or heads > 65535");
+  return cuda_status(fc::launch_h3_decode(q, k, v, kring, state, Cshift, dt, lambda, Bp, Cp, D, o, B, heads,
+                                          head_dim, N, shift_len, pos, dtype, (cudaStream_t)stream),
+                     "h3_mixer_decode_step launch");
+}
+
 FC_API unsigned int fc_tc_timeouts(void) {
-  return fc::mixer_tc_timeouts() + fc::fftconv_tc_timeouts() + fc::statepass_tc_timeouts() + fc::gen_tc_timeouts();
+  return fc::mixer_tc_timeouts() + fc::fftconv_tc_timeouts() + fc::fftconv_tcl_timeouts() +
+         fc::statepass_tc_timeouts() + fc::gen_tc_timeouts();
 }
 
 FC_TEST_API unsigned int fc_debug_tc_timeouts(void) { return fc_tc_timeouts(); }

@@ -5,7 +5,7 @@
 
 namespace fc {
 template cudaError_t launch_fftconv_dispatch<__nv_bfloat16>(const __nv_bfloat16*, const float*, int, SsmArgs, const float*, __nv_bfloat16*,
-                                               int, int, long long, int, int, cudaStream_t);
+                                               int, int, long long, int, int, int, cudaStream_t);
 }  // namespace fc
 
 FC_CHECK_READER(fc_check_fftconv_bf16)

@@ -5,7 +5,7 @@
 
 namespace fc {
 template cudaError_t launch_fftconv_dispatch<float>(const float*, const float*, int, SsmArgs, const float*, float*,
-                                               int, int, long long, int, int, cudaStream_t);
+                                               int, int, long long, int, int, int, cudaStream_t);
 }  // namespace fc
 
 FC_CHECK_READER(fc_check_fftconv_f32)

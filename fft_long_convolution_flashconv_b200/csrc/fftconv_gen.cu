@@ -8,10 +8,10 @@ template <typename T>
 cudaError_t launch_fftconv_gen(const T* u, const float* f, int fstride, SsmArgs sp, const float* D, T* y, int B,
                                int H, long long Lrow, int Lc, int C, cudaStream_t st) {
   switch (Lc) {
-    case 1024: return launch_fftconv_t<T, 11, true>(u, f, fstride, sp, D, y, B, H, Lrow, C, st);
-    case 2048: return launch_fftconv_t<T, 12, true>(u, f, fstride, sp, D, y, B, H, Lrow, C, st);
-    case 4096: return launch_fftconv_t<T, 13, true>(u, f, fstride, sp, D, y, B, H, Lrow, C, st);
-    case 8192: return launch_fftconv_t<T, 14, true>(u, f, fstride, sp, D, y, B, H, Lrow, C, st);
+    case 1024: return launch_fftconv_t<T, 11, true>(u, f, fstride, sp, D, y, B, H, Lrow, C, 0, st);
+    case 2048: return launch_fftconv_t<T, 12, true>(u, f, fstride, sp, D, y, B, H, Lrow, C, 0, st);
+    case 4096: return launch_fftconv_t<T, 13, true>(u, f, fstride, sp, D, y, B, H, Lrow, C, 0, st);
+    case 8192: return launch_fftconv_t<T, 14, true>(u, f, fstride, sp, D, y, B, H, Lrow, C, 0, st);
     default: return cudaErrorInvalidValue;
   }
 }

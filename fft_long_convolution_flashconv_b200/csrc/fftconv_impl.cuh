@@ -157,7 +157,8 @@ struct GenGeom {
 template <typename T, int LOGM, bool GEN>
 __global__ void __launch_bounds__(ConvGeom<LOGM>::THREADS, ConvGeom<LOGM>::MINB)
     fftconv_kernel(const T* __restrict__ u, const float* __restrict__ f, int fstride, SsmArgs sp,
-                   const float* __restrict__ D, T* __restrict__ y, int B, int H, long long Lrow, int C) {
+                   const float* __restrict__ D, T* __restrict__ y, int B, int H, long long Lrow, int C,
+                   int conj_filter) {
   using P = FftPlan<LOGM>;
   using Gm = ConvGeom<LOGM>;
   constexpr int M = P::M, TG = P::TG, RM = P::RMAX, R0 = P::R0, RL = P::RLAST;
@@ -271,13 +272,16 @@ __global__ void __launch_bounds__(ConvGeom<LOGM>::THREADS, ConvGeom<LOGM>::MINB)
       }
       fft_fwd<LOGM>(v, buf, tid, tw);
       constexpr float inv_m = 1.0f / (float)M;
+      // conj_filter: multiply by conj(F^) instead, i.e. correlate with f (the
+      // input gradient of the convolution)
+      const float im_sign = conj_filter ? -inv_m : inv_m;
 #pragma unroll
       for (int i = 0; i < PERL; ++i) {
         const int j = tid + i * TG;
 #pragma unroll
         for (int r = 0; r < RL; ++r) {
           const int m = j + r * (M / RL);
-          if (m <= M / 2) fh[m] = make_float2(v[i * RL + r].x * inv_m, v[i * RL + r].y * inv_m);
+          if (m <= M / 2) fh[m] = make_float2(v[i * RL + r].x * inv_m, v[i * RL + r].y * im_sign);
         }
       }
       hcur = h;
@@ -331,7 +335,7 @@ cudaError_t launch_fftconv_gen(const T* u, const float* f, int fstride, SsmArgs 
 
 template <typename T, int LOGM, bool GEN>
 static cudaError_t launch_fftconv_t(const T* u, const float* f, int fstride, SsmArgs sp, const float* D, T* y,
-                                    int B, int H, long long Lrow, int C, cudaStream_t st) {
+                                    int B, int H, long long Lrow, int C, int conj_filter, cudaStream_t st) {
   using Gm = ConvGeom<LOGM>;
   auto kern = fftconv_kernel<T, LOGM, GEN>;
   const size_t smem = Gm::smem_bytes;
@@ -353,25 +357,27 @@ static cudaError_t launch_fftconv_t(const T* u, const float* f, int fstride, Ssm
   } else {
     grid = (H + Gm::G - 1) / Gm::G;
   }
-  kern<<<(unsigned)grid, Gm::THREADS, smem, st>>>(u, f, fstride, sp, D, y, B, H, Lrow, C);
+  kern<<<(unsigned)grid, Gm::THREADS, smem, st>>>(u, f, fstride, sp, D, y, B, H, Lrow, C, conj_filter);
   return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t launch_fftconv_dispatch(const T* u, const float* f, int fstride, SsmArgs sp, const float* D,
-                                           T* y, int B, int H, long long Lrow, int Lc, int C, cudaStream_t st) {
+                                           T* y, int B, int H, long long Lrow, int Lc, int C, int conj_filter,
+                                           cudaStream_t st) {
   if (sp.dt != nullptr) return launch_fftconv_gen<T>(u, f, fstride, sp, D, y, B, H, Lrow, Lc, C, st);
+  
   switch (Lc) {
-    case 16: return launch_fftconv_t<T, 5, false>(u, f, fstride, sp, D, y, B, H, Lrow, C, st);
-    case 32: return launch_fftconv_t<T, 6, false>(u, f, fstride, sp, D, y, B, H, Lrow, C, st);
-    case 64: return launch_fftconv_t<T, 7, false>(u, f, fstride, sp, D, y, B, H, Lrow, C, st);
-    case 128: return launch_fftconv_t<T, 8, false>(u, f, fstride, sp, D, y, B, H, Lrow, C, st);
-    case 256: return launch_fftconv_t<T, 9, false>(u, f, fstride, sp, D, y, B, H, Lrow, C, st);
-    case 512: return launch_fftconv_t<T, 10, false>(u, f, fstride, sp, D, y, B, H, Lrow, C, st);
-    case 1024: return launch_fftconv_t<T, 11, false>(u, f, fstride, sp, D, y, B, H, Lrow, C, st);
-    case 2048: return launch_fftconv_t<T, 12, false>(u, f, fstride, sp, D, y, B, H, Lrow, C, st);
-    case 4096: return launch_fftconv_t<T, 13, false>(u, f, fstride, sp, D, y, B, H, Lrow, C, st);
-    case 8192: return launch_fftconv_t<T, 14, false>(u, f, fstride, sp, D, y, B, H, Lrow, C, st);
+    case 16: return launch_fftconv_t<T, 5, false>(u, f, fstride, sp, D, y, B, H, Lrow, C, conj_filter, st);
+    case 32: return launch_fftconv_t<T, 6, false>(u, f, fstride, sp, D, y, B, H, Lrow, C, conj_filter, st);
+    case 64: return launch_fftconv_t<T, 7, false>(u, f, fstride, sp, D, y, B, H, Lrow, C, conj_filter, st);
+    case 128: return launch_fftconv_t<T, 8, false>(u, f, fstride, sp, D, y, B, H, Lrow, C, conj_filter, st);
+    case 256: return launch_fftconv_t<T, 9, false>(u, f, fstride, sp, D, y, B, H, Lrow, C, conj_filter, st);
+    case 512: return launch_fftconv_t<T, 10, false>(u, f, fstride, sp, D, y, B, H, Lrow, C, conj_filter, st);
+    case 1024: return launch_fftconv_t<T, 11, false>(u, f, fstride, sp, D, y, B, H, Lrow, C, conj_filter, st);
+    case 2048: return launch_fftconv_t<T, 12, false>(u, f, fstride, sp, D, y, B, H, Lrow, C, conj_filter, st);
+    case 4096: return launch_fftconv_t<T, 13, false>(u, f, fstride, sp, D, y, B, H, Lrow, C, conj_filter, st);
+    case 8192: return launch_fftconv_t<T, 14, false>(u, f, fstride, sp, D, y, B, H, Lrow, C, conj_filter, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -108,7 +108,7 @@ template <> struct Op<__nv_bfloat16> {
 template <typename T>
 __global__ void __launch_bounds__(kThr, 2) fftconv_tc_kernel(const T* __restrict__ u, const float* __restrict__ f,
                                                              const float* __restrict__ D, T* __restrict__ y, int B,
-                                                             int H) {
+                                                             int H, int conj_filter) {
   extern __shared__ __align__(1024) uint8_t smraw[];
   TcSmem& sm = *reinterpret_cast<TcSmem*>(smraw);
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -327,8 +327,10 @@ __global__ void __launch_bounds__(kThr, 2) fftconv_tc_kernel(const T* __restrict
       float xr[16], xi[16];
       tc::tmem_ld16x2_wait(tmem + lane_off, tmem + lane_off + 16u, xr, xi);
       constexpr float sc = 32.0f * 32.0f / (float)kM;  // undo the 1/32 of stage B, x32 for the pairs, 1/M
+      // conj_filter: conj(F^), i.e. correlation with f (the input gradient)
+      const float sci = conj_filter ? -sc : sc;
 #pragma unroll
-      for (int k2 = 0; k2 < kN2; ++k2) fh[k2] = make_float2(xr[k2] * sc, xi[k2] * sc);
+      for (int k2 = 0; k2 < kN2; ++k2) fh[k2] = make_float2(xr[k2] * sc, xi[k2] * sci);
     }
 #pragma unroll 1
     for (int p = grp; p < P; p += 2) {
@@ -462,7 +464,7 @@ __global__ void __launch_bounds__(kThr, 2) fftconv_tc_kernel(const T* __restrict
 
 template <typename T>
 static cudaError_t fftconv_tc_t(const void* u, const float* f, const float* D, void* y, int B, int H, bool pdl,
-                                cudaStream_t st) {
+                                cudaStream_t st, bool conj_filter) {
   auto kern = fftconv_tc_kernel<T>;
   const size_t smem = sizeof(TcSmem);
   cudaError_t e = smem_optin<fftconv_tc_kernel<T>>(smem);
@@ -479,16 +481,16 @@ static cudaError_t fftconv_tc_t(const void* u, const float* f, const float* D, v
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kern, (const T*)u, f, D, (T*)y, B, H);
+  return cudaLaunchKernelEx(&cfg, kern, (const T*)u, f, D, (T*)y, B, H, conj_filter ? 1 : 0);
 }
 
 bool fftconv_tc_supported(int L, int dtype) { return L == kL && (dtype == 1 || dtype == 2); }
 
 cudaError_t launch_fftconv_tc(const void* u, const float* f, const float* D, void* y, int B, int H, int L, int dtype,
-                              bool after_filter_kernel, cudaStream_t st) {
+                              bool after_filter_kernel, cudaStream_t st, bool conj_filter) {
   if (!fftconv_tc_supported(L, dtype)) return cudaErrorInvalidValue;
-  return dtype == 1 ? fftconv_tc_t<__half>(u, f, D, y, B, H, after_filter_kernel, st)
-                    : fftconv_tc_t<__nv_bfloat16>(u, f, D, y, B, H, after_filter_kernel, st);
+  return dtype == 1 ? fftconv_tc_t<__half>(u, f, D, y, B, H, after_filter_kernel, st, conj_filter)
+                    : fftconv_tc_t<__nv_bfloat16>(u, f, D, y, B, H, after_filter_kernel, st, conj_filter);
 }
 
 unsigned int fftconv_tc_timeouts() {

@@ -29,8 +29,11 @@ cudaError_t launch_ssm_gen(const float* dt, const float* lam, const float* Bp, c
 // dtype: 0 f32, 1 f16, 2 bf16.  Lc = transform half-length (chunk), C chunks per row.
 // sp.dt != nullptr: generate the filter from the SSM parameters inside the
 // kernel (Lc >= 1024); otherwise read it from f (row stride fstride).
+// conj_filter = 1 multiplies by the conjugate filter spectrum: the result is
+// then the anti-causal correlation sum_{t>=s} f[t-s] u[t] + D u[s] (the input
+// gradient of the convolution); not with generated filters.
 cudaError_t launch_fftconv(const void* u, const float* f, int fstride, SsmArgs sp, const float* D, void* y, int B,
-                           int H, long long Lrow, int Lc, int C, int dtype, cudaStream_t st);
+                           int H, long long Lrow, int Lc, int C, int dtype, cudaStream_t st, int conj_filter = 0);
 
 cudaError_t launch_statepass_tail(const void* u, const float* dt, const float* lam, const float* Bp,
                                   const float* Cp, void* y, int B, int H, int L, int N, int T,
@@ -59,6 +62,17 @@ cudaError_t launch_h3_mixer_tc(const void* q, const void* k, const void* v, cons
 // Number of tensor-core CTAs that gave up waiting for an MMA (0 in normal operation).
 unsigned int mixer_tc_timeouts();
 
+// Recurrent view: Tn tokens of x <- A x + B u_t, y_t = 2 Re(C x) + D u_t per
+// (b, h) row; u, y: B x H x Tn; x: B x H x N complex, updated in place.
+cudaError_t launch_ssm_decode(const void* u, float* x, const float* dt, const float* lam, const float* Bp,
+                              const float* Cp, const float* D, void* y, int B, int H, int N, int Tn, int dtype,
+                              cudaStream_t st);
+// One token of the H3 mixer in recurrent form (state, kring updated in place).
+cudaError_t launch_h3_decode(const void* q, const void* k, const void* v, void* kring, float* state, const float* Cs,
+                             const float* dt, const float* lam, const float* Bp, const float* Cp, const float* D,
+                             void* o, int B, int heads, int hd, int N, int S, long long pos, int dtype,
+                             cudaStream_t st);
+
 // Tensor-core fused FFT convolution (block-FFT stages as tcgen05 GEMMs).
 bool fftconv_tc_supported(int L, int dtype);
 // after_filter_kernel: f is written by the kernel launched just before on the
@@ -66,8 +80,24 @@ bool fftconv_tc_supported(int L, int dtype);
 // dependent (prologue overlapped; the filter is read only after that kernel
 // has completed).
 cudaError_t launch_fftconv_tc(const void* u, const float* f, const float* D, void* y, int B, int H, int L, int dtype,
-                              bool after_filter_kernel, cudaStream_t st);
+                              bool after_filter_kernel, cudaStream_t st, bool conj_filter = false);
+
+// Gradient of the convolution with respect to the filter and D:
+//   df[h,k] = sum_b sum_{t>=k} dy[b,h,t] u[b,h,t-k],  dD[h] = sum_b sum_t dy u
+// (CUDA cores, L a power of two in [16, 8192]).
+cudaError_t launch_fftconv_dfilter(const void* dy, const void* u, float* df, float* dD, int B, int H, int L,
+                                   int dtype, cudaStream_t st);
 unsigned int fftconv_tc_timeouts();
+
+// Tensor-core fused FFT convolution for transform half-lengths Lc = 2048,
+// 4096, 8192 (16-bit I/O), rows laid out as launch_fftconv (C chunks of Lc
+// per row of Lrow).  after_filter_kernel as launch_fftconv_tc; conj_filter as
+// launch_fftconv.
+bool fftconv_tcl_supported(int Lc, int dtype);
+cudaError_t launch_fftconv_tcl(const void* u, const float* f, int fstride, const float* D, void* y, int B, int H,
+                               long long Lrow, int Lc, int C, int dtype, bool after_filter_kernel, bool conj_filter,
+                               cudaStream_t st);
+unsigned int fftconv_tcl_timeouts();
 // Tensor-core filter generation CTAs that gave up waiting for an MMA.
 unsigned int gen_tc_timeouts();
 

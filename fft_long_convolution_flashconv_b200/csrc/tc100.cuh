@@ -176,5 +176,24 @@ __device__ __forceinline__ void tmem_ld16x2_wait(uint32_t ta, uint32_t tb, float
   }
 }
 
+// Split TMEM loads: issue several loads, then one wait, then tmem_regs_ready on
+// every destination register (an empty volatile asm that takes the register
+// as an in/out operand, so no use of it can be scheduled before the wait).
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, uint32_t* u) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld2(uint32_t taddr, uint32_t* u) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];" : "=r"(u[0]), "=r"(u[1]) : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* u) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_regs_ready(uint32_t& r) { asm volatile("" : "+r"(r)); }
+
 }  // namespace tc
 }  // namespace fc

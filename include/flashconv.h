@@ -120,6 +120,23 @@ FC_API fc_status ssm_kernel_gen(const float* dt, const float* lambda, const floa
 FC_API fc_status fftconv_fwd(const void* u, const float* f, const float* D, void* y,
                              int B, int H, int L, fc_dtype dtype, void* stream);
 
+/* fftconv_bwd -- backward pass of fftconv_fwd (gradients of a loss with
+ * respect to u, f and D, given its gradient dy with respect to y).
+ * H3 summary, appendix C.1 "Backward Pass": the backward of the FFT
+ * convolution is computed with FFTs too, with conjugate transforms, plus the
+ * D u term's gradient.  Differentiating y = f * u + D u:
+ *   du[b,h,s] = sum_{t>=s} f[h,t-s] dy[b,h,t] + D[h] dy[b,h,s]   (conj(F^) . DY)
+ *   df[h,k]   = sum_b sum_{t>=k} dy[b,h,t] u[b,h,t-k]            (sum_b DY . conj(U))
+ *   dD[h]     = sum_b sum_t dy[b,h,t] u[b,h,t]
+ * dy, u, du: B x H x L in `dtype`; f: H x L floats; D, dD: H floats; df:
+ * H x L floats.  du may be NULL (then f and D may be NULL too); df and dD are
+ * given together or both NULL.  df and dD are overwritten, not accumulated.
+ * Limits as fftconv_fwd.  Precision: du is fftconv_fwd's kernel (same
+ * rounding) with the conjugate filter spectrum; df and dD are float32 FFTs
+ * and sums on the CUDA cores. */
+FC_API fc_status fftconv_bwd(const void* dy, const void* u, const float* f, const float* D, void* du, float* df,
+                             float* dD, int B, int H, int L, fc_dtype dtype, void* stream);
+
 /* ssm_conv_fwd -- ssm_kernel_gen followed by fftconv_fwd in one call (the
  * filter is regenerated on the device every call).  workspace must hold
  * ssm_conv_workspace(H, L) bytes (the H x L filter).  Precision: that of
@@ -181,6 +198,42 @@ FC_API fc_status h3_mixer_fwd(const void* q, const void* k, const void* v, const
                               const float* D, void* o, int B, int L, int heads, int head_dim, int N,
                               int shift_len, void* workspace, size_t ws_bytes, fc_dtype dtype,
                               void* stream);
+
+/* ssm_decode_step -- the recurrent view, for generation: T >= 1 tokens of
+ *   x <- A x + B u_t,   y_t = 2 Re sum_n C_n x_n + D u_t,   A = exp(dt lambda)
+ * H3 summary section 2 "Recurrent view" (each output from the current state
+ * and the new input, O(N) per token) and section 5 (generation runs step by
+ * step); H3 blog "Background" (x_i from x_{i-1} and u_i).
+ * u, y: B x H x T in `dtype` (T = 1 for one generated token); x: B x H x N
+ * complex float32 state, read and written in place (zero for an empty
+ * history; after a call it is the state after the last token, so calls
+ * chain).  Parameters as ssm_kernel_gen, D: H floats.  Limits: N <= 1024,
+ * H <= 65535.  Precision: float32 state and arithmetic, y rounded once. */
+FC_API fc_status ssm_decode_step(const void* u, float* x, const float* dt, const float* lambda, const float* Bp,
+                                 const float* Cp, const float* D, void* y, int B, int H, int N, int T,
+                                 fc_dtype dtype, void* stream);
+
+/* h3_mixer_decode_step -- one token of the H3 mixer (h3_mixer_fwd) in
+ * recurrent form, for generation.  H3 summary section 2 "Recurrent view" and
+ * section 5; H3 blog "The Solution, Part 1".  Per head h and channels i, j:
+ *   k~_i   = sum_{s<shift_len, s<=pos} Cshift[i,s] k_{pos-s,i}   (shift SSM)
+ *   X_ij  <- A_h X_ij + B_h k~_i v_j                                (N modes)
+ *   o_j    = sum_i q_i (2 Re sum_n C_h,n X_ij,n + D_h k~_i v_j)
+ * q, k, v, o: B x (heads*head_dim) in `dtype`, the token at position pos.
+ * kring: B x (shift_len-1) x (heads*head_dim) in `dtype`, the keys of the
+ * previous shift_len-1 tokens (slot p % (shift_len-1) holds position p; read
+ * only for positions >= 0, so it needs no initialisation; the call stores
+ * this token's keys into it; NULL allowed when shift_len == 1).  state:
+ * h3_decode_state_bytes(...) bytes = B x heads x head_dim x head_dim x N
+ * complex float32 ([b][head][i][j][n]), zero before position 0, updated in
+ * place.  Other parameters as h3_mixer_fwd.  Calls for consecutive positions
+ * must be ordered (same stream).  Limits: head_dim <= 64, shift_len <= 8,
+ * N <= 1024.  Precision: float32 state and arithmetic, o rounded once. */
+FC_API size_t h3_decode_state_bytes(int B, int heads, int head_dim, int N);
+FC_API fc_status h3_mixer_decode_step(const void* q, const void* k, const void* v, void* kring, float* state,
+                                      const float* Cshift, const float* dt, const float* lambda, const float* Bp,
+                                      const float* Cp, const float* D, void* o, int B, int heads, int head_dim,
+                                      int N, int shift_len, long long pos, fc_dtype dtype, void* stream);
 
 /* ssm_conv_fwd_noalloc -- ssm_conv_fwd for callers that cannot allocate
  * device memory.  The pages have no counterpart to this call.

@@ -290,3 +290,169 @@ def test_h3_mixer_cfg5_full_sampled():
     ts = np.unique(np.concatenate([[0, 1, 3, 63, 64, 65, 1023, 2047], rng.choice(2048, 40, replace=False)]))
     ref = _mixer_ref(mw, rows=rows, ts=ts)
     assert _head_err(o, ref, mw, rows, ts) < 2e-2
+
+
+# ------------------------------------------------------------------ (f)1 backward pass
+@pytest.mark.parametrize("B,H,L,dtype", [
+    (3, 5, 16, "f32"), (2, 3, 256, "f32"), (3, 4, 1024, "f32"), (2, 3, 8192, "f32"),
+    (3, 5, 1024, "f16"), (5, 6, 1024, "bf16"),          # du on the tensor-core conv
+    (2, 3, 512, "f16"), (2, 4, 4096, "bf16"), (1, 3, 8192, "f16"),
+])
+def test_fftconv_bwd(B, H, L, dtype):
+    """du, df, dD against the oracle's gradient sums (per-row max-norm; df per
+    channel, dD over channels)."""
+    wl = W.make_conv(B=B, H=H, L=L, N=16, dtype=dtype, seed=L + B, dt_range=("loguniform", -3.0, -1.0))
+    f32 = W.round_to(O.ssm_filter(wl.dt, wl.lam, wl.Bp, wl.Cp, L), "f32")
+    dy = W.round_to(np.random.default_rng(L).normal(size=(B, H, L)), dtype)
+    du, df, dD = api.fftconv_bwd(dev(dy, dtype), dev(wl.u, dtype), dev(f32), dev(wl.D))
+    rdu, rdf, rdD = O.causal_conv_bwd(dy, wl.u, f32, wl.D)
+    assert O.row_rel_err(host(du).reshape(-1, L), rdu.reshape(-1, L)) < TOL[dtype]
+    # df and dD come from the 16-bit inputs exactly and are float32 sums: fp32 tolerance
+    # scaled by the summation length
+    assert O.row_rel_err(host(df), rdf) < 1e-4 * max(1.0, np.log2(L * B) / 4)
+    assert np.max(np.abs(host(dD) - rdD)) < 1e-4 * np.max(np.abs(rdD)) * max(1.0, np.log2(L * B) / 4)
+
+
+def test_fftconv_bwd_parts_and_impulse():
+    """du alone and df alone give the same values as the full call; an impulse
+    dy at t0 gives du = f reversed in time up to t0 (bit-exact zeros after t0
+    are not required: the FFT leaves rounding noise) and df[k] = u[t0 - k]."""
+    B, H, L = 2, 3, 512
+    wl = W.make_conv(B=B, H=H, L=L, N=16, dtype="f32", seed=77)
+    f32 = W.round_to(O.ssm_filter(wl.dt, wl.lam, wl.Bp, wl.Cp, L), "f32")
+    dy = np.zeros((B, H, L))
+    t0 = 300
+    dy[:, :, t0] = 1.0
+    du, df, dD = api.fftconv_bwd(dev(dy), dev(wl.u), dev(f32), dev(wl.D))
+    du1, n1, n2 = api.fftconv_bwd(dev(dy), dev(wl.u), dev(f32), dev(wl.D), need_dfilter=False)
+    assert n1 is None and n2 is None
+    n3, df2, dD2 = api.fftconv_bwd(dev(dy), dev(wl.u), dev(f32), dev(wl.D), need_du=False)
+    assert n3 is None
+    assert torch.equal(du, du1) and torch.equal(df, df2) and torch.equal(dD, dD2)
+    want_du = np.zeros((B, H, L))
+    for s in range(t0 + 1):
+        want_du[:, :, s] = f32[None, :, t0 - s]
+    want_du[:, :, t0] += wl.D[None, :]
+    assert np.max(np.abs(host(du) - want_du)) < 1e-5 * np.max(np.abs(want_du))
+    want_df = np.zeros((H, L))
+    for k in range(t0 + 1):
+        want_df[:, k] = wl.u[:, :, t0 - k].sum(0)
+    assert np.max(np.abs(host(df) - want_df)) < 1e-5 * np.max(np.abs(want_df))
+
+
+# ------------------------------------------------------------------ (f)2 recurrent decode
+@pytest.mark.parametrize("B,H,N,dtype", [(2, 3, 16, "f32"), (3, 5, 64, "f32"), (2, 3, 200, "f32"),
+                                         (1, 2, 700, "f32"), (2, 4, 64, "f16"), (3, 2, 33, "bf16")])
+def test_ssm_decode_matches_recurrence(B, H, N, dtype):
+    """T tokens in one call, then single tokens chained through the state,
+    against the oracle recurrence over the whole sequence (outputs and the
+    final state)."""
+    L1, L2 = 37, 5
+    wl = W.make_conv(B=B, H=H, L=L1 + L2, N=N, dtype=dtype, seed=N + B)
+    dtt, lam, Bp, Cp, D = params(wl)
+    u = dev(wl.u, dtype)
+    x = torch.zeros((B, H, N, 2), dtype=torch.float32, device="cuda")
+    ys = [api.ssm_decode_step(u[..., :L1].contiguous(), x, dtt, lam, Bp, Cp, D)]
+    for t in range(L1, L1 + L2):
+        ys.append(api.ssm_decode_step(u[..., t:t + 1].contiguous(), x, dtt, lam, Bp, Cp, D))
+    y = host(torch.cat(ys, -1))
+    A, Bc, Cc = oracle_A(wl)
+    ref, xref = cref.ssm_recurrence(wl.u, A, Bc, Cc, wl.D.astype(np.float64))
+    assert O.row_rel_err(y.reshape(-1, L1 + L2), ref.reshape(-1, L1 + L2)) < TOL[dtype]
+    xg = host(x)
+    xg = xg[..., 0] + 1j * xg[..., 1]
+    assert np.max(np.abs(xg - xref)) < 1e-4 * np.max(np.abs(xref))
+
+
+@pytest.mark.parametrize("S,dtype", [(4, "f32"), (1, "f32"), (3, "f16"), (8, "bf16")])
+def test_h3_mixer_decode_matches_parallel_form(S, dtype):
+    """Token-by-token decode of the H3 mixer against the oracle's recurrent
+    form (pinned to the convolutional form) on every position."""
+    B, L, heads, hd, N = 2, 20, 2, 64, 8
+    mw = W.make_mixer(B=B, L=L, heads=heads, head_dim=hd, N=N, shift_len=S, dtype=dtype, seed=40 + S)
+    q, k, v = dev(mw.q, dtype), dev(mw.k, dtype), dev(mw.v, dtype)
+    Cs, dtt, lam, Bp, Cp, D = dev(mw.Cshift), dev(mw.dt), dev(mw.lam), dev(mw.Bp), dev(mw.Cp), dev(mw.D)
+    state = api.h3_decode_state(B, heads, hd, N, "cuda")
+    kring = torch.zeros((B, max(S - 1, 1), heads * hd), dtype=q.dtype, device="cuda")
+    outs = []
+    for t in range(L):
+        outs.append(api.h3_mixer_decode_step(q[:, t].contiguous(), k[:, t].contiguous(), v[:, t].contiguous(),
+                                             kring, state, Cs, dtt, lam, Bp, Cp, D, heads, t))
+    o = host(torch.stack(outs, 1))
+    A = O.discretize(mw.dt, mw.lam)
+    ref = O.h3_mixer_recurrent(mw.q, mw.k, mw.v, mw.Cshift, A, O.as_complex(mw.Bp), O.as_complex(mw.Cp), mw.D,
+                               heads)
+    err = 0.0
+    for b in range(B):
+        for h in range(heads):
+            sl = slice(h * hd, (h + 1) * hd)
+            err = max(err, float(np.max(np.abs(o[b, :, sl] - ref[b, :, sl])) / np.max(np.abs(ref[b, :, sl]))))
+    assert err < TOL[dtype], err
+
+
+# ------------------------------------------------------------------ tensor-core conv: layout and range edges
+@pytest.mark.parametrize("B,H,L,dtype", [(1, 200, 8192, "bf16"), (3, 300, 2048, "f16"), (2, 7, 4096, "bf16"),
+                                         (5, 160, 4096, "f16"), (2, 151, 8192, "f16")])
+def test_fftconv_tensor_core_long(B, H, L, dtype):
+    """L = 2048..8192 block-FFT conv: odd B, B = 1, and more channels than SMs
+    (CTA item ranges that start and end inside a channel)."""
+    wl = W.make_conv(B=B, H=H, L=L, N=16, dtype=dtype, seed=H + L, dt_range=("loguniform", -3.0, -1.0))
+    f32 = W.round_to(O.ssm_filter(wl.dt, wl.lam, wl.Bp, wl.Cp, L), "f32")
+    y = host(api.fftconv_fwd(dev(wl.u, dtype), dev(f32), dev(wl.D)))
+    rng = np.random.default_rng(H)
+    hs = np.unique(np.concatenate([rng.choice(H, min(H, 24), replace=False), [0, H - 1]]))
+    ref = cref.causal_conv(wl.u[:, hs], f32[hs], wl.D[hs].astype(np.float64))
+    assert O.row_rel_err(y[:, hs].reshape(-1, L), ref.reshape(-1, L)) < TOL[dtype]
+
+
+@pytest.mark.parametrize("L,dtype", [(1024, "f16"), (1024, "bf16"), (2048, "bf16"), (8192, "f16")])
+def test_fftconv_tensor_core_impulse_alignment(L, dtype):
+    """Impulses through the tensor-core paths (odd B, so one row has no pair
+    partner): u = delta at t0 gives y = f shifted by t0 plus D delta; the
+    argmax of |y - D delta| sits at t0 + argmax|f| and y is ~0 before t0."""
+    B, H = 3, 2
+    t0s = [0, 1, 15, 16, 511, L - 1]
+    rng = np.random.default_rng(L)
+    f = np.zeros((H, L))
+    f[:, :40] = rng.normal(size=(H, 40))
+    f[:, 7] = 5.0  # a unique peak at lag 7
+    f32 = W.round_to(f, "f32")
+    D = np.array([0.5, -0.25])
+    for t0 in t0s:
+        u = np.zeros((B, H, L))
+        u[:, :, t0] = 1.0
+        y = host(api.fftconv_fwd(dev(u, dtype), dev(f32), dev(D)))
+        for b in range(B):
+            for h in range(H):
+                want = np.zeros(L)
+                n = L - t0
+                want[t0:] = f32[h, :n]
+                want[t0] += D[h]
+                assert np.max(np.abs(y[b, h] - want)) < 2e-2 * 5.0, (t0, b, h)
+                if t0 + 7 < L:
+                    assert int(np.argmax(np.abs(y[b, h] - D[h] * u[b, h]))) == t0 + 7
+                if t0 > 0:
+                    assert np.max(np.abs(y[b, h, :t0])) < 2e-2 * 5.0
+
+
+@pytest.mark.parametrize("L", [1024, 8192])
+def test_fftconv_fp16_slow_filters_constant_step_and_large_inputs(L):
+    """fp16 I/O on the tensor-core paths with slow filters (dt ~ 1e-3): a
+    constant input, a step input and a random input near the |u| limit
+    (scaled so the outputs stay within fp16 range), against the oracle."""
+    B, H = 2, 4
+    wl = W.make_conv(B=B, H=H, L=L, N=64, dtype="f16", seed=3, dt_range=("loguniform", -3.0, -2.9))
+    f32 = W.round_to(O.ssm_filter(wl.dt, wl.lam, wl.Bp, wl.Cp, L), "f32")
+    gain = np.max(np.sum(np.abs(f32), axis=1)) + np.max(np.abs(wl.D))
+    amp = min(30000.0, 30000.0 / gain)
+    cases = {
+        "constant": np.full((B, H, L), amp),
+        "step": np.where(np.arange(L)[None, None, :] >= L // 3, amp, -0.5 * amp) * np.ones((B, H, 1)),
+        "large random": np.clip(np.random.default_rng(5).normal(size=(B, H, L)) * amp / 3, -amp, amp),
+    }
+    for name, u in cases.items():
+        u16 = W.round_to(u, "f16")
+        y = host(api.fftconv_fwd(dev(u16, "f16"), dev(f32), dev(wl.D)))
+        ref = cref.causal_conv(u16, f32, wl.D.astype(np.float64))
+        assert np.all(np.isfinite(y)), name
+        assert O.row_rel_err(y.reshape(-1, L), ref.reshape(-1, L)) < 2e-2, name
