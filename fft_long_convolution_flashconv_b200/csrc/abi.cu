@@ -34,6 +34,14 @@ bool dtype_ok(int d) { return d == FC_F32 || d == FC_F16 || d == FC_BF16; }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Transform half-length for a convolution of length L: the next power of two
+// >= max(L, 16) (rows shorter than it are zero-padded on chip).
+int transform_half(int L) {
+  int Lc = 16;
+  while (Lc < L) Lc <<= 1;
+  return Lc;
+}
+
 #define FC_REQUIRE(cond, st, ...) \
   do {                            \
     if (!(cond)) return fail(st, __VA_ARGS__); \
@@ -67,13 +75,14 @@ cudaError_t run_ssm_conv(const void* u, const float* dt, const float* lambda, co
     if (e != cudaSuccess) return e;
     return launch_fftconv_tcl(u, f, L, D, y, B, H, L, L, 1, dtype, true, false, st);
   }
-  if (L >= 1024 && N > 64) {  // filter generated inside the convolution kernel (no tensor-core generator)
+  const int Lc = transform_half(L);
+  if (Lc >= 1024 && N > 64) {  // filter generated inside the convolution kernel (no tensor-core generator)
     const SsmArgs sp{dt, (const float2*)lambda, (const float2*)Bp, (const float2*)Cp, N};
-    return launch_fftconv(u, nullptr, L, sp, D, y, B, H, L, L, 1, dtype, st);
+    return launch_fftconv(u, nullptr, L, sp, D, y, B, H, L, Lc, 1, dtype, st);
   }
   e = launch_ssm_gen(dt, lambda, Bp, Cp, H, N, L, f, st);
   if (e != cudaSuccess) return e;
-  return launch_fftconv(u, f, L, none, D, y, B, H, L, L, 1, dtype, st);
+  return launch_fftconv(u, f, L, none, D, y, B, H, L, Lc, 1, dtype, st);
 }
 }  // namespace fc
 
@@ -128,8 +137,7 @@ FC_API fc_status fftconv_fwd(const void* u, const float* f, const float* D, void
   if (s != FC_OK) return s;
   FC_REQUIRE(f && D, FC_EINVAL, "null f or D");
   FC_REQUIRE(aligned(f, 16) && aligned(D, 4), FC_EINVAL, "f must be 16-byte aligned, D 4-byte aligned");
-  FC_REQUIRE(pow2(L) && L >= 16 && L <= 8192, FC_EUNSUPPORTED,
-             "fftconv_fwd: L must be a power of two in [16, 8192] (got %d)", L);
+  FC_REQUIRE(L >= 1 && L <= 8192, FC_EUNSUPPORTED, "fftconv_fwd: L must be in [1, 8192] (got %d)", L);
   if (fc::fftconv_tc_supported(L, dtype))
     return cuda_status(fc::launch_fftconv_tc(u, f, D, y, B, H, L, dtype, false, (cudaStream_t)stream),
                        "fftconv_fwd (tensor cores) launch");
@@ -137,8 +145,9 @@ FC_API fc_status fftconv_fwd(const void* u, const float* f, const float* D, void
     return cuda_status(fc::launch_fftconv_tcl(u, f, L, D, y, B, H, L, L, 1, dtype, false, false, (cudaStream_t)stream),
                        "fftconv_fwd (tensor cores) launch");
   const fc::SsmArgs none{nullptr, nullptr, nullptr, nullptr, 0};
-  return cuda_status(fc::launch_fftconv(u, f, L, none, D, y, B, H, L, L, 1, dtype, (cudaStream_t)stream),
-                     "fftconv_fwd launch");
+  return cuda_status(
+      fc::launch_fftconv(u, f, L, none, D, y, B, H, L, transform_half(L), 1, dtype, (cudaStream_t)stream),
+      "fftconv_fwd launch");
 }
 
 FC_API fc_status fftconv_bwd(const void* dy, const void* u, const float* f, const float* D, void* du, float* df,
@@ -156,8 +165,7 @@ FC_API fc_status fftconv_bwd(const void* dy, const void* u, const float* f, cons
     s = check_conv_io(dy, du, B, H, L, dtype);
     if (s != FC_OK) return s;
   }
-  FC_REQUIRE(pow2(L) && L >= 16 && L <= 8192, FC_EUNSUPPORTED,
-             "fftconv_bwd: L must be a power of two in [16, 8192] (got %d)", L);
+  FC_REQUIRE(L >= 1 && L <= 8192, FC_EUNSUPPORTED, "fftconv_bwd: L must be in [1, 8192] (got %d)", L);
   FC_REQUIRE(H <= 65535, FC_EUNSUPPORTED, "H = %d > 65535", H);
   if (du) FC_REQUIRE(f && D && aligned(f, 16) && aligned(D, 4), FC_EINVAL, "du needs f (16-byte aligned) and D");
   if (df)
@@ -172,7 +180,7 @@ FC_API fc_status fftconv_bwd(const void* dy, const void* u, const float* f, cons
             ? cuda_status(fc::launch_fftconv_tcl(dy, f, L, D, du, B, H, L, L, 1, dtype, false, true, st),
                           "fftconv_bwd: du (tensor cores) launch")
             : cuda_status(fc::launch_fftconv(dy, f, L, fc::SsmArgs{nullptr, nullptr, nullptr, nullptr, 0}, D, du, B,
-                                             H, L, L, 1, dtype, st, 1),
+                                             H, L, transform_half(L), 1, dtype, st, 1),
                           "fftconv_bwd: du launch");
     if (s != FC_OK) return s;
   }
@@ -197,8 +205,7 @@ FC_API fc_status ssm_conv_fwd(const void* u, const float* dt, const float* lambd
   if (s != FC_OK) return s;
   FC_REQUIRE(D && aligned(D, 4), FC_EINVAL, "null or misaligned D");
   FC_REQUIRE(N >= 1 && N <= 1024, FC_EUNSUPPORTED, "N must be in [1, 1024] (got %d)", N);
-  FC_REQUIRE(pow2(L) && L >= 16 && L <= 8192, FC_EUNSUPPORTED,
-             "ssm_conv_fwd: L must be a power of two in [16, 8192] (got %d)", L);
+  FC_REQUIRE(L >= 1 && L <= 8192, FC_EUNSUPPORTED, "ssm_conv_fwd: L must be in [1, 8192] (got %d)", L);
   FC_REQUIRE(H <= 65535, FC_EUNSUPPORTED, "H = %d > 65535", H);
   FC_REQUIRE(workspace && aligned(workspace, 256), FC_EINVAL, "workspace must be non-null and 256-byte aligned");
   FC_REQUIRE(ws_bytes >= ssm_conv_workspace(H, L), FC_EINVAL, "workspace too small: %zu < %zu bytes", ws_bytes,

@@ -11,6 +11,15 @@
 
 namespace fc {
 
+// Diagonal-SSM parameters for kernels that generate their filter (dt == nullptr: none).
+struct SsmArgs {
+  const float* dt;
+  const float2* lam;
+  const float2* Bp;
+  const float2* Cp;
+  int N;
+};
+
 // ---- per-device launch setup, cached so that repeated calls do not repeat
 // runtime queries.  Devices with an ordinal >= 64 are served uncached.
 inline int current_device() {

@@ -9,7 +9,8 @@
 //   dD[h]   = sum_b sum_t dy[b,h,t] u[b,h,t]
 // With both sequences zero-padded to M = 2L, df is the circular correlation
 //   df = IFFT( sum_b DY_b . conj(U_b) )  cropped to k < L
-// (a lag k >= 0 never wraps for t, t - k in [0, L)).
+// (a lag k >= 0 never wraps for t, t - k in [0, L)).  Rows shorter than the
+// transform half-length (L < M/2, any L) are read with zeros past L.
 //
 // One group of TG threads owns a channel and walks its B rows.  Each row's u
 // and dy are packed as one complex sequence z = u + i dy, so one FFT gives
@@ -26,7 +27,7 @@ namespace fc {
 template <typename T, int LOGM>
 __global__ void __launch_bounds__(ConvGeom<LOGM>::THREADS, ConvGeom<LOGM>::MINB)
     fftconv_df_kernel(const T* __restrict__ dy, const T* __restrict__ u, float* __restrict__ df,
-                      float* __restrict__ dD, int B, int H) {
+                      float* __restrict__ dD, int B, int H, int Lv) {
   using P = FftPlan<LOGM>;
   using Gm = ConvGeom<LOGM>;
   constexpr int M = P::M, TG = P::TG, RM = P::RMAX, R0 = P::R0, RL = P::RLAST;
@@ -54,7 +55,7 @@ __global__ void __launch_bounds__(ConvGeom<LOGM>::THREADS, ConvGeom<LOGM>::MINB)
   float dsum = 0.f;
   float2 v[RM];
   for (int b = 0; b < B; ++b) {  // every group runs B rows: the barriers stay uniform
-    const size_t row = ((size_t)b * H + (gv ? h : 0)) * (size_t)L;
+    const size_t row = ((size_t)b * H + (gv ? h : 0)) * (size_t)Lv;
 #pragma unroll
     for (int i = 0; i < PER0; ++i) {
       const int j = tid + i * TG;
@@ -62,7 +63,7 @@ __global__ void __launch_bounds__(ConvGeom<LOGM>::THREADS, ConvGeom<LOGM>::MINB)
       for (int r = 0; r < R0; ++r) {
         const int n = j + r * (M / R0);
         float2 z = make_float2(0.f, 0.f);
-        if (r < R0 / 2 && gv) {
+        if (r < R0 / 2 && gv && n < Lv) {
           z = make_float2(IO<T>::ld(u + row + n), IO<T>::ld(dy + row + n));
           dsum = fmaf(z.x, z.y, dsum);
         }
@@ -116,12 +117,13 @@ __global__ void __launch_bounds__(ConvGeom<LOGM>::THREADS, ConvGeom<LOGM>::MINB)
   __syncthreads();
   fft_inv<LOGM>(v, buf, tid, tw);
   if (gv) {
-    float* dfh = df + (size_t)h * L;
+    float* dfh = df + (size_t)h * Lv;
 #pragma unroll
     for (int i = 0; i < PER0; ++i) {
       const int j = tid + i * TG;
 #pragma unroll
-      for (int r = 0; r < R0 / 2; ++r) dfh[j + r * (M / R0)] = v[i * R0 + r].x;
+      for (int r = 0; r < R0 / 2; ++r)
+        if (j + r * (M / R0) < Lv) dfh[j + r * (M / R0)] = v[i * R0 + r].x;
     }
   }
   // dD: reduce dsum over the group's TG threads
@@ -144,7 +146,8 @@ __global__ void __launch_bounds__(ConvGeom<LOGM>::THREADS, ConvGeom<LOGM>::MINB)
 }
 
 template <typename T, int LOGM>
-static cudaError_t launch_df_t(const void* dy, const void* u, float* df, float* dD, int B, int H, cudaStream_t st) {
+static cudaError_t launch_df_t(const void* dy, const void* u, float* df, float* dD, int B, int H, int Lv,
+                               cudaStream_t st) {
   using Gm = ConvGeom<LOGM>;
   const size_t smem = Gm::smem_bytes;
   if (smem > 48 * 1024) {
@@ -152,24 +155,26 @@ static cudaError_t launch_df_t(const void* dy, const void* u, float* df, float* 
     if (e != cudaSuccess) return e;
   }
   const unsigned grid = (unsigned)((H + Gm::G - 1) / Gm::G);
-  fftconv_df_kernel<T, LOGM><<<grid, Gm::THREADS, smem, st>>>((const T*)dy, (const T*)u, df, dD, B, H);
+  fftconv_df_kernel<T, LOGM><<<grid, Gm::THREADS, smem, st>>>((const T*)dy, (const T*)u, df, dD, B, H, Lv);
   return cudaGetLastError();
 }
 
 template <typename T>
 static cudaError_t launch_df_dispatch(const void* dy, const void* u, float* df, float* dD, int B, int H, int L,
                                       cudaStream_t st) {
-  switch (L) {
-    case 16: return launch_df_t<T, 5>(dy, u, df, dD, B, H, st);
-    case 32: return launch_df_t<T, 6>(dy, u, df, dD, B, H, st);
-    case 64: return launch_df_t<T, 7>(dy, u, df, dD, B, H, st);
-    case 128: return launch_df_t<T, 8>(dy, u, df, dD, B, H, st);
-    case 256: return launch_df_t<T, 9>(dy, u, df, dD, B, H, st);
-    case 512: return launch_df_t<T, 10>(dy, u, df, dD, B, H, st);
-    case 1024: return launch_df_t<T, 11>(dy, u, df, dD, B, H, st);
-    case 2048: return launch_df_t<T, 12>(dy, u, df, dD, B, H, st);
-    case 4096: return launch_df_t<T, 13>(dy, u, df, dD, B, H, st);
-    case 8192: return launch_df_t<T, 14>(dy, u, df, dD, B, H, st);
+  int Lc = 16;
+  while (Lc < L) Lc <<= 1;
+  switch (Lc) {
+    case 16: return launch_df_t<T, 5>(dy, u, df, dD, B, H, L, st);
+    case 32: return launch_df_t<T, 6>(dy, u, df, dD, B, H, L, st);
+    case 64: return launch_df_t<T, 7>(dy, u, df, dD, B, H, L, st);
+    case 128: return launch_df_t<T, 8>(dy, u, df, dD, B, H, L, st);
+    case 256: return launch_df_t<T, 9>(dy, u, df, dD, B, H, L, st);
+    case 512: return launch_df_t<T, 10>(dy, u, df, dD, B, H, L, st);
+    case 1024: return launch_df_t<T, 11>(dy, u, df, dD, B, H, L, st);
+    case 2048: return launch_df_t<T, 12>(dy, u, df, dD, B, H, L, st);
+    case 4096: return launch_df_t<T, 13>(dy, u, df, dD, B, H, L, st);
+    case 8192: return launch_df_t<T, 14>(dy, u, df, dD, B, H, L, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -22,8 +22,8 @@
 
 #include <algorithm>
 
+#include "common.cuh"
 #include "fft_stockham.cuh"
-#include "kernels.cuh"
 #include "ssm_tables.cuh"
 
 namespace fc {
@@ -153,7 +153,10 @@ struct GenGeom {
 // u, y: rows of a B x H x Lrow array; each row holds C chunks of length
 // Lc = M/2 (C = 1 for a plain convolution).  Sub-row q in [0, B*C) of channel
 // h starts at ((q / C) * H + h) * Lrow + (q % C) * Lc.  Filter: f + h*fstride
-// (Lc taps), or generated from the SSM parameters when GEN.
+// (Lc taps), or generated from the SSM parameters when GEN.  With C = 1 a row
+// may be shorter than Lc (any L <= Lc): the transform runs at Lc with the
+// positions t >= L read as zeros and never stored.  The causal outputs t < L
+// depend only on u and f at positions <= t, so they are exact.
 template <typename T, int LOGM, bool GEN>
 __global__ void __launch_bounds__(ConvGeom<LOGM>::THREADS, ConvGeom<LOGM>::MINB)
     fftconv_kernel(const T* __restrict__ u, const float* __restrict__ f, int fstride, SsmArgs sp,
@@ -193,6 +196,7 @@ __global__ void __launch_bounds__(ConvGeom<LOGM>::THREADS, ConvGeom<LOGM>::MINB)
   auto row_off = [&](int h, int q) -> size_t {
     return ((size_t)(q / C) * H + h) * (size_t)Lrow + (size_t)(q % C) * Lc;
   };
+  const int Lv = (C == 1 && Lrow < Lc) ? (int)Lrow : Lc;  // valid positions of a sub-row
   auto prefetch = [&](long long it, UPair<T>* dst) {
     const int h = (int)(it / NP), p = (int)(it - (long long)h * NP);
     const int q0 = 2 * p, q1 = 2 * p + 1;
@@ -205,7 +209,7 @@ __global__ void __launch_bounds__(ConvGeom<LOGM>::THREADS, ConvGeom<LOGM>::MINB)
 #pragma unroll
       for (int r = 0; r < R0 / 2; ++r) {
         const int n = j + r * (M / R0);
-        if (gv && FC_OK_IDX(11, (long long)row_off(h, q0) + n, (long long)B * H * Lrow))
+        if (gv && n < Lv && FC_OK_IDX(11, (long long)row_off(h, q0) + n, (long long)B * H * Lrow))
           dst[i * (R0 / 2) + r].load(u0 + n, u1 + n, has1);
         else
           dst[i * (R0 / 2) + r].zero();
@@ -264,7 +268,7 @@ __global__ void __launch_bounds__(ConvGeom<LOGM>::THREADS, ConvGeom<LOGM>::MINB)
           const int j = tid + i * TG;
 #pragma unroll
           for (int r = 0; r < R0; ++r)
-            v[i * R0 + r] = (r < R0 / 2 && gv &&
+            v[i * R0 + r] = (r < R0 / 2 && gv && j + r * (M / R0) < Lv &&
                              FC_OK_IDX(10, (long long)h * fstride + j + r * (M / R0), (long long)H * fstride))
                                 ? make_float2(__ldg(fr + j + r * (M / R0)), 0.f)
                                 : make_float2(0.f, 0.f);
@@ -316,7 +320,7 @@ __global__ void __launch_bounds__(ConvGeom<LOGM>::THREADS, ConvGeom<LOGM>::MINB)
 #pragma unroll
         for (int r = 0; r < R0 / 2; ++r) {
           const int n = j + r * (M / R0);
-          if (!FC_OK_IDX(13, (long long)row_off(h, q0) + n, (long long)B * H * Lrow)) continue;
+          if (n >= Lv || !FC_OK_IDX(13, (long long)row_off(h, q0) + n, (long long)B * H * Lrow)) continue;
           const float2 uu = ucur[i * (R0 / 2) + r].get();
           IO<T>::st(y0 + n, fmaf(dh, uu.x, v[i * R0 + r].x));
           if (has1) IO<T>::st(y1 + n, fmaf(dh, uu.y, v[i * R0 + r].y));

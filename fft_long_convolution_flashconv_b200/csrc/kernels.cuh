@@ -8,14 +8,6 @@
 
 namespace fc {
 
-// Diagonal-SSM parameters for kernels that generate their filter (dt == nullptr: none).
-struct SsmArgs {
-  const float* dt;
-  const float2* lam;
-  const float2* Bp;
-  const float2* Cp;
-  int N;
-};
 
 // ssm_conv_fwd's dispatch: filter generation into f (H x L floats of scratch),
 // then the fused convolution (tensor cores where supported).

@@ -66,8 +66,7 @@ FC_API fc_status ssm_conv_fwd_noalloc(const void* u, const float* dt, const floa
   if (!u || !y || !dt || !lambda || !Bp || !Cp || !D) return na_fail(FC_EINVAL, "null pointer argument");
   if (!al(u, 16) || !al(y, 16) || !al(dt, 4) || !al(lambda, 8) || !al(Bp, 8) || !al(Cp, 8) || !al(D, 4))
     return na_fail(FC_EINVAL, "misaligned pointer (u, y: 16 bytes; dt, D: 4; complex parameters: 8)");
-  if (L < 16 || L > 8192 || (L & (L - 1)) != 0)
-    return na_fail(FC_EUNSUPPORTED, "L must be a power of two in [16, 8192]");
+  if (L < 1 || L > 8192) return na_fail(FC_EUNSUPPORTED, "L must be in [1, 8192]");
   if (N > 1024 || H > 65535) return na_fail(FC_EUNSUPPORTED, "N must be <= 1024 and H <= 65535");
   if (B > (1 << 30)) return na_fail(FC_EUNSUPPORTED, "B must be <= 2^30");
   if ((size_t)H * (size_t)L > kNoAllocFilterFloats)

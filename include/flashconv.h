@@ -107,16 +107,19 @@ FC_API fc_status ssm_kernel_gen(const float* dt, const float* lambda, const floa
  *   y[b,h,t] = sum_{s<=t} f[h,t-s] u[b,h,s] + D[h] u[b,h,t]
  * evaluated as IFFT_{2L}(FFT_{2L}(pad u) * FFT_{2L}(pad f)) cropped to t < L.
  * u, y: B x H x L in `dtype`; f: H x L floats (any real filter, not only an
- * SSM's); D: H floats.  Limits: L a power of two, 16 <= L <= 8192; B, H >= 1.
- * u and y may not overlap.
- * Precision: FC_F32 and every L without a tensor-core kernel: float32
- * FFTs on the CUDA cores, one rounding at the store.  16-bit I/O at
- * L = 1024 runs the block-FFT stages on the tensor cores: the filter (with D
- * added to its tap 0) is rounded to the I/O type; the DFT-128 stages take
- * their data operand in the I/O type (exact for u); the DFT-16 stages take
- * float16 operands scaled by 1/32, which stay finite for |u| <= 32752; the
- * inverse stage's input is rounded to the I/O type; accumulation is float32
- * and y is rounded once at the store. */
+ * SSM's); D: H floats.  Limits: 1 <= L <= 8192 (any length; rows whose L is
+ * not a power of two >= 16 are zero-padded on chip to the next one, which
+ * leaves the causal outputs t < L exact); B, H >= 1.  u and y may not
+ * overlap.
+ * Precision: FC_F32 and every L without a tensor-core kernel (L < 1024 or
+ * not a power of two): float32 FFTs on the CUDA cores, one rounding at the
+ * store.  16-bit I/O at L = 1024, 2048, 4096, 8192 runs the block-FFT
+ * stages on the tensor cores: the filter (with D added to its tap 0) is
+ * rounded to the I/O type; the DFT-128 stages take their data operand in the
+ * I/O type (exact for u); the column DFT stages take float16 operands scaled
+ * so that they stay within 2 max|u| (finite for |u| <= 32752); the inverse
+ * stage's input is rounded to the I/O type; accumulation is float32 and y is
+ * rounded once at the store. */
 FC_API fc_status fftconv_fwd(const void* u, const float* f, const float* D, void* y,
                              int B, int H, int L, fc_dtype dtype, void* stream);
 

@@ -50,12 +50,10 @@ def _err():
 
 def test_fftconv_rejects_bad_arguments():
     lib = _lib.load()
-    # L not a power of two
-    assert lib.fftconv_fwd(P, P2, P3, P + (1 << 26), 2, 3, 1000, 1, None) == _lib.FC_EUNSUPPORTED
-    assert "power of two" in _err()
-    # L too large / too small
+    # L too large (any L in [1, 8192] is accepted, powers of two or not)
     assert lib.fftconv_fwd(P, P2, P3, P + (1 << 26), 2, 3, 16384, 1, None) == _lib.FC_EUNSUPPORTED
-    assert lib.fftconv_fwd(P, P2, P3, P + (1 << 26), 2, 3, 8, 1, None) == _lib.FC_EUNSUPPORTED
+    assert "[1, 8192]" in _err()
+    assert lib.fftconv_fwd(P, P2, P3, P + (1 << 26), 2, 3, 8193, 1, None) == _lib.FC_EUNSUPPORTED
     # null pointers
     assert lib.fftconv_fwd(None, P2, P3, P, 2, 3, 64, 1, None) == _lib.FC_EINVAL
     assert lib.fftconv_fwd(P, None, P3, P + (1 << 26), 2, 3, 64, 1, None) == _lib.FC_EINVAL
@@ -130,7 +128,7 @@ def test_mixer_rejects_bad_arguments():
 
 def test_error_message_is_per_call():
     lib = _lib.load()
-    assert lib.fftconv_fwd(P, P2, P3, P + (1 << 26), 2, 3, 1000, 1, None) != 0
+    assert lib.fftconv_fwd(P, P2, P3, P + (1 << 26), 2, 3, 16384, 1, None) != 0
     assert _err()
     assert lib.fc_status_string(0) == b"ok"
 
@@ -142,5 +140,31 @@ def test_noalloc_rejects_oversize_before_any_launch():
     y = P + (1 << 28)
     assert lib.ssm_conv_fwd_noalloc(P, P2, P3, P, P2, P3, y, 1, 256, 8192, 64, 1, None) == _lib.FC_EUNSUPPORTED
     assert b"fixed scratch" in lib.ssm_conv_noalloc_last_error()
-    assert lib.ssm_conv_fwd_noalloc(P, P2, P3, P, P2, P3, y, 1, 4, 1000, 64, 1, None) == _lib.FC_EUNSUPPORTED
+    assert lib.ssm_conv_fwd_noalloc(P, P2, P3, P, P2, P3, y, 1, 4, 10000, 64, 1, None) == _lib.FC_EUNSUPPORTED
     assert lib.ssm_conv_fwd_noalloc(None, P2, P3, P, P2, P3, y, 1, 4, 1024, 64, 1, None) == _lib.FC_EINVAL
+
+
+def test_backward_and_decode_reject_bad_arguments():
+    lib = _lib.load()
+    du = P + (1 << 26)
+    # nothing requested, df without dD, L out of range, overlap of dy and du
+    assert lib.fftconv_bwd(P, P2, P3, P, None, None, None, 2, 3, 64, 1, None) == _lib.FC_EINVAL
+    assert lib.fftconv_bwd(P, P2, P3, P, None, P2, None, 2, 3, 64, 1, None) == _lib.FC_EINVAL
+    assert lib.fftconv_bwd(P, P2, P3, P, du, None, None, 2, 3, 9000, 1, None) == _lib.FC_EUNSUPPORTED
+    assert lib.fftconv_bwd(P, P2, P3, P, P + 64, None, None, 2, 3, 64, 1, None) == _lib.FC_EINVAL
+    # du requested without f
+    assert lib.fftconv_bwd(P, P2, None, P, du, None, None, 2, 3, 64, 1, None) == _lib.FC_EINVAL
+    # decode: T < 1, N too large, misaligned state
+    y = P + (1 << 26)
+    assert lib.ssm_decode_step(P, P2, P, P2, P3, P, P, y, 2, 3, 16, 0, 1, None) == _lib.FC_EINVAL
+    assert lib.ssm_decode_step(P, P2, P, P2, P3, P, P, y, 2, 3, 2000, 1, 1, None) == _lib.FC_EUNSUPPORTED
+    assert lib.ssm_decode_step(P, P2 + 4, P, P2, P3, P, P, y, 2, 3, 16, 1, 1, None) == _lib.FC_EINVAL
+    # mixer decode: head_dim too large, shift_len out of range, negative position
+    o = P + (1 << 26)
+    assert lib.h3_mixer_decode_step(P, P, P, P, P2, P, P, P2, P3, P, P, o, 1, 2, 65, 8, 4, 0, 1,
+                                    None) == _lib.FC_EUNSUPPORTED
+    assert lib.h3_mixer_decode_step(P, P, P, P, P2, P, P, P2, P3, P, P, o, 1, 2, 64, 8, 9, 0, 1,
+                                    None) == _lib.FC_EUNSUPPORTED
+    assert lib.h3_mixer_decode_step(P, P, P, P, P2, P, P, P2, P3, P, P, o, 1, 2, 64, 8, 4, -1, 1,
+                                    None) == _lib.FC_EINVAL
+    assert lib.h3_decode_state_bytes(2, 3, 64, 8) == 2 * 3 * 64 * 64 * 8 * 8

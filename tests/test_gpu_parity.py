@@ -456,3 +456,32 @@ def test_fftconv_fp16_slow_filters_constant_step_and_large_inputs(L):
         ref = cref.causal_conv(u16, f32, wl.D.astype(np.float64))
         assert np.all(np.isfinite(y)), name
         assert O.row_rel_err(y.reshape(-1, L), ref.reshape(-1, L)) < 2e-2, name
+
+
+# ------------------------------------------------------------------ (f)4 any length
+@pytest.mark.parametrize("L,dtype", [(1, "f32"), (7, "f32"), (100, "f16"), (1000, "bf16"), (1500, "f32"),
+                                     (3000, "f16"), (5000, "bf16"), (8191, "f32")])
+def test_fftconv_any_length(L, dtype):
+    """Lengths that are not powers of two (EEG-clip-like lengths): zero padding
+    to the next power of two on chip, causal outputs exact up to rounding."""
+    B, H = 3, 5
+    rng = np.random.default_rng(L)
+    u = W.round_to(rng.normal(size=(B, H, L)), dtype)
+    f = W.round_to(rng.normal(size=(H, L)) * np.exp(-np.arange(L) / max(1.0, L / 7.0)), "f32")  # arbitrary filters
+    D = rng.normal(size=H)
+    y = host(api.fftconv_fwd(dev(u, dtype), dev(f), dev(D)))
+    ref = cref.causal_conv(u, f, D)
+    assert O.row_rel_err(y.reshape(-1, L), ref.reshape(-1, L)) < TOL[dtype]
+    dy = W.round_to(rng.normal(size=(B, H, L)), dtype)
+    du, df, dD = api.fftconv_bwd(dev(dy, dtype), dev(u, dtype), dev(f), dev(D))
+    rdu, rdf, rdD = O.causal_conv_bwd(dy, u, f, D)
+    assert O.row_rel_err(host(du).reshape(-1, L), rdu.reshape(-1, L)) < TOL[dtype]
+    assert O.row_rel_err(host(df), rdf) < 1e-4 * max(1.0, np.log2(L * B + 1) / 4)
+
+
+def test_ssm_conv_any_length():
+    wl = W.make_conv(B=2, H=6, L=1234, N=80, dtype="f32", seed=9)  # N > 64: fused generation path
+    y = host(api.ssm_conv_fwd(dev(wl.u), *params(wl)))
+    f = O.ssm_filter(wl.dt, wl.lam, wl.Bp, wl.Cp, wl.L)
+    ref = cref.causal_conv(wl.u, f, wl.D.astype(np.float64))
+    assert O.row_rel_err(y.reshape(-1, wl.L), ref.reshape(-1, wl.L)) < 1e-4
