@@ -11,6 +11,8 @@ import subprocess
 import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+import gen_tables  # noqa: E402
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libflashconv_b200.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
@@ -69,6 +71,7 @@ def build(force: bool = False, verbose: bool = False, jobs: int = 0, check: bool
     the bounds-checked debug variant (-DFC_CHECK) into
     libflashconv_b200_check.so; load it by setting FC_LIB_PATH."""
     lib = LIB.replace(".so", "_check.so") if check else LIB
+    gen_tables.write()  # constant DFT blocks and twiddles (rewritten only when they change)
     if not check and not force and not _stale():
         return LIB
     objdir = os.path.join(HERE, "_build_check" if check else "_build")

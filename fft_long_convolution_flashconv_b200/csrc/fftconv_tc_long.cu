@@ -26,7 +26,8 @@
 // GEMM with fp32 accumulation in TMEM.  Stages A and A' use the constant
 // DFT-128 blocks CA, CB of the L = 1024 kernel (data operands in the I/O
 // type); stages B and B' take fp16 operands, scaled by 1/(32 R) so that the
-// stage-B input stays within 2 max|u|.
+// stage-B input stays within 2 max|u|.  The constant blocks and twiddle
+// bases come from tables built with the library (tc_tables.inc).
 //
 // Work: one CTA per SM walks a contiguous range of (channel, row pair)
 // items; two real rows are packed as u0 + i u1 (f is real, so the real and
@@ -41,6 +42,10 @@
 #include "fft_stockham.cuh"
 #include "kernels.cuh"
 #include "tc100.cuh"
+
+#define FC_TABLES_DFT128
+#define FC_TABLES_LONG
+#include "tc_tables.inc"
 
 namespace fc {
 
@@ -63,7 +68,7 @@ struct LG {
   static constexpr uint32_t tcols = 4 * N2;         // TMEM: work [0, 2 N2) | filter [2 N2, 4 N2)
   static constexpr uint32_t o_ca = 0, o_cb = kCBytes, o_gf = 2 * kCBytes, o_gi = o_gf + R * 2048,
                             o_x = o_gi + R * 2048, o_yv = o_x + 2 * xplane, o_fst = o_yv + yv,
-                            o_cos = o_fst + 4 * Lc, o_mbar = o_cos + 128 * 8, o_tmem = o_mbar + 8,
+                            o_mbar = o_fst + 4 * Lc, o_tmem = o_mbar + 8,
                             bytes = o_tmem + 8;
   static_assert(256u * N2 * 2 == yv, "Z must fit the stage-B tiles");
 };
@@ -71,6 +76,8 @@ struct LG {
 template <typename T> struct OpL;
 template <> struct OpL<__half> {
   static constexpr int bf16 = 0;
+  static __device__ __forceinline__ const uint16_t* ca() { return g_ca_f16; }
+  static __device__ __forceinline__ const uint16_t* cb() { return g_cb_f16; }
   static __device__ __forceinline__ uint32_t pack(float a, float b) {
     __half2 h = __floats2half2_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&h);
@@ -78,12 +85,32 @@ template <> struct OpL<__half> {
 };
 template <> struct OpL<__nv_bfloat16> {
   static constexpr int bf16 = 1;
+  static __device__ __forceinline__ const uint16_t* ca() { return g_ca_bf16; }
+  static __device__ __forceinline__ const uint16_t* cb() { return g_cb_bf16; }
   static __device__ __forceinline__ uint32_t pack(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&h);
   }
 };
 __device__ __forceinline__ uint32_t pack_h(float a, float b) { return OpL<__half>::pack(a, b); }
+
+// per-R tables: stage-B blocks [k2b][forward, inverse], ta[k1][n2a], tb[k1][n2b]
+template <int R> struct LT;
+template <> struct LT<2> {
+  static __device__ __forceinline__ const uint16_t* blocks() { return g_gblk_r2; }
+  static __device__ __forceinline__ const float* ta() { return g_ta_r2; }
+  static __device__ __forceinline__ const float* tb() { return g_tb_r2; }
+};
+template <> struct LT<4> {
+  static __device__ __forceinline__ const uint16_t* blocks() { return g_gblk_r4; }
+  static __device__ __forceinline__ const float* ta() { return g_ta_r4; }
+  static __device__ __forceinline__ const float* tb() { return g_tb_r4; }
+};
+template <> struct LT<8> {
+  static __device__ __forceinline__ const uint16_t* blocks() { return g_gblk_r8; }
+  static __device__ __forceinline__ const float* ta() { return g_ta_r8; }
+  static __device__ __forceinline__ const float* tb() { return g_tb_r8; }
+};
 
 __device__ __forceinline__ void cp_async16(uint32_t saddr, const void* g) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(g) : "memory");
@@ -104,7 +131,6 @@ __global__ void __launch_bounds__(kThrL, 1)
   using G = LG<R>;
   constexpr int N2 = G::N2, Lc = G::Lc, M = G::M;
   extern __shared__ __align__(1024) uint8_t sm[];
-  float2* costab = reinterpret_cast<float2*>(sm + G::o_cos);
   uint64_t* mbar = reinterpret_cast<uint64_t*>(sm + G::o_mbar);
   uint32_t* tmem_p = reinterpret_cast<uint32_t*>(sm + G::o_tmem);
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -122,65 +148,33 @@ __global__ void __launch_bounds__(kThrL, 1)
     tc::mbar_init(mbar, 1);
     tc::fence_mbar_init();
   }
-  if (tid < 128) {
-    float s, c;
-    sincospif(2.0f * (float)tid / 128.0f, &s, &c);
-    costab[tid] = make_float2(c, s);
-  }
-  __syncthreads();
-  // DFT-128 blocks in the I/O type (as the L = 1024 kernel): CA[k1][j] = j < 64 ? cos : sin, CB = j < 64 ? -sin : cos
-  for (int idx = tid; idx < 128 * 16; idx += kThrL) {
-    const int k1 = idx >> 4, j0 = (idx & 15) * 8;
-    float a[8], b[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int j = j0 + i, jj = j & 63;
-      const float2 cs = costab[(k1 * jj) & 127];
-      a[i] = j < 64 ? cs.x : cs.y;
-      b[i] = j < 64 ? -cs.y : cs.x;
+  // constant blocks (tables built with the library, already in the operand layouts): CA, CB in the
+  // I/O type; the forward / inverse stage-B blocks of every k2b in fp16
+  {
+    const uint8_t* gca = reinterpret_cast<const uint8_t*>(OpL<T>::ca());
+    const uint8_t* gcb = reinterpret_cast<const uint8_t*>(OpL<T>::cb());
+    const uint8_t* gbl = reinterpret_cast<const uint8_t*>(LT<R>::blocks());
+    for (int i = tid; i < (int)(kCBytes / 16); i += kThrL) {
+      cp_async16(ca + i * 16, gca + i * 16);
+      cp_async16(cb + i * 16, gcb + i * 16);
     }
-    const uint32_t off = tc::kmaj_off(k1, j0, 128);
-    *reinterpret_cast<uint4*>(sm + G::o_ca + off) = make_uint4(OpL<T>::pack(a[0], a[1]), OpL<T>::pack(a[2], a[3]),
-                                                              OpL<T>::pack(a[4], a[5]), OpL<T>::pack(a[6], a[7]));
-    *reinterpret_cast<uint4*>(sm + G::o_cb + off) = make_uint4(OpL<T>::pack(b[0], b[1]), OpL<T>::pack(b[2], b[3]),
-                                                              OpL<T>::pack(b[4], b[5]), OpL<T>::pack(b[6], b[7]));
-  }
-  // stage-B blocks (fp16, K-major 32 x 32): forward G_k2b rows c = output (k2a, re|im), columns = input (n2a, re|im);
-  // inverse rows = output (n2a, re|im), columns = input (k2a, re|im); angle 2 pi n2a (R k2a + k2b) / N2
-  for (int idx = tid; idx < R * 2 * 32 * 4; idx += kThrL) {
-    const int k2b = idx / 256, inv = (idx >> 7) & 1, c = (idx >> 2) & 31, j0 = (idx & 3) * 8;
-    float a[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int jj = j0 + i;
-      const int n2a = inv ? (c & 15) : (jj & 15), k2a = inv ? (jj & 15) : (c & 15);
-      const int m = (n2a * (R * k2a + k2b)) % N2;
-      const float2 cs = costab[m * (128 / N2)];
-      const bool oim = c >= 16, iim = jj >= 16;
-      // forward (e^{-i theta}): Re += xr cos + xi sin, Im += xi cos - xr sin; the inverse flips sin
-      const float fw = (oim == iim) ? cs.x : (iim ? cs.y : -cs.y);
-      a[i] = inv ? ((oim == iim) ? cs.x : -fw) : fw;
+    for (int i = tid; i < R * 2 * 128; i += kThrL) {  // block (2 k2b + inv), 128 chunks of 16 bytes each
+      const int blk = i >> 7, k2b = blk >> 1, inv = blk & 1;
+      cp_async16((inv ? gi : gf) + k2b * 2048 + (i & 127) * 16, gbl + i * 16);
     }
-    const uint32_t off = (uint32_t)(inv ? G::o_gi : G::o_gf) + (uint32_t)k2b * 2048 + (uint32_t)(c >> 3) * kTSbo +
-                         (uint32_t)(j0 >> 3) * kTLbo + (uint32_t)(c & 7) * 16;
-    *reinterpret_cast<uint4*>(sm + off) = make_uint4(pack_h(a[0], a[1]), pack_h(a[2], a[3]), pack_h(a[4], a[5]),
-                                                     pack_h(a[6], a[7]));
+    cp_async_commit();
   }
-  // this thread's twiddle factors: k1 = row, n2a = 4 set + l
+  // this thread's twiddle factors: k1 = row, n2a = 4 set + l, n2b < R (from the tables)
   float2 ta_s[4], ta_c[4], tb[R];
 #pragma unroll
   for (int l = 0; l < 4; ++l) {
-    float s, c;
-    sincospif(-2.0f * (float)(row * (4 * set + l)) / (float)M, &s, &c);
-    ta_s[l] = make_float2(c * (1.f / (32.f * R)), s * (1.f / (32.f * R)));
-    ta_c[l] = make_float2(c * (32.f * R), -s * (32.f * R));
+    const float2 t = *reinterpret_cast<const float2*>(LT<R>::ta() + 2 * (row * 16 + 4 * set + l));
+    ta_s[l] = make_float2(t.x * (1.f / (32.f * R)), t.y * (1.f / (32.f * R)));
+    ta_c[l] = make_float2(t.x * (32.f * R), -t.y * (32.f * R));
   }
 #pragma unroll
-  for (int b2 = 0; b2 < R; ++b2) {
-    float s, c;
-    sincospif(-2.0f * (float)(16 * row * b2) / (float)M, &s, &c);
-    tb[b2] = make_float2(c, s);
-  }
+  for (int b2 = 0; b2 < R; ++b2) tb[b2] = *reinterpret_cast<const float2*>(LT<R>::tb() + 2 * (row * R + b2));
+  cp_async_wait_all();
   tc::fence_smem_to_async();
   tc::fence_before_sync();
   __syncthreads();
