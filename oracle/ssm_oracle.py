@@ -38,7 +38,7 @@ __all__ = [
     "as_complex", "discretize", "ssm_powers", "ssm_filter", "ssm_filter_from_A",
     "causal_conv_direct", "ssm_recurrence", "statepass_chunked",
     "shift_ssm", "h3_mixer_outer", "h3_mixer_toeplitz", "row_rel_err",
-    "causal_conv_bwd", "h3_mixer_recurrent",
+    "causal_conv_bwd", "h3_mixer_recurrent", "statepass_bwd",
 ]
 
 
@@ -356,3 +356,42 @@ def h3_mixer_recurrent(q, k, v, Cshift, A, Bc, Cc, D, heads: int) -> np.ndarray:
                 y = 2.0 * np.real(np.sum(Cc[h][None, None, :] * X[h], axis=2)) + D[h] * kv
                 o[b, t, sl] = q[b, t, sl] @ y
     return o
+
+
+def statepass_bwd(dy, A, Bc, Cc, D, dstate_out=None):
+    """Gradients of the long-sequence SSM (state passing) with respect to u
+    and the initial state.
+
+    H3 summary, section 4 "Long-sequence computation" with appendix C.1
+    "Backward Pass": the forward y_t = 2 Re(C x_t) + D u_t, x_t = A x_{t-1} +
+    B u_t over the whole sequence (x_{-1} = state_in, state_out = x_{L-1});
+    chunking does not change it.  For a real loss with dL/dy = dy and
+    dL/d(state_out) = G (complex convention: G = dL/dRe + i dL/dIm), the
+    derivatives of those sums are
+      du[t]        = sum_{s>=t} f[s-t] dy[s] + D dy[t] + Re sum_n conj(G_n) A_n^(L-1-t) B_n
+      dstate_in[n] = sum_t dy[t] 2 conj(C_n A_n^(t+1)) + conj(A_n^L) G_n
+    with f[k] = 2 Re sum_n C_n A_n^k B_n, written here as plain sums.
+    dy: (B, H, L); A, Bc, Cc: (H, N) complex; D: (H,); dstate_out:
+    (B, H, N) complex or None.  Returns (du, dstate_in)."""
+    dy = np.asarray(dy, dtype=np.float64)
+    A = np.asarray(A, dtype=np.complex128)
+    Bc = np.asarray(Bc, dtype=np.complex128)
+    Cc = np.asarray(Cc, dtype=np.complex128)
+    D = np.asarray(D, dtype=np.float64)
+    Bn, H, L = dy.shape
+    N = A.shape[1]
+    G = np.zeros((Bn, H, N), dtype=np.complex128) if dstate_out is None \
+        else np.asarray(dstate_out, dtype=np.complex128)
+    k = np.arange(L)
+    P = A[:, :, None] ** k[None, None, :]                       # H x N x L: A^k
+    f = 2.0 * np.real(np.sum((Cc * Bc)[:, :, None] * P, axis=1))  # H x L
+    du = np.empty_like(dy)
+    dsin = np.empty((Bn, H, N), dtype=np.complex128)
+    for b in range(Bn):
+        for h in range(H):
+            for t in range(L):
+                du[b, h, t] = np.dot(f[h, :L - t], dy[b, h, t:]) + D[h] * dy[b, h, t] + \
+                    np.real(np.sum(np.conj(G[b, h]) * P[h, :, L - 1 - t] * Bc[h]))
+            CA = Cc[h][:, None] * (A[h][:, None] ** (k[None, :] + 1))   # N x L: C A^(t+1)
+            dsin[b, h] = 2.0 * np.sum(dy[b, h][None, :] * np.conj(CA), axis=1) + np.conj(A[h] ** L) * G[b, h]
+    return du, dsin

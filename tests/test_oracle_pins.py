@@ -399,6 +399,50 @@ def test_mixer_recurrent_equals_outer_form():
     assert np.max(np.abs(o_lag - o_conv)) > 1e-3 * np.max(np.abs(o_conv))
 
 
+def test_statepass_bwd_by_linearity_brute_force():
+    """The loss <dy, y> + Re<G, state_out> is linear in (u, state_in): every
+    gradient entry is the loss at a basis vector (through the pinned
+    recurrence), including the imaginary directions of the state."""
+    rng = np.random.default_rng(21)
+    B, H, L, N = 1, 2, 9, 3
+    A = 0.9 * np.exp(1j * rng.uniform(0, np.pi, size=(H, N)))
+    Bc = rng.normal(size=(H, N)) + 1j * rng.normal(size=(H, N))
+    Cc = rng.normal(size=(H, N)) + 1j * rng.normal(size=(H, N))
+    D = rng.normal(size=H)
+    dy = rng.normal(size=(B, H, L))
+    G = rng.normal(size=(B, H, N)) + 1j * rng.normal(size=(B, H, N))
+    du, dsin = O.statepass_bwd(dy, A, Bc, Cc, D, dstate_out=G)
+
+    def loss(u, x0):
+        y, x = O.ssm_recurrence(u, A, Bc, Cc, D, x0=x0)
+        return np.sum(dy * y) + np.sum(np.real(np.conj(G) * x))
+    zero_u = np.zeros((B, H, L))
+    zero_x = np.zeros((B, H, N), dtype=np.complex128)
+    for h in range(H):
+        for t in range(L):
+            e = zero_u.copy()
+            e[0, h, t] = 1.0
+            assert abs(loss(e, zero_x) - du[0, h, t]) < 1e-12
+        for n in range(N):
+            for unit, part in ((1.0, "re"), (1j, "im")):
+                x0 = zero_x.copy()
+                x0[0, h, n] = unit
+                want = dsin[0, h, n].real if part == "re" else dsin[0, h, n].imag
+                assert abs(loss(zero_u, x0) - want) < 1e-12
+
+
+def test_statepass_bwd_without_state_grad_is_conv_bwd():
+    """With no gradient on the final state, du is the convolution's input
+    gradient (anti-causal correlation with f plus D dy)."""
+    rng = np.random.default_rng(22)
+    wl, A, Bc, Cc = _small(L=48, H=3, B=2)
+    dy = rng.normal(size=wl.u.shape)
+    du, _ = O.statepass_bwd(dy, A, Bc, Cc, wl.D)
+    f = O.ssm_filter_from_A(A, Bc, Cc, wl.L)
+    du2, _, _ = O.causal_conv_bwd(dy, wl.u, f, wl.D)
+    assert np.max(np.abs(du - du2)) < 1e-10 * np.max(np.abs(du2))
+
+
 # ---------------------------------------------------------------- planted mistakes
 def test_pins_catch_planted_mistakes(golden):
     """Mutated copies of oracle steps (made here, on the CPU) must fail a pin."""
