@@ -33,6 +33,9 @@ SIGNATURES = {
     "fftconv_statepass_workspace": (_sz, [_i, _i, _i, _i, _i]),
     "fftconv_statepass": (_i, [_vp, _fp, _fp, _fp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _fp, _fp, _vp, _sz,
                                _i, _vp]),
+    "fftconv_statepass_bwd_workspace": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "fftconv_statepass_bwd": (_i, [_vp, _fp, _fp, _fp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _fp, _fp, _vp, _sz,
+                                   _i, _vp]),
     "ssm_conv_fwd_noalloc": (_i, [_vp, _fp, _fp, _fp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _vp]),
     "ssm_conv_noalloc_max_filter_floats": (_sz, []),
     "ssm_conv_noalloc_last_error": (ctypes.c_char_p, []),

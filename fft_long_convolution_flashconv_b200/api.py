@@ -209,6 +209,29 @@ def fftconv_statepass(u, dt, lam, Bp, Cp, D, chunk: int, state_in: Optional[torc
     return (out, sout) if return_state else out
 
 
+def fftconv_statepass_bwd(dy, dt, lam, Bp, Cp, D, chunk: int, dstate_out: Optional[torch.Tensor] = None,
+                          need_dstate_in: bool = False, workspace: Optional[torch.Tensor] = None,
+                          out: Optional[torch.Tensor] = None):
+    """Gradients of fftconv_statepass: du (and dstate_in, B x H x N x 2, if
+    need_dstate_in) given dy and optionally dstate_out."""
+    lib = _lib.load()
+    B, H, L = dy.shape
+    dt, lam, Bp, Cp, D = _f32(dt), _cpx(lam), _cpx(Bp), _cpx(Cp), _f32(D)
+    N = lam.shape[1]
+    need = int(lib.fftconv_statepass_bwd_workspace(B, H, L, N, chunk, _dtype(dy)))
+    if workspace is None:
+        workspace = _alloc_ws(need, dy.device)
+    if out is None:
+        out = torch.empty_like(dy)
+    gin = _cpx(dstate_out) if dstate_out is not None else None
+    gsin = torch.empty((B, H, N, 2), dtype=torch.float32, device=dy.device) if need_dstate_in else None
+    check(lib.fftconv_statepass_bwd(_ptr(dy), _ptr(dt), _ptr(lam), _ptr(Bp), _ptr(Cp), _ptr(D), _ptr(out), B, H, L,
+                                    N, chunk, _ptr(gin), _ptr(gsin), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _dtype(dy), _stream()),
+          "fftconv_statepass_bwd")
+    return (out, gsin) if need_dstate_in else out
+
+
 def h3_mixer_workspace_bytes(B, L, heads, head_dim, N) -> int:
     return int(_lib.load().h3_mixer_workspace(B, L, heads, head_dim, N))
 

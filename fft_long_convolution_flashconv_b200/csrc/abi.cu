@@ -215,6 +215,26 @@ FC_API fc_status ssm_conv_fwd(const void* u, const float* dt, const float* lambd
                      "ssm_conv_fwd launch");
 }
 
+// The state-passing pipeline on validated arguments: chunk filter, chunk
+// convolutions, then end states, carry and initial-state term.
+static fc_status statepass_run(const void* u, const float* dt, const float* lambda, const float* Bp, const float* Cp,
+                               const float* D, void* y, int B, int H, int L, int N, int chunk, const float* state_in,
+                               float* state_out, float* fT, float* s_ws, float* x_ws, int dtype, cudaStream_t st) {
+  const int C = L / chunk;
+  fc_status s = cuda_status(fc::launch_ssm_gen(dt, lambda, Bp, Cp, H, N, chunk, fT, st), "statepass: filter launch");
+  if (s != FC_OK) return s;
+  const fc::SsmArgs none{nullptr, nullptr, nullptr, nullptr, 0};
+  s = fc::fftconv_tcl_supported(chunk, dtype)
+          ? cuda_status(fc::launch_fftconv_tcl(u, fT, chunk, D, y, B, H, L, chunk, C, dtype, true, false, st),
+                        "statepass: chunk conv (tensor cores) launch")
+          : cuda_status(fc::launch_fftconv(u, fT, chunk, none, D, y, B, H, L, chunk, C, dtype, st),
+                        "statepass: chunk conv launch");
+  if (s != FC_OK) return s;
+  return cuda_status(fc::launch_statepass_tail(u, dt, lambda, Bp, Cp, y, B, H, L, N, chunk, state_in, state_out,
+                                               s_ws, x_ws, dtype, st),
+                     "statepass: state launch");
+}
+
 // workspace layout: [f_T: H*T floats][s: B*H*C*N complex][x: B*H*C*N complex], each 256-aligned
 FC_API size_t fftconv_statepass_workspace(int B, int H, int L, int N, int chunk) {
   if (B < 1 || H < 1 || L < 1 || N < 1 || chunk < 1 || L % chunk) return 0;
@@ -248,22 +268,71 @@ FC_API fc_status fftconv_statepass(const void* u, const float* dt, const float* 
   const int C = L / chunk;
   const size_t fb = round_up((size_t)H * chunk * sizeof(float), 256);
   const size_t sb = round_up((size_t)B * H * C * N * 2 * sizeof(float), 256);
-  float* fT = (float*)workspace;
-  float* s_ws = (float*)((char*)workspace + fb);
-  float* x_ws = (float*)((char*)workspace + fb + sb);
+  return statepass_run(u, dt, lambda, Bp, Cp, D, y, B, H, L, N, chunk, state_in, state_out, (float*)workspace,
+                       (float*)((char*)workspace + fb), (float*)((char*)workspace + fb + sb), dtype,
+                       (cudaStream_t)stream);
+}
+
+// workspace: [forward workspace][lambda', B', C': 3 x H x N complex][x0': B x H x N complex]
+//            [lambda_0: B x H x N complex][dy reversed][du reversed], each 256-aligned
+FC_API size_t fftconv_statepass_bwd_workspace(int B, int H, int L, int N, int chunk, fc_dtype dtype) {
+  const size_t fw = fftconv_statepass_workspace(B, H, L, N, chunk);
+  if (fw == 0 || !dtype_ok(dtype)) return 0;
+  const size_t pb = round_up((size_t)H * N * 2 * sizeof(float), 256);
+  const size_t xb = round_up((size_t)B * H * N * 2 * sizeof(float), 256);
+  const size_t rb = round_up((size_t)B * H * L * dtype_size(dtype), 256);
+  return fw + 3 * pb + 2 * xb + 2 * rb;
+}
+
+FC_API fc_status fftconv_statepass_bwd(const void* dy, const float* dt, const float* lambda, const float* Bp,
+                                       const float* Cp, const float* D, void* du, int B, int H, int L, int N,
+                                       int chunk, const float* dstate_out, float* dstate_in, void* workspace,
+                                       size_t ws_bytes, fc_dtype dtype, void* stream) {
+  g_err[0] = 0;
+  FC_REQUIRE(L >= 1, FC_EINVAL, "L must be >= 1");
+  fc_status s = check_conv_io(dy, du, B, H, L, dtype);
+  if (s != FC_OK) return s;
+  s = check_params(dt, lambda, Bp, Cp);
+  if (s != FC_OK) return s;
+  FC_REQUIRE(D && aligned(D, 4), FC_EINVAL, "null or misaligned D");
+  FC_REQUIRE(N >= 1 && N <= 256, FC_EUNSUPPORTED, "N must be in [1, 256] (got %d)", N);
+  FC_REQUIRE(pow2(chunk) && chunk >= 16 && chunk <= 8192, FC_EUNSUPPORTED,
+             "chunk must be a power of two in [16, 8192] (got %d)", chunk);
+  FC_REQUIRE(L % chunk == 0, FC_EINVAL, "L = %d is not a multiple of chunk = %d", L, chunk);
+  FC_REQUIRE(H <= 65535 && B <= 65535, FC_EUNSUPPORTED, "B or H > 65535");
+  FC_REQUIRE(!dstate_out || aligned(dstate_out, 8), FC_EINVAL, "dstate_out must be 8-byte aligned");
+  FC_REQUIRE(!dstate_in || aligned(dstate_in, 8), FC_EINVAL, "dstate_in must be 8-byte aligned");
+  FC_REQUIRE(workspace && aligned(workspace, 256), FC_EINVAL, "workspace must be non-null and 256-byte aligned");
+  const size_t need = fftconv_statepass_bwd_workspace(B, H, L, N, chunk, dtype);
+  FC_REQUIRE(ws_bytes >= need, FC_EINVAL, "workspace too small: %zu < %zu bytes", ws_bytes, need);
+  const int C = L / chunk;
+  const size_t fb = round_up((size_t)H * chunk * sizeof(float), 256);
+  const size_t sb = round_up((size_t)B * H * C * N * 2 * sizeof(float), 256);
+  const size_t fw = fftconv_statepass_workspace(B, H, L, N, chunk);
+  const size_t pb = round_up((size_t)H * N * 2 * sizeof(float), 256);
+  const size_t xb = round_up((size_t)B * H * N * 2 * sizeof(float), 256);
+  const size_t rb = round_up((size_t)B * H * L * dtype_size(dtype), 256);
+  char* w = (char*)workspace;
+  float* lam_a = (float*)(w + fw);
+  float* B_a = (float*)(w + fw + pb);
+  float* C_a = (float*)(w + fw + 2 * pb);
+  float* x0_a = (float*)(w + fw + 3 * pb);
+  float* lam0 = (float*)(w + fw + 3 * pb + xb);
+  void* dy_rev = w + fw + 3 * pb + 2 * xb;
+  void* du_rev = w + fw + 3 * pb + 2 * xb + rb;
   cudaStream_t st = (cudaStream_t)stream;
-  s = cuda_status(fc::launch_ssm_gen(dt, lambda, Bp, Cp, H, N, chunk, fT, st), "statepass: filter launch");
+  s = cuda_status(fc::launch_sp_adjoint_params(dt, lambda, Bp, Cp, dstate_out, lam_a, B_a, C_a, x0_a, B, H, N, st),
+                  "statepass_bwd: adjoint parameters launch");
   if (s != FC_OK) return s;
-  const fc::SsmArgs none{nullptr, nullptr, nullptr, nullptr, 0};
-  s = fc::fftconv_tcl_supported(chunk, dtype)
-          ? cuda_status(fc::launch_fftconv_tcl(u, fT, chunk, D, y, B, H, L, chunk, C, dtype, true, false, st),
-                        "statepass: chunk conv (tensor cores) launch")
-          : cuda_status(fc::launch_fftconv(u, fT, chunk, none, D, y, B, H, L, chunk, C, dtype, st),
-                        "statepass: chunk conv launch");
+  s = cuda_status(fc::launch_reverse_rows(dy, dy_rev, (long long)B * H, L, dtype, st), "statepass_bwd: reverse dy");
   if (s != FC_OK) return s;
-  return cuda_status(fc::launch_statepass_tail(u, dt, lambda, Bp, Cp, y, B, H, L, N, chunk, state_in, state_out,
-                                               s_ws, x_ws, dtype, st),
-                     "statepass: state launch");
+  s = statepass_run(dy_rev, dt, lam_a, B_a, C_a, D, du_rev, B, H, L, N, chunk, dstate_out ? x0_a : nullptr,
+                    dstate_in ? lam0 : nullptr, (float*)w, (float*)(w + fb), (float*)(w + fb + sb), dtype, st);
+  if (s != FC_OK) return s;
+  s = cuda_status(fc::launch_reverse_rows(du_rev, du, (long long)B * H, L, dtype, st), "statepass_bwd: reverse du");
+  if (s != FC_OK || !dstate_in) return s;
+  return cuda_status(fc::launch_sp_adjoint_state(dt, lambda, lam0, dstate_in, B, H, N, st),
+                     "statepass_bwd: initial-state gradient launch");
 }
 
 // workspace layout: [f: heads*L floats][k~: B*L*heads*head_dim 16-bit elements], each 256-aligned

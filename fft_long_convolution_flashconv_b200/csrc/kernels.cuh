@@ -65,6 +65,16 @@ cudaError_t launch_h3_decode(const void* q, const void* k, const void* v, void* 
                              void* o, int B, int heads, int hd, int N, int S, long long pos, int dtype,
                              cudaStream_t st);
 
+// State-passing backward helpers: the adjoint SSM's parameters (lambda' =
+// conj(lambda), B' = 2 conj(C), C' = conj(B) / 2, x0' = G / conj(A) when G is
+// given), row reversal in time, and dstate_in = conj(A) lambda_0.
+cudaError_t launch_sp_adjoint_params(const float* dt, const float* lam, const float* Bp, const float* Cp,
+                                     const float* G, float* lam_a, float* B_a, float* C_a, float* x0_a, int B, int H,
+                                     int N, cudaStream_t st);
+cudaError_t launch_reverse_rows(const void* in, void* out, long long rows, int L, int dtype, cudaStream_t st);
+cudaError_t launch_sp_adjoint_state(const float* dt, const float* lam, const float* lam0, float* dsin, int B, int H,
+                                    int N, cudaStream_t st);
+
 // Tensor-core fused FFT convolution (block-FFT stages as tcgen05 GEMMs).
 bool fftconv_tc_supported(int L, int dtype);
 // after_filter_kernel: f is written by the kernel launched just before on the

@@ -178,6 +178,29 @@ FC_API fc_status fftconv_statepass(const void* u, const float* dt, const float* 
                                    int chunk, const float* state_in, float* state_out, void* workspace,
                                    size_t ws_bytes, fc_dtype dtype, void* stream);
 
+/* fftconv_statepass_bwd -- backward pass of fftconv_statepass: gradients
+ * with respect to u and state_in, given dy (the gradient with respect to y)
+ * and optionally dstate_out (the gradient with respect to state_out), so that
+ * a sequence split over several calls back-propagates call by call.
+ * H3 summary section 4 "Long-sequence computation" and appendix C.1
+ * "Backward Pass".  With complex gradients G = dL/dRe + i dL/dIm:
+ *   du[t]        = sum_{s>=t} f[s-t] dy[s] + D dy[t] + Re sum_n conj(G_n) A_n^(L-1-t) B_n
+ *   dstate_in[n] = sum_t dy[t] 2 conj(C_n A_n^(t+1)) + conj(A_n^L) G_n
+ * (f[k] = 2 Re sum_n C_n A_n^k B_n).  It is evaluated as the adjoint SSM, a
+ * forward state-passing run over the time-reversed dy with A' = conj(A),
+ * B' = 2 conj(C), C' = conj(B) / 2 and initial state G / conj(A) (so A must not
+ * underflow to zero where G is given).
+ * dy, du: B x H x L in `dtype`; dstate_out, dstate_in: B x H x N complex or
+ * NULL (NULL dstate_out: zero; NULL dstate_in: not written).  Parameters,
+ * chunk and limits as fftconv_statepass.  workspace: at least
+ * fftconv_statepass_bwd_workspace(...) bytes, 256-byte aligned.  Precision:
+ * as fftconv_statepass (du is rounded like its y). */
+FC_API size_t fftconv_statepass_bwd_workspace(int B, int H, int L, int N, int chunk, fc_dtype dtype);
+FC_API fc_status fftconv_statepass_bwd(const void* dy, const float* dt, const float* lambda, const float* Bp,
+                                       const float* Cp, const float* D, void* du, int B, int H, int L, int N,
+                                       int chunk, const float* dstate_out, float* dstate_in, void* workspace,
+                                       size_t ws_bytes, fc_dtype dtype, void* stream);
+
 /* h3_mixer_fwd -- H3 layer core, projections excluded (A10-A11).
  * H3 blog "The Solution, Part 1": O = Q (.) SSM_diag(SSM_shift(K) (.) V);
  * H3 summary section 3 "H3 design" and appendix D.2 "H3 Complexity" (heads).

@@ -28,7 +28,8 @@ def test_header_declares_expected_entry_points():
     for s in ("ssm_kernel_gen", "fftconv_fwd", "fftconv_statepass", "h3_mixer_fwd",
               "fftconv_statepass_workspace", "h3_mixer_workspace", "ssm_conv_fwd", "ssm_conv_workspace",
               "fc_last_error", "fc_status_string", "fc_version", "fftconv_bwd", "fc_tc_timeouts",
-              "ssm_decode_step", "h3_mixer_decode_step", "h3_decode_state_bytes"):
+              "ssm_decode_step", "h3_mixer_decode_step", "h3_decode_state_bytes",
+              "fftconv_statepass_bwd", "fftconv_statepass_bwd_workspace"):
         assert s in syms
 
 

@@ -486,3 +486,28 @@ def test_ssm_conv_any_length():
     f = O.ssm_filter(wl.dt, wl.lam, wl.Bp, wl.Cp, wl.L)
     ref = cref.causal_conv(wl.u, f, wl.D.astype(np.float64))
     assert O.row_rel_err(y.reshape(-1, wl.L), ref.reshape(-1, wl.L)) < 1e-4
+
+
+# ------------------------------------------------------------------ (f)3 state-passing backward
+@pytest.mark.parametrize("B,H,L,T,N,dtype,with_g", [
+    (2, 3, 256, 64, 8, "f32", True), (1, 2, 512, 128, 16, "f32", False), (2, 2, 1024, 256, 33, "f32", True),
+    (1, 3, 8192, 2048, 16, "f16", True), (1, 2, 16384, 8192, 64, "bf16", False),
+])
+def test_statepass_bwd(B, H, L, T, N, dtype, with_g):
+    """du and dstate_in against the oracle's gradient sums; with a gradient on
+    the final state and without."""
+    wl = W.make_conv(B=B, H=H, L=L, N=N, dtype=dtype, seed=L + N, dt_range=("loguniform", -3.0, -1.0))
+    dtt, lam, Bp, Cp, D = params(wl)
+    rng = np.random.default_rng(T)
+    dy = W.round_to(rng.normal(size=(B, H, L)), dtype)
+    G = (rng.normal(size=(B, H, N)) + 1j * rng.normal(size=(B, H, N))) if with_g else None
+    g_t = torch.view_as_real(torch.tensor(G.astype(np.complex64))).cuda().contiguous() if with_g else None
+    du, dsin = api.fftconv_statepass_bwd(dev(dy, dtype), dtt, lam, Bp, Cp, D, T, dstate_out=g_t, need_dstate_in=True)
+    A, Bc, Cc = oracle_A(wl)
+    G64 = G.astype(np.complex64).astype(np.complex128) if with_g else None
+    rdu, rdsin = O.statepass_bwd(dy, A, Bc, Cc, wl.D.astype(np.float64), dstate_out=G64)
+    assert O.row_rel_err(host(du).reshape(-1, L), rdu.reshape(-1, L)) < TOL[dtype]
+    g = host(dsin)
+    g = g[..., 0] + 1j * g[..., 1]
+    tol = 1e-4 if dtype == "f32" else 5e-3
+    assert np.max(np.abs(g - rdsin)) < tol * np.max(np.abs(rdsin))
