@@ -68,7 +68,9 @@ constexpr uint32_t kFBytes = kL * 4;                                     // fp32
 constexpr uint32_t kWBytes = (kMaxPairs + 1) * kYTile;                   // stage-B tiles, then Z
 static_assert(kWBytes >= kMaxPairs * kN2 * 2 * kN1 * 2, "Z must fit the work buffer");
 // shared memory layout (bytes)
-constexpr uint32_t kOCa = 0, kOCb = kCBytes, kOWf = 2 * kCBytes, kOWi = kOWf + 2048, kOPipe = kOWi + 2048;
+constexpr uint32_t kTwBytes = kN1 * kN2 * 8;  // fp32 twiddles w_2048^(k1 n2) / 32
+constexpr uint32_t kOCa = 0, kOCb = kCBytes, kOWf = 2 * kCBytes, kOWi = kOWf + 2048, kOTw = kOWi + 2048,
+                   kOPipe = kOTw + kTwBytes;
 constexpr uint32_t kPipeBytes = kXBytes + kFBytes + kWBytes;
 constexpr uint32_t kOX = 0, kOF = kXBytes, kOW = kXBytes + kFBytes;  // within a pipeline's part
 constexpr uint32_t kOMbar = kOPipe + kPipes * kPipeBytes, kOTmem = kOMbar + 8 * kPipes;
@@ -139,6 +141,7 @@ __global__ void __launch_bounds__(kThr, 1) fftconv_tc_kernel(const T* __restrict
   uint32_t* tmem_p = reinterpret_cast<uint32_t*>(sm + kOTmem);
   const uint32_t s0 = tc::smem_u32(sm);
   const uint32_t ca = s0 + kOCa, cb = s0 + kOCb, wfa = s0 + kOWf, wia = s0 + kOWi;
+  const float2* tws = reinterpret_cast<const float2*>(sm + kOTw);  // [k1][n2]
   const uint32_t pbase = kOPipe + (uint32_t)pipe * kPipeBytes;
   const uint32_t xs = s0 + pbase + kOX, fs = s0 + pbase + kOF, ws = s0 + pbase + kOW;
   uint8_t* const wsp = sm + pbase + kOW;
@@ -158,6 +161,8 @@ __global__ void __launch_bounds__(kThr, 1) fftconv_tc_kernel(const T* __restrict
     }
     if (tid < 128) cp_async16(wfa + tid * 16, reinterpret_cast<const uint8_t*>(g_wf16_f16) + tid * 16);
     else if (tid < 256) cp_async16(wia + (tid - 128) * 16, reinterpret_cast<const uint8_t*>(g_wi16_f16) + (tid - 128) * 16);
+    for (int i = tid; i < (int)(kTwBytes / 16); i += kThr)
+      cp_async16(s0 + kOTw + i * 16, reinterpret_cast<const uint8_t*>(g_tw1k) + i * 16);
   }
   cp_async_commit();
 
@@ -190,10 +195,14 @@ __global__ void __launch_bounds__(kThr, 1) fftconv_tc_kernel(const T* __restrict
   };
   long long it = blockIdx.x + (long long)gridDim.x * pipe;
   if (it < nitems) issue_u(it);
+  float d_next = 0.f;  // D of the next item's channel, loaded with its inputs
   // the filter is written by the kernel this one may be launched as a
   // programmatic dependent of: read it only after the wait
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (it < nitems) issue_f(it);
+  if (it < nitems) {
+    issue_f(it);
+    d_next = D[(int)(it / ngroups)];
+  }
   cp_async_commit();
   cp_async_wait_all();
   tc::fence_smem_to_async();
@@ -226,6 +235,7 @@ __global__ void __launch_bounds__(kThr, 1) fftconv_tc_kernel(const T* __restrict
     const int NC = NS * kN2;                           // stage-A columns per real/imag half
     const uint32_t lboX = (uint32_t)(NC / 8) * 128;    // X: MN-major, 64 K-rows (n1) x NC
     const uint32_t xr = xs, xi = xs + 8 * lboX;
+    const float dh = d_next;
     cp_async_wait_all();
     pipe_sync(bar_id);  // every thread's copies have landed
     // filter block (column block 0): fp32 staging -> operand type, D folded into tap 0
@@ -234,7 +244,7 @@ __global__ void __launch_bounds__(kThr, 1) fftconv_tc_kernel(const T* __restrict
       const int t = n1 * kN2 + hf * 8;
       float4 a = *reinterpret_cast<const float4*>(sm + pbase + kOF + t * 4);
       const float4 b = *reinterpret_cast<const float4*>(sm + pbase + kOF + t * 4 + 16);
-      if (t == 0) a.x += D[h];  // y = f * u + D u = (f + D delta) * u
+      if (t == 0) a.x += dh;  // y = f * u + D u = (f + D delta) * u
       const uint32_t off = (uint32_t)hf * 128 + (uint32_t)(n1 >> 3) * lboX + (uint32_t)(n1 & 7) * 16;
       *reinterpret_cast<uint4*>(sm + pbase + kOX + off) = make_uint4(Op<T>::pack(a.x, a.y), Op<T>::pack(a.z, a.w),
                                                                     Op<T>::pack(b.x, b.y), Op<T>::pack(b.z, b.w));
@@ -267,13 +277,14 @@ __global__ void __launch_bounds__(kThr, 1) fftconv_tc_kernel(const T* __restrict
     if (it + stride < nitems) {
       issue_u(it + stride);
       issue_f(it + stride);
+      d_next = D[(int)((it + stride) / ngroups)];
     }
     cp_async_commit();
     // ---- pass 1: Y' = Y w_2048^(k1 n2) / 32 -> fp16 stage-B tile per sequence (this thread: n2 = 8 half + i)
     {
       float2 tw[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) tw[i] = ldf2(g_tw1k + 2 * (row * kN2 + 8 * half + i));
+      for (int i = 0; i < 8; ++i) tw[i] = tws[row * kN2 + 8 * half + i];
 #pragma unroll 1
       for (int s = 0; s < NS; s += 2) {
         const bool two = s + 1 < NS;
@@ -390,7 +401,7 @@ __global__ void __launch_bounds__(kThr, 1) fftconv_tc_kernel(const T* __restrict
       float2 tw[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float2 w = ldf2(g_tw1k + 2 * (row * kN2 + 8 * half + i));
+        const float2 w = tws[row * kN2 + 8 * half + i];
         tw[i] = make_float2(32.f * w.x, -32.f * w.y);
       }
 #pragma unroll 1

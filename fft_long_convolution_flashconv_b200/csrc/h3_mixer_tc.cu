@@ -324,7 +324,8 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
 // has its own completion barriers, so each parity wait is at most one phase
 // behind.  Rows past L are zero-filled by the copies themselves.
 namespace {
-constexpr int kThr2 = 256;
+constexpr int kThr2 = 512;
+constexpr int kMaxLf = 12288;  // filter rows up to this length are staged in shared memory
 constexpr uint32_t kQT = (kT / 8) * kQSbo;   // Q / K~ tile bytes (padded)
 constexpr uint32_t kVT = (kT / 8) * kVLbo;   // V tile bytes (padded)
 constexpr uint32_t kPT = kT * kT * 2;        // P tile bytes
@@ -336,6 +337,7 @@ struct Mix2Smem {
   float fs[2][2 * kT];
   uint64_t bq, bk[2], bv[3], bs[2], bo[2];
   uint32_t tmem_base;
+  // followed by the head's filter row (L floats, dynamic)
 };
 // 16-byte copy; src_bytes = 0 fills the destination with zeros (nothing is read)
 __device__ __forceinline__ void cp_async16_zfill(uint32_t saddr, const void* g, int src_bytes) {
@@ -357,7 +359,8 @@ __global__ void __launch_bounds__(kThr2, 1) h3_mixer_tc2_kernel(const T* __restr
   Mix2Smem& sm = *reinterpret_cast<Mix2Smem*>(smraw);
   const int tid = threadIdx.x, warp = tid >> 5;
   const int row = tid & 127;         // TMEM lane: t row of the tile
-  const int half = warp >> 2;        // S columns [64 half, 64 half + 64)
+  const int quarter = warp >> 2;     // S columns [32 quarter, 32 quarter + 32); O columns [16 quarter, +16)
+  float* frow = reinterpret_cast<float*>(smraw + sizeof(Mix2Smem));  // f of the current head, t < L
   const int dm = heads * kHD;
   const int nT = (L + kT - 1) / kT;
   const long long nitems = (long long)B * heads * nT;
@@ -417,6 +420,10 @@ __global__ void __launch_bounds__(kThr2, 1) h3_mixer_tc2_kernel(const T* __restr
     const uint16_t* vb = reinterpret_cast<const uint16_t*>(v) + base;
     const float dh = D[h];
     const float* fh = fdiag + (size_t)h * L;
+    // the head's filter row -> shared memory when it fits (the previous item's last reads were
+    // before the item-end barrier); longer rows are read from global memory
+    if (L <= kMaxLf)
+      for (int i = tid; i < L; i += kThr2) frow[i] = fh[i];
     // ---- item start: Q, K~(0), V(0) (and K~(1))
     copy_rows(sm.q, qb, t0, false, &sm.bq);
     copy_rows(sm.k[gs & 1], kb, 0, false, &sm.bk[gs & 1]);
@@ -459,7 +466,7 @@ __global__ void __launch_bounds__(kThr2, 1) h3_mixer_tc2_kernel(const T* __restr
       // (c) Toeplitz weights of (t0, s0): fs[idx] = f[t - s] (+ D at t = s), idx = t - s - (t0 - s0) + 127
       for (int idx = tid; idx < 2 * kT - 1; idx += kThr2) {
         const int d = idx - (kT - 1) + (t0 - s0);
-        float w = (d >= 0 && d < L) ? fh[d] : 0.f;
+        float w = (d >= 0 && d < L) ? (L <= kMaxLf ? frow[d] : fh[d]) : 0.f;
         if (d == 0) w += dh;
         sm.fs[sb][idx] = w;
       }
@@ -471,8 +478,8 @@ __global__ void __launch_bounds__(kThr2, 1) h3_mixer_tc2_kernel(const T* __restr
       // (e) P = S(j) (.) weights, rounded to the operand type, into P tile sb (K-major)
       const uint32_t tS = tmem + (uint32_t)(128 * sb);
       uint8_t* pt = sm.p[sb];
-#pragma unroll 1
-      for (int c = 64 * half; c < 64 * half + 64; c += 32) {
+      {
+        const int c = 32 * quarter;
         float sv[2][16];
         tc::tmem_ld16x2_wait(tS + lane_off + (uint32_t)c, tS + lane_off + (uint32_t)(c + 16), sv[0], sv[1]);
 #pragma unroll
@@ -516,13 +523,12 @@ __global__ void __launch_bounds__(kThr2, 1) h3_mixer_tc2_kernel(const T* __restr
     tc::fence_after_sync();
     {
       const int t = t0 + row;
-      float ov[2][16];
-      tc::tmem_ld16x2_wait(tO + lane_off + (uint32_t)(32 * half), tO + lane_off + (uint32_t)(32 * half + 16), ov[0],
-                           ov[1]);
+      float ov[1][16];
+      tc::tmem_ld16_wait(tO + lane_off + (uint32_t)(16 * quarter), ov[0]);
       if (t < L) {
-        uint16_t* orow = reinterpret_cast<uint16_t*>(o) + base + (size_t)t * dm + 32 * half;
+        uint16_t* orow = reinterpret_cast<uint16_t*>(o) + base + (size_t)t * dm + 16 * quarter;
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
+        for (int hh = 0; hh < 1; ++hh) {
           uint4 lo, hi;
           lo.x = Bits<T>::pack(ov[hh][0], ov[hh][1]);
           lo.y = Bits<T>::pack(ov[hh][2], ov[hh][3]);
@@ -569,7 +575,7 @@ static cudaError_t mixer_tc_t(const void* q, const void* k, const void* v, const
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t smem = sizeof(Mix2Smem) + 1024;
+  const size_t smem = sizeof(Mix2Smem) + (size_t)(L <= kMaxLf ? L : 0) * sizeof(float) + 1024;
   e = smem_optin<h3_mixer_tc2_kernel<T>>(smem);
   if (e != cudaSuccess) return e;
   const long long nitems = (long long)B * heads * ((L + kT - 1) / kT);
