@@ -311,249 +311,6 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
   if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
-// ---------------------------------------------------------------- pipelined mixer
-// One CTA per SM (256 threads) walks a list of (b, head, t tile) items, the
-// heaviest (most s tiles) first, dealt to the CTAs in snake order so that the
-// causal work is balanced.  Per item and s tile j:
-//   S(j+1) = Q K~(j+1)^T is issued before the epilogue of S(j) runs, into the
-//   other of two S accumulators, so the tensor cores and the epilogue overlap;
-//   P(j) goes to one of two P tiles (the one O(j-2) has finished reading), and
-//   O += P(j) V(j) is issued as soon as P(j) is stored.
-// K~ tiles (double-buffered) and V tiles (three buffers) are copied with
-// cp.async whose completion arrives on one mbarrier per buffer; every buffer
-// has its own completion barriers, so each parity wait is at most one phase
-// behind.  Rows past L are zero-filled by the copies themselves.
-namespace {
-constexpr int kThr2 = 512;
-constexpr int kMaxLf = 12288;  // filter rows up to this length are staged in shared memory
-constexpr uint32_t kQT = (kT / 8) * kQSbo;   // Q / K~ tile bytes (padded)
-constexpr uint32_t kVT = (kT / 8) * kVLbo;   // V tile bytes (padded)
-constexpr uint32_t kPT = kT * kT * 2;        // P tile bytes
-struct Mix2Smem {
-  uint8_t q[kQT];
-  uint8_t k[2][kQT];
-  uint8_t v[3][kVT];
-  uint8_t p[2][kPT];
-  float fs[2][2 * kT];
-  uint64_t bq, bk[2], bv[3], bs[2], bo[2];
-  uint32_t tmem_base;
-  // followed by the head's filter row (L floats, dynamic)
-};
-// 16-byte copy; src_bytes = 0 fills the destination with zeros (nothing is read)
-__device__ __forceinline__ void cp_async16_zfill(uint32_t saddr, const void* g, int src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr), "l"(g), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_arrive(uint64_t* mbar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(tc::smem_u32(mbar)) : "memory");
-}
-__device__ __forceinline__ bool cta_or(bool v) { return __syncthreads_or(v) != 0; }
-}  // namespace
-
-template <typename T>
-__global__ void __launch_bounds__(kThr2, 1) h3_mixer_tc2_kernel(const T* __restrict__ q, const T* __restrict__ kt,
-                                                                const T* __restrict__ v,
-                                                                const float* __restrict__ fdiag,
-                                                                const float* __restrict__ D, T* __restrict__ o, int B,
-                                                                int L, int heads) {
-  extern __shared__ __align__(1024) uint8_t smraw[];
-  Mix2Smem& sm = *reinterpret_cast<Mix2Smem*>(smraw);
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int row = tid & 127;         // TMEM lane: t row of the tile
-  const int quarter = warp >> 2;     // S columns [32 quarter, 32 quarter + 32); O columns [16 quarter, +16)
-  float* frow = reinterpret_cast<float*>(smraw + sizeof(Mix2Smem));  // f of the current head, t < L
-  const int dm = heads * kHD;
-  const int nT = (L + kT - 1) / kT;
-  const long long nitems = (long long)B * heads * nT;
-  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-
-  if (warp == 0) tc::tmem_alloc(&sm.tmem_base, 512);
-  if (tid == 0) {
-    tc::mbar_init(&sm.bq, kThr2);
-    for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&sm.bk[i], kThr2);
-      tc::mbar_init(&sm.bs[i], 1);
-      tc::mbar_init(&sm.bo[i], 1);
-    }
-    for (int i = 0; i < 3; ++i) tc::mbar_init(&sm.bv[i], kThr2);
-    tc::fence_mbar_init();
-  }
-  tc::fence_before_sync();
-  __syncthreads();
-  tc::fence_after_sync();
-  const uint32_t tmem = sm.tmem_base;
-  const uint32_t tO = tmem + 256;
-  const uint32_t idS = tc::idesc_f16(128, 128, Bits<T>::bf16);
-  const uint32_t idO = tc::idesc_f16(128, kHD, Bits<T>::bf16, 0, 1);
-  // phase parity of every barrier, one bit each: q 0, k 1-2, v 3-5, s 6-7, o 8-9
-  uint32_t ph = 0;
-  bool failed = false;
-  long long gs = 0;  // running s-tile counter of this CTA (selects buffers)
-
-  auto wait = [&](uint64_t* mb, int bit) -> bool {
-    const bool ok = tc::mbar_wait_bounded(mb, (ph >> bit) & 1u, kWaitNs);
-    ph ^= 1u << bit;
-    return ok;
-  };
-  // rows r0 .. r0+127 of a (b, head) slice: 16-byte chunks into a padded tile (K-major or V layout)
-  auto copy_rows = [&](uint8_t* dst, const uint16_t* src, int r0, bool vlayout, uint64_t* mb) {
-    const uint32_t d0 = tc::smem_u32(dst);
-    for (int idx = tid; idx < kT * (kHD / 8); idx += kThr2) {
-      const int r = idx >> 3, c8 = (idx & 7) * 8;
-      const int s = r0 + r;
-      const bool in = s < L;
-      cp_async16_zfill(d0 + (vlayout ? voff(r, c8) : qoff(r, c8)), src + (size_t)(in ? s : 0) * dm + c8, in ? 16 : 0);
-    }
-    cp_async_arrive(mb);
-  };
-
-  const long long G = gridDim.x;
-  for (long long rnd = 0;; ++rnd) {
-    const long long k = rnd * G + ((rnd & 1) ? (G - 1 - blockIdx.x) : blockIdx.x);
-    if (k >= nitems || failed) break;
-    const int tt = nT - 1 - (int)(k / ((long long)B * heads));  // heaviest items first
-    const int bh = (int)(k % ((long long)B * heads));
-    const int b = bh / heads, h = bh - (bh / heads) * heads;
-    const int t0 = tt * kT, NSt = tt + 1;
-    const size_t base = (size_t)b * L * dm + (size_t)h * kHD;
-    const uint16_t* qb = reinterpret_cast<const uint16_t*>(q) + base;
-    const uint16_t* kb = reinterpret_cast<const uint16_t*>(kt) + base;
-    const uint16_t* vb = reinterpret_cast<const uint16_t*>(v) + base;
-    const float dh = D[h];
-    const float* fh = fdiag + (size_t)h * L;
-    // the head's filter row -> shared memory when it fits (the previous item's last reads were
-    // before the item-end barrier); longer rows are read from global memory
-    if (L <= kMaxLf)
-      for (int i = tid; i < L; i += kThr2) frow[i] = fh[i];
-    // ---- item start: Q, K~(0), V(0) (and K~(1))
-    copy_rows(sm.q, qb, t0, false, &sm.bq);
-    copy_rows(sm.k[gs & 1], kb, 0, false, &sm.bk[gs & 1]);
-    copy_rows(sm.v[gs % 3], vb, 0, true, &sm.bv[gs % 3]);
-    if (NSt > 1) copy_rows(sm.k[(gs + 1) & 1], kb, kT, false, &sm.bk[(gs + 1) & 1]);
-    bool ok = wait(&sm.bq, 0) & wait(&sm.bk[gs & 1], 1 + (int)(gs & 1));
-    if (cta_or(!ok)) { failed = true; break; }
-    tc::fence_after_sync();
-    if (tid == 0) {  // S(0)
-      tc::fence_smem_to_async();
-      const uint32_t qa = tc::smem_u32(sm.q), ka = tc::smem_u32(sm.k[gs & 1]);
-#pragma unroll
-      for (int kk = 0; kk < kHD / 16; ++kk)
-        tc::mma_f16(tmem + (uint32_t)(128 * (gs & 1)), tc::desc_kmajor(qa + kk * 2 * kQLbo, kQLbo, kQSbo),
-                    tc::desc_kmajor(ka + kk * 2 * kQLbo, kQLbo, kQSbo), idS, kk > 0 ? 1u : 0u);
-      tc::mma_commit(&sm.bs[gs & 1]);
-    }
-    for (int j = 0; j < NSt && !failed; ++j) {
-      const long long g = gs + j;
-      const int sb = (int)(g & 1);
-      const int s0 = j * kT;
-      // (a) S(j+1) into the other accumulator (its last reader, the epilogue of j-1, is done)
-      if (j + 1 < NSt) {
-        ok = wait(&sm.bk[(g + 1) & 1], 1 + (int)((g + 1) & 1));
-        if (cta_or(!ok)) { failed = true; break; }
-        tc::fence_after_sync();
-        if (tid == 0) {
-          tc::fence_smem_to_async();
-          const uint32_t qa = tc::smem_u32(sm.q), ka = tc::smem_u32(sm.k[(g + 1) & 1]);
-#pragma unroll
-          for (int kk = 0; kk < kHD / 16; ++kk)
-            tc::mma_f16(tmem + (uint32_t)(128 * ((g + 1) & 1)), tc::desc_kmajor(qa + kk * 2 * kQLbo, kQLbo, kQSbo),
-                        tc::desc_kmajor(ka + kk * 2 * kQLbo, kQLbo, kQSbo), idS, kk > 0 ? 1u : 0u);
-          tc::mma_commit(&sm.bs[(g + 1) & 1]);
-        }
-      }
-      // (b) S(j) complete; its K~ buffer is free for K~(j+2)
-      ok = wait(&sm.bs[sb], 6 + sb);
-      if (j + 2 < NSt && ok) copy_rows(sm.k[sb], kb, s0 + 2 * kT, false, &sm.bk[sb]);
-      // (c) Toeplitz weights of (t0, s0): fs[idx] = f[t - s] (+ D at t = s), idx = t - s - (t0 - s0) + 127
-      for (int idx = tid; idx < 2 * kT - 1; idx += kThr2) {
-        const int d = idx - (kT - 1) + (t0 - s0);
-        float w = (d >= 0 && d < L) ? (L <= kMaxLf ? frow[d] : fh[d]) : 0.f;
-        if (d == 0) w += dh;
-        sm.fs[sb][idx] = w;
-      }
-      // (d) O(j-2) complete: P tile sb and V buffer (g+1)%3 are free
-      if (j >= 2) ok = ok & wait(&sm.bo[sb], 8 + sb);
-      if (cta_or(!ok)) { failed = true; break; }
-      tc::fence_after_sync();
-      if (j + 1 < NSt) copy_rows(sm.v[(g + 1) % 3], vb, s0 + kT, true, &sm.bv[(g + 1) % 3]);
-      // (e) P = S(j) (.) weights, rounded to the operand type, into P tile sb (K-major)
-      const uint32_t tS = tmem + (uint32_t)(128 * sb);
-      uint8_t* pt = sm.p[sb];
-      {
-        const int c = 32 * quarter;
-        float sv[2][16];
-        tc::tmem_ld16x2_wait(tS + lane_off + (uint32_t)c, tS + lane_off + (uint32_t)(c + 16), sv[0], sv[1]);
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int cc = c + 16 * hh;
-          uint32_t pw[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float a = sv[hh][2 * i] * sm.fs[sb][row - (cc + 2 * i) + (kT - 1)];
-            const float bb = sv[hh][2 * i + 1] * sm.fs[sb][row - (cc + 2 * i + 1) + (kT - 1)];
-            pw[i] = Bits<T>::pack(a, bb);
-          }
-          *reinterpret_cast<uint4*>(pt + (uint32_t)(row >> 3) * kPSbo + (uint32_t)(cc >> 3) * kPLbo + (row & 7) * 16) =
-              make_uint4(pw[0], pw[1], pw[2], pw[3]);
-          *reinterpret_cast<uint4*>(pt + (uint32_t)(row >> 3) * kPSbo + (uint32_t)((cc + 8) >> 3) * kPLbo +
-                                    (row & 7) * 16) = make_uint4(pw[4], pw[5], pw[6], pw[7]);
-        }
-      }
-      tc::fence_smem_to_async();
-      tc::fence_before_sync();
-      // (f) O += P(j) V(j)
-      ok = wait(&sm.bv[g % 3], 3 + (int)(g % 3));
-      if (cta_or(!ok)) { failed = true; break; }
-      tc::fence_after_sync();
-      if (tid == 0) {
-        tc::fence_smem_to_async();
-        const uint32_t pa = tc::smem_u32(pt), va = tc::smem_u32(sm.v[g % 3]);
-#pragma unroll
-        for (int kk = 0; kk < kT / 16; ++kk)
-          tc::mma_f16(tO, tc::desc_kmajor(pa + kk * 2 * kPLbo, kPLbo, kPSbo),
-                      tc::desc_kmajor(va + kk * 2 * kVLbo, kVLbo, kVSbo), idO, (j > 0 || kk > 0) ? 1u : 0u);
-        tc::mma_commit(&sm.bo[sb]);
-      }
-    }
-    if (failed) break;
-    // ---- the item's last O accumulations (consumed in order), then O -> global
-    const long long gl = gs + NSt - 1;
-    if (NSt >= 2) ok = wait(&sm.bo[(gl - 1) & 1], 8 + (int)((gl - 1) & 1));
-    ok = ok & wait(&sm.bo[gl & 1], 8 + (int)(gl & 1));
-    if (cta_or(!ok)) { failed = true; break; }
-    tc::fence_after_sync();
-    {
-      const int t = t0 + row;
-      float ov[1][16];
-      tc::tmem_ld16_wait(tO + lane_off + (uint32_t)(16 * quarter), ov[0]);
-      if (t < L) {
-        uint16_t* orow = reinterpret_cast<uint16_t*>(o) + base + (size_t)t * dm + 16 * quarter;
-#pragma unroll
-        for (int hh = 0; hh < 1; ++hh) {
-          uint4 lo, hi;
-          lo.x = Bits<T>::pack(ov[hh][0], ov[hh][1]);
-          lo.y = Bits<T>::pack(ov[hh][2], ov[hh][3]);
-          lo.z = Bits<T>::pack(ov[hh][4], ov[hh][5]);
-          lo.w = Bits<T>::pack(ov[hh][6], ov[hh][7]);
-          hi.x = Bits<T>::pack(ov[hh][8], ov[hh][9]);
-          hi.y = Bits<T>::pack(ov[hh][10], ov[hh][11]);
-          hi.z = Bits<T>::pack(ov[hh][12], ov[hh][13]);
-          hi.w = Bits<T>::pack(ov[hh][14], ov[hh][15]);
-          *reinterpret_cast<uint4*>(orow + 16 * hh) = lo;
-          *reinterpret_cast<uint4*>(orow + 16 * hh + 8) = hi;
-        }
-      }
-    }
-    tc::fence_before_sync();
-    __syncthreads();  // O read out before the next item's first O-MMA; Q buffer free
-    gs += NSt;
-  }
-  cp_async_wait_all();
-  if (failed && tid == 0) atomicAdd(&g_mixer_timeouts, 1u);
-  tc::fence_before_sync();
-  __syncthreads();
-  if (warp == 0) tc::tmem_dealloc(tmem, 512);
-}
-
 template <typename T>
 static cudaError_t mixer_tc_t(const void* q, const void* k, const void* v, const float* Cs, const float* f,
                               const float* D, void* o, void* kt, int B, int L, int heads, int S, cudaStream_t st) {
@@ -575,13 +332,12 @@ static cudaError_t mixer_tc_t(const void* q, const void* k, const void* v, const
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t smem = sizeof(Mix2Smem) + (size_t)(L <= kMaxLf ? L : 0) * sizeof(float) + 1024;
-  e = smem_optin<h3_mixer_tc2_kernel<T>>(smem);
+  const size_t smem = sizeof(MixSmem) + 1024;
+  auto kern = h3_mixer_tc_kernel<T>;
+  e = smem_optin<h3_mixer_tc_kernel<T>>(smem);
   if (e != cudaSuccess) return e;
-  const long long nitems = (long long)B * heads * ((L + kT - 1) / kT);
-  const int grid = (int)(nitems < num_sms() ? nitems : num_sms());
-  h3_mixer_tc2_kernel<T><<<grid, kThr2, smem, st>>>((const T*)q, (const T*)kt, (const T*)v, f, D, (T*)o, B, L,
-                                                    heads);
+  dim3 grid((L + kT - 1) / kT, heads, B);
+  kern<<<grid, kThr, smem, st>>>((const T*)q, (const T*)kt, (const T*)v, f, D, (T*)o, L, heads);
   return cudaGetLastError();
 }
 

@@ -85,69 +85,67 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 
 template <int NC>
-struct StateSmem {
-  uint8_t ph[kTab];                // A: P hi, 128 rows (2n + re/im) x 128 K (il)
-  uint8_t pl[kTab];                // A: P lo
-  uint8_t ub[2][(NC / 8) * kSbo];  // B: u chunk, NC rows (ih) x 128 K (il), double-buffered
-  uint64_t mbar;
-  uint32_t tmem_base;
-};
-
-template <int NC>
-struct CorrSmem {
-  uint8_t ahh[kTab];               // A: AH hi, 128 rows (th) x 128 K (2n + re/im)
-  uint8_t ahl[kTab];               // A: AH lo
-  uint8_t qh[(NC / 8) * kSbo];     // B: Q hi, NC rows (tl) x 128 K
-  uint8_t ql[(NC / 8) * kSbo];     // B: Q lo
-  float red[kThr / 32];
-  uint64_t mbar;
-  uint32_t tmem_base;
-};
-
-template <int NC>
 constexpr uint32_t tmem_cols() {
   return NC < 32 ? 32u : (uint32_t)NC;
-}
-
-// u chunk (NC * 128 contiguous 16-bit elements) -> K-major B tile, 16 bytes per copy.
-template <int NC>
-__device__ __forceinline__ void stage_u(uint8_t* dst, const uint16_t* src, int tid) {
-  const uint32_t d0 = tc::smem_u32(dst);
-#pragma unroll
-  for (int i = 0; i < NC * 16 / kThr; ++i) {
-    const int q = tid + i * kThr;  // 16-byte vector: row ih = q / 16, K group q % 16
-    cp_async16(d0 + toff(q >> 4, q & 15), src + (size_t)q * 8);
-  }
 }
 
 }  // namespace
 
 // ---------------------------------------------------------------- A7: local end-states
-// grid (H, B), 128 threads; s_ws[((b H + h) C + c) N + n] = s_c[n].
+// grid (H, B), 256 threads; s_ws[((b H + h) C + c) N + n] = s_c[n].  Warps 0-3 and 4-7
+// cover the 128 TMEM lanes twice: each half runs the Horner recurrence over half of the
+// chunk's NC columns, and the two partial sums combine with one product by A^(128 NC/2).
+// The accumulator is double-buffered in TMEM so that chunk c+1's MMA runs during
+// chunk c's recurrence, and the u chunks are double-buffered in shared memory.
+constexpr int kThrS = 256;
+template <int NC>
+struct StateSmem2 {
+  uint8_t ph[kTab];                // A: P hi, 128 rows (2n + re/im) x 128 K (il)
+  uint8_t pl[kTab];                // A: P lo
+  uint8_t ub[2][(NC / 8) * kSbo];  // B: u chunk, NC rows (ih) x 128 K (il), double-buffered
+  float2 part[128];                // the upper half's partial sums
+  uint64_t mbar[2];
+  uint32_t tmem_base;
+};
+
+template <int NC>
+__device__ __forceinline__ void stage_u2(uint8_t* dst, const uint16_t* src, int tid) {
+  const uint32_t d0 = tc::smem_u32(dst);
+  for (int q = tid; q < NC * 16; q += kThrS)  // 16-byte vector: row ih = q / 16, K group q % 16
+    cp_async16(d0 + toff(q >> 4, q & 15), src + (size_t)q * 8);
+}
+
 template <typename T, int NC>
-__global__ void __launch_bounds__(kThr, 2) sp_state_tc_kernel(const T* __restrict__ u, const float* __restrict__ dt,
-                                                               const float2* __restrict__ lam,
-                                                               const float2* __restrict__ Bp, int H, int L, int N,
-                                                               float2* __restrict__ s_ws) {
+__global__ void __launch_bounds__(kThrS, 2) sp_state_tc_kernel(const T* __restrict__ u, const float* __restrict__ dt,
+                                                                const float2* __restrict__ lam,
+                                                                const float2* __restrict__ Bp, int H, int L, int N,
+                                                                float2* __restrict__ s_ws) {
   extern __shared__ __align__(1024) uint8_t smraw[];
-  StateSmem<NC>& sm = *reinterpret_cast<StateSmem<NC>*>(smraw);
+  StateSmem2<NC>& sm = *reinterpret_cast<StateSmem2<NC>*>(smraw);
   constexpr int Tc = NC * kKS;
+  constexpr int HC = NC / 2;  // columns per half
   const int h = blockIdx.x, b = blockIdx.y;
   const int C = L / Tc;
   const int tid = threadIdx.x, warp = tid >> 5;
+  const int lane = tid & 127, half = tid >> 7;
   const float d = dt[h];
   const uint16_t* urow = reinterpret_cast<const uint16_t*>(u) + ((size_t)b * H + h) * (size_t)L;
 
-  if (warp == 0) tc::tmem_alloc(&sm.tmem_base, tmem_cols<NC>());
+  if (warp == 0) tc::tmem_alloc(&sm.tmem_base, 2 * tmem_cols<NC>());
   if (tid == 0) {
-    tc::mbar_init(&sm.mbar, 1);
+    tc::mbar_init(&sm.mbar[0], 1);
+    tc::mbar_init(&sm.mbar[1], 1);
     tc::fence_mbar_init();
   }
-  stage_u<NC>(sm.ub[0], urow, tid);
+  stage_u2<NC>(sm.ub[0], urow, tid);
   cp_async_commit();
+  if (C > 1) {
+    stage_u2<NC>(sm.ub[1], urow + (size_t)Tc, tid);
+    cp_async_commit();
+  }
 
   // P[2n][il] + i P[2n+1][il] = A_n^(127 - il): one exact power per 8 il, then a short chain.
-  for (int it = tid; it < 64 * 16; it += kThr) {
+  for (int it = tid; it < 64 * 16; it += kThrS) {
     const int n = it >> 4, g = it & 15;
     float re[8], im[8];
     if (n < N) {
@@ -176,101 +174,148 @@ __global__ void __launch_bounds__(kThr, 2) sp_state_tc_kernel(const T* __restric
     *reinterpret_cast<uint4*>(sm.pl + toff(2 * n + 1, g)) = make_uint4(il_[0], il_[1], il_[2], il_[3]);
   }
 
-  // this lane's mode: row r = tid -> mode tid / 2, real (even) or imaginary (odd) part
-  const int n = tid >> 1, part = tid & 1;
-  float2 w128 = make_float2(0.f, 0.f), bn = make_float2(0.f, 0.f);
+  // this lane's mode: row r = lane -> mode lane / 2, real (even) or imaginary (odd) part
+  const int n = lane >> 1, part = lane & 1;
+  float2 w128 = make_float2(0.f, 0.f), whalf = make_float2(0.f, 0.f), bn = make_float2(0.f, 0.f);
   if (n < N) {
     const float2 lm = lam[(size_t)h * N + n];
     w128 = ssm_pow(d, lm.x, lm.y, (double)kKS);
+    whalf = ssm_pow(d, lm.x, lm.y, (double)kKS * HC);
     bn = Bp[(size_t)h * N + n];
   }
   const uint32_t idesc = tc::idesc_f16(128, NC, Op16<T>::bf16);
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  uint32_t phase = 0;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+  uint32_t phase = 0;  // bit b: parity of mbar[b]
   bool failed = false;
-  uint32_t tmem = 0;
-
+  auto issue = [&](int c) {  // MMA of chunk c into TMEM buffer c & 1
+    const uint32_t pa = tc::smem_u32(sm.ph), pb = tc::smem_u32(sm.pl), ua = tc::smem_u32(sm.ub[c & 1]);
+    const uint32_t tm = sm.tmem_base + (uint32_t)((c & 1) * tmem_cols<NC>());
+#pragma unroll
+    for (int kk = 0; kk < kKS / 16; ++kk)
+      tc::mma_f16(tm, tc::desc_kmajor(pa + kk * 2 * kLbo, kLbo, kSbo), tc::desc_kmajor(ua + kk * 2 * kLbo, kLbo, kSbo),
+                  idesc, kk > 0 ? 1u : 0u);
+#pragma unroll
+    for (int kk = 0; kk < kKS / 16; ++kk)
+      tc::mma_f16(tm, tc::desc_kmajor(pb + kk * 2 * kLbo, kLbo, kSbo), tc::desc_kmajor(ua + kk * 2 * kLbo, kLbo, kSbo),
+                  idesc, 1u);
+    tc::mma_commit(&sm.mbar[c & 1]);
+  };
+  // chunk 0 landed (chunk 1 may still be in flight)
+  if (C > 1) cp_async_wait<1>(); else cp_async_wait<0>();
+  tc::fence_smem_to_async();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (tid == 0) issue(0);
   for (int c = 0; c < C; ++c) {
-    if (c + 1 < C) {
-      stage_u<NC>(sm.ub[(c + 1) & 1], urow + (size_t)(c + 1) * Tc, tid);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
+    if (c + 1 < C) {  // chunk c+1's MMA (its u has landed; its TMEM buffer was read by chunk c-1's recurrence)
       cp_async_wait<0>();
+      tc::fence_smem_to_async();
+      tc::fence_before_sync();
+      __syncthreads();
+      tc::fence_after_sync();
+      if (tid == 0) issue(c + 1);
     }
-    tc::fence_smem_to_async();
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    tmem = sm.tmem_base;
-    if (tid == 0) {
-      const uint32_t pa = tc::smem_u32(sm.ph), pb = tc::smem_u32(sm.pl), ua = tc::smem_u32(sm.ub[c & 1]);
-#pragma unroll
-      for (int kk = 0; kk < kKS / 16; ++kk)
-        tc::mma_f16(tmem, tc::desc_kmajor(pa + kk * 2 * kLbo, kLbo, kSbo),
-                    tc::desc_kmajor(ua + kk * 2 * kLbo, kLbo, kSbo), idesc, kk > 0 ? 1u : 0u);
-#pragma unroll
-      for (int kk = 0; kk < kKS / 16; ++kk)
-        tc::mma_f16(tmem, tc::desc_kmajor(pb + kk * 2 * kLbo, kLbo, kSbo),
-                    tc::desc_kmajor(ua + kk * 2 * kLbo, kLbo, kSbo), idesc, 1u);
-      tc::mma_commit(&sm.mbar);
-    }
-    const bool ok = tc::mbar_wait_bounded(&sm.mbar, phase, kWaitNs);
-    phase ^= 1u;
+    const bool ok = tc::mbar_wait_bounded(&sm.mbar[c & 1], (phase >> (c & 1)) & 1u, kWaitNs);
+    phase ^= 1u << (c & 1);
     if (__syncthreads_or(!ok)) {
       failed = true;
       break;
     }
     tc::fence_after_sync();
-    float z[NC];
+    // chunk c's u buffer is free: chunk c+2 comes in
+    if (c + 2 < C) {
+      stage_u2<NC>(sm.ub[c & 1], urow + (size_t)(c + 2) * Tc, tid);
+      cp_async_commit();
+    }
+    // Horner in A^128 over this half's columns ih = HC half .. HC half + HC - 1
+    const uint32_t tm = sm.tmem_base + (uint32_t)((c & 1) * tmem_cols<NC>());
+    float z[HC];
 #pragma unroll
-    for (int j = 0; j < NC; j += 16) tc::tmem_ld16_wait(tmem + lane_off + (uint32_t)j, z + j);
-    // Horner in A^128 over ih: R = sum_ih z[ih] A^(128 (NC-1-ih)) (complex, from a real row)
+    for (int j = 0; j < HC; j += 8) {
+      uint32_t v[8];
+      tc::tmem_ld8(tm + lane_off + (uint32_t)(HC * half + j), v);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        tc::tmem_regs_ready(v[e]);
+        z[j + e] = __uint_as_float(v[e]);
+      }
+    }
     float ar = 0.f, ai = 0.f;
 #pragma unroll
-    for (int ih = 0; ih < NC; ++ih) {
+    for (int ih = 0; ih < HC; ++ih) {
       const float nr = fmaf(ar, w128.x, fmaf(-ai, w128.y, z[ih]));
       ai = fmaf(ar, w128.y, ai * w128.x);
       ar = nr;
     }
-    // even lane holds R_re-row, odd lane R_im-row: sum = R_re + i R_im
-    const float pr = __shfl_xor_sync(0xffffffffu, ar, 1);
-    const float pi = __shfl_xor_sync(0xffffffffu, ai, 1);
-    if (part == 0 && n < N) {
-      const float2 s = make_float2(ar - pi, ai + pr);
-      s_ws[(((size_t)b * H + h) * C + c) * N + n] = cmul(s, bn);
+    // lower half: times A^(128 HC) (its columns come HC blocks earlier), plus the upper half
+    if (half == 1) sm.part[lane] = make_float2(ar, ai);
+    tc::fence_before_sync();
+    __syncthreads();
+    if (half == 0) {
+      const float2 lo = cmul(make_float2(ar, ai), whalf);
+      const float2 hi = sm.part[lane];
+      ar = lo.x + hi.x;
+      ai = lo.y + hi.y;
+      // even lane holds the R_re row, odd lane the R_im row: sum = R_re + i R_im
+      const float pr = __shfl_xor_sync(0xffffffffu, ar, 1);
+      const float pi = __shfl_xor_sync(0xffffffffu, ai, 1);
+      if (part == 0 && n < N) {
+        const float2 sres = make_float2(ar - pi, ai + pr);
+        s_ws[(((size_t)b * H + h) * C + c) * N + n] = cmul(sres, bn);
+      }
     }
   }
   cp_async_wait<0>();
   if (failed && tid == 0) atomicAdd(&g_sp_tc_timeouts, 1u);
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 0) tc::tmem_dealloc(sm.tmem_base, tmem_cols<NC>());
+  if (warp == 0) tc::tmem_dealloc(sm.tmem_base, 2 * tmem_cols<NC>());
 }
 
 // ---------------------------------------------------------------- A9: correction
-// grid (H, B), 128 threads; y[b, h, c T + t] += correction, chunks c >= c_begin.
+// grid (H, B), 256 threads; y[b, h, c T + t] += correction, chunks c >= c_begin.  Warps 0-3
+// and 4-7 cover the 128 TMEM lanes twice and split each row's NC outputs in halves.  The
+// accumulator is double-buffered in TMEM: chunk c+1's operand is built and its MMA issued
+// before chunk c's epilogue runs; each thread's y values of the next chunk are loaded
+// while the current chunk finishes.
+template <int NC>
+struct CorrSmem2 {
+  uint8_t ahh[kTab];               // A: AH hi, 128 rows (th) x 128 K (2n + re/im)
+  uint8_t ahl[kTab];               // A: AH lo
+  uint8_t qh[(NC / 8) * kSbo];     // B: Q hi, NC rows (tl) x 128 K
+  uint8_t ql[(NC / 8) * kSbo];     // B: Q lo
+  float red[kThrS / 32];
+  uint64_t mbar[2];
+  uint32_t tmem_base;
+};
+
 template <typename T, int NC>
-__global__ void __launch_bounds__(kThr, 2) sp_corr_tc_kernel(T* __restrict__ y, const float* __restrict__ dt,
-                                                              const float2* __restrict__ lam,
-                                                              const float2* __restrict__ Cp,
-                                                              const float2* __restrict__ x_ws, int H, int L, int N,
-                                                              int c_begin) {
+__global__ void __launch_bounds__(kThrS, 2) sp_corr_tc_kernel(T* __restrict__ y, const float* __restrict__ dt,
+                                                               const float2* __restrict__ lam,
+                                                               const float2* __restrict__ Cp,
+                                                               const float2* __restrict__ x_ws, int H, int L, int N,
+                                                               int c_begin) {
   extern __shared__ __align__(1024) uint8_t smraw[];
-  CorrSmem<NC>& sm = *reinterpret_cast<CorrSmem<NC>*>(smraw);
+  CorrSmem2<NC>& sm = *reinterpret_cast<CorrSmem2<NC>*>(smraw);
   constexpr int Tc = NC * kKS;
+  constexpr int HC = NC / 2;               // outputs per thread per chunk
+  constexpr int kGr = (NC / 8 + 3) / 4;    // Q row groups per thread (groups gq + 4 r < NC / 8)
   const int h = blockIdx.x, b = blockIdx.y;
   const int C = L / Tc;
   const int tid = threadIdx.x, warp = tid >> 5;
+  const int lane = tid & 127, half = tid >> 7;
   const float d = dt[h];
 
-  if (warp == 0) tc::tmem_alloc(&sm.tmem_base, tmem_cols<NC>());
+  if (warp == 0) tc::tmem_alloc(&sm.tmem_base, 2 * tmem_cols<NC>());
   if (tid == 0) {
-    tc::mbar_init(&sm.mbar, 1);
+    tc::mbar_init(&sm.mbar[0], 1);
+    tc::mbar_init(&sm.mbar[1], 1);
     tc::fence_mbar_init();
   }
   // AH[th][2n] + i AH[th][2n+1] = A_n^(NC th): one exact power per 8 rows, then a chain in A^NC.
-  for (int it = tid; it < 64 * 16; it += kThr) {
+  for (int it = tid; it < 64 * 16; it += kThrS) {
     const int n = it & 63, g = it >> 6;
     float2 p = make_float2(0.f, 0.f), step = make_float2(0.f, 0.f);
     if (n < N) {
@@ -288,9 +333,8 @@ __global__ void __launch_bounds__(kThr, 2) sp_corr_tc_kernel(T* __restrict__ y, 
       p = cmul(p, step);
     }
   }
-  // this thread's mode and Q row groups: n = tid % 64, tl groups (tid / 64) + 2 r
-  constexpr int kGr = NC / 16;
-  const int n = tid & 63;
+  // this thread's mode and Q row groups: n = tid % 64, tl groups gq + 4 r (gq = tid / 64)
+  const int n = tid & 63, gq = tid >> 6;
   float2 a1 = make_float2(0.f, 0.f), cn = make_float2(0.f, 0.f), st[kGr];
 #pragma unroll
   for (int r = 0; r < kGr; ++r) st[r] = make_float2(0.f, 0.f);
@@ -299,21 +343,16 @@ __global__ void __launch_bounds__(kThr, 2) sp_corr_tc_kernel(T* __restrict__ y, 
     a1 = ssm_pow(d, lm.x, lm.y, 1.0);
     cn = Cp[(size_t)h * N + n];
 #pragma unroll
-    for (int r = 0; r < kGr; ++r) st[r] = ssm_pow(d, lm.x, lm.y, 8.0 * ((tid >> 6) + 2 * r) + 1.0);
+    for (int r = 0; r < kGr; ++r)
+      if (gq + 4 * r < NC / 8) st[r] = ssm_pow(d, lm.x, lm.y, 8.0 * (gq + 4 * r) + 1.0);
   }
   const uint32_t idesc = tc::idesc_f16(128, NC, 0);
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  uint32_t phase = 0;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+  uint32_t phase = 0;  // bit b: parity of mbar[b]
   bool failed = false;
-  uint32_t tmem = 0;
   const size_t rowoff = ((size_t)b * H + h) * (size_t)L;
-
-  for (int c = c_begin; c < C; ++c) {
-    // this lane's NC outputs t = NC * tid + tl: issue the loads of y early
-    uint16_t* yp = reinterpret_cast<uint16_t*>(y) + rowoff + (size_t)c * Tc + (size_t)NC * tid;
-    uint4 yv[NC / 8];
-#pragma unroll
-    for (int i = 0; i < NC / 8; ++i) yv[i] = *reinterpret_cast<const uint4*>(yp + 8 * i);
+  // Q of chunk c into shared memory; returns the inverse of its power-of-two scale
+  auto build_q = [&](int c) -> float {
     float2 w = make_float2(0.f, 0.f);
     if (n < N) {
       const float2 x = x_ws[(((size_t)b * H + h) * C + c) * N + n];
@@ -326,7 +365,9 @@ __global__ void __launch_bounds__(kThr, 2) sp_corr_tc_kernel(T* __restrict__ y, 
     mx = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(mx)));
     if ((tid & 31) == 0) sm.red[warp] = mx;
     __syncthreads();
-    mx = fmaxf(fmaxf(sm.red[0], sm.red[1]), fmaxf(sm.red[2], sm.red[3]));
+    mx = 0.f;
+#pragma unroll
+    for (int i = 0; i < kThrS / 32; ++i) mx = fmaxf(mx, sm.red[i]);
     int ex = 0;
     float scale = 1.f, inv = 1.f;
     if (mx > 0.f && mx <= 3.0e38f) {
@@ -339,7 +380,8 @@ __global__ void __launch_bounds__(kThr, 2) sp_corr_tc_kernel(T* __restrict__ y, 
     // Q[tl][2n] - i Q[tl][2n+1] = w_n A_n^(tl+1)
 #pragma unroll
     for (int r = 0; r < kGr; ++r) {
-      const int tg = (tid >> 6) + 2 * r;
+      const int tg = gq + 4 * r;
+      if (tg >= NC / 8) continue;
       float2 p = cmul(w, st[r]);
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
@@ -351,57 +393,94 @@ __global__ void __launch_bounds__(kThr, 2) sp_corr_tc_kernel(T* __restrict__ y, 
         p = cmul(p, a1);
       }
     }
+    return inv;
+  };
+  auto issue = [&](int c) {
+    const uint32_t ah = tc::smem_u32(sm.ahh), al = tc::smem_u32(sm.ahl);
+    const uint32_t qh = tc::smem_u32(sm.qh), ql = tc::smem_u32(sm.ql);
+    const uint32_t tm = sm.tmem_base + (uint32_t)((c & 1) * tmem_cols<NC>());
+#pragma unroll
+    for (int kk = 0; kk < kKS / 16; ++kk)
+      tc::mma_f16(tm, tc::desc_kmajor(ah + kk * 2 * kLbo, kLbo, kSbo), tc::desc_kmajor(qh + kk * 2 * kLbo, kLbo, kSbo),
+                  idesc, kk > 0 ? 1u : 0u);
+#pragma unroll
+    for (int kk = 0; kk < kKS / 16; ++kk)
+      tc::mma_f16(tm, tc::desc_kmajor(ah + kk * 2 * kLbo, kLbo, kSbo), tc::desc_kmajor(ql + kk * 2 * kLbo, kLbo, kSbo),
+                  idesc, 1u);
+#pragma unroll
+    for (int kk = 0; kk < kKS / 16; ++kk)
+      tc::mma_f16(tm, tc::desc_kmajor(al + kk * 2 * kLbo, kLbo, kSbo), tc::desc_kmajor(qh + kk * 2 * kLbo, kLbo, kSbo),
+                  idesc, 1u);
+    tc::mma_commit(&sm.mbar[c & 1]);
+  };
+  // this thread's outputs of chunk c: t = NC lane + HC half + j, j < HC
+  auto yptr = [&](int c) {
+    return reinterpret_cast<uint16_t*>(y) + rowoff + (size_t)c * Tc + (size_t)NC * lane + (size_t)HC * half;
+  };
+  if (c_begin < C) {
+    float inv_cur = build_q(c_begin);
     tc::fence_smem_to_async();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    tmem = sm.tmem_base;
-    if (tid == 0) {
-      const uint32_t ah = tc::smem_u32(sm.ahh), al = tc::smem_u32(sm.ahl);
-      const uint32_t qh = tc::smem_u32(sm.qh), ql = tc::smem_u32(sm.ql);
+    if (tid == 0) issue(c_begin);
+    uint4 yv[HC / 8];
+    {
+      const uint16_t* yp = yptr(c_begin);
 #pragma unroll
-      for (int kk = 0; kk < kKS / 16; ++kk)
-        tc::mma_f16(tmem, tc::desc_kmajor(ah + kk * 2 * kLbo, kLbo, kSbo),
-                    tc::desc_kmajor(qh + kk * 2 * kLbo, kLbo, kSbo), idesc, kk > 0 ? 1u : 0u);
-#pragma unroll
-      for (int kk = 0; kk < kKS / 16; ++kk)
-        tc::mma_f16(tmem, tc::desc_kmajor(ah + kk * 2 * kLbo, kLbo, kSbo),
-                    tc::desc_kmajor(ql + kk * 2 * kLbo, kLbo, kSbo), idesc, 1u);
-#pragma unroll
-      for (int kk = 0; kk < kKS / 16; ++kk)
-        tc::mma_f16(tmem, tc::desc_kmajor(al + kk * 2 * kLbo, kLbo, kSbo),
-                    tc::desc_kmajor(qh + kk * 2 * kLbo, kLbo, kSbo), idesc, 1u);
-      tc::mma_commit(&sm.mbar);
+      for (int i = 0; i < HC / 8; ++i) yv[i] = *reinterpret_cast<const uint4*>(yp + 8 * i);
     }
-    const bool ok = tc::mbar_wait_bounded(&sm.mbar, phase, kWaitNs);
-    phase ^= 1u;
-    if (__syncthreads_or(!ok)) {
-      failed = true;
-      break;
-    }
-    tc::fence_after_sync();
+    for (int c = c_begin; c < C; ++c) {
+      const bool ok = tc::mbar_wait_bounded(&sm.mbar[c & 1], (phase >> (c & 1)) & 1u, kWaitNs);
+      phase ^= 1u << (c & 1);
+      if (__syncthreads_or(!ok)) {
+        failed = true;
+        break;
+      }
+      tc::fence_after_sync();
+      float inv_next = 1.f;
+      if (c + 1 < C) {  // chunk c+1: operand (Q is free: MMA c has read it), then its MMA
+        inv_next = build_q(c + 1);
+        tc::fence_smem_to_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+        if (tid == 0) issue(c + 1);
+      }
+      // epilogue of chunk c: y += correction (scale multiplied back out exactly)
+      const uint32_t tm = sm.tmem_base + (uint32_t)((c & 1) * tmem_cols<NC>());
+      uint16_t* yp = yptr(c);
 #pragma unroll
-    for (int j = 0; j < NC; j += 16) {
-      float v[16];
-      tc::tmem_ld16_wait(tmem + lane_off + (uint32_t)j, v);
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint32_t* wv = reinterpret_cast<uint32_t*>(&yv[j / 8 + q]);
+      for (int j = 0; j < HC; j += 8) {
+        uint32_t v[8];
+        tc::tmem_ld8(tm + lane_off + (uint32_t)(HC * half + j), v);
+        tc::tmem_wait_ld();
+        uint32_t* wv = reinterpret_cast<uint32_t*>(&yv[j / 8]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float lo = fmaf(v[8 * q + 2 * e], inv, Op16<T>::back(wv[e] & 0xffffu));
-          const float hi = fmaf(v[8 * q + 2 * e + 1], inv, Op16<T>::back(wv[e] >> 16));
+          tc::tmem_regs_ready(v[2 * e]);
+          tc::tmem_regs_ready(v[2 * e + 1]);
+          const float lo = fmaf(__uint_as_float(v[2 * e]), inv_cur, Op16<T>::back(wv[e] & 0xffffu));
+          const float hi = fmaf(__uint_as_float(v[2 * e + 1]), inv_cur, Op16<T>::back(wv[e] >> 16));
           wv[e] = Op16<T>::bits(lo) | (Op16<T>::bits(hi) << 16);
         }
       }
-    }
 #pragma unroll
-    for (int i = 0; i < NC / 8; ++i) *reinterpret_cast<uint4*>(yp + 8 * i) = yv[i];
+      for (int i = 0; i < HC / 8; ++i) *reinterpret_cast<uint4*>(yp + 8 * i) = yv[i];
+      if (c + 1 < C) {
+        const uint16_t* yn = yptr(c + 1);
+#pragma unroll
+        for (int i = 0; i < HC / 8; ++i) yv[i] = *reinterpret_cast<const uint4*>(yn + 8 * i);
+      }
+      inv_cur = inv_next;
+      tc::fence_before_sync();
+      __syncthreads();  // TMEM buffer c & 1 read before chunk c+2's MMA is issued into it
+    }
   }
   if (failed && tid == 0) atomicAdd(&g_sp_tc_timeouts, 1u);
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 0) tc::tmem_dealloc(sm.tmem_base, tmem_cols<NC>());
+  if (warp == 0) tc::tmem_dealloc(sm.tmem_base, 2 * tmem_cols<NC>());
 }
 
 // ---------------------------------------------------------------- launchers
@@ -415,17 +494,17 @@ static cudaError_t sp_tc_t(const void* u, void* y, const float* dt, const float*
                            bool corr, cudaStream_t st) {
   dim3 grid(H, B);
   if (!corr) {
-    const size_t smem = sizeof(StateSmem<NC>) + 1024;
+    const size_t smem = sizeof(StateSmem2<NC>) + 1024;
     auto kern = sp_state_tc_kernel<T, NC>;
     cudaError_t e = smem_optin<sp_state_tc_kernel<T, NC>>(smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThr, smem, st>>>((const T*)u, dt, (const float2*)lam, (const float2*)Bp, H, L, N, (float2*)s_ws);
+    kern<<<grid, kThrS, smem, st>>>((const T*)u, dt, (const float2*)lam, (const float2*)Bp, H, L, N, (float2*)s_ws);
   } else {
-    const size_t smem = sizeof(CorrSmem<NC>) + 1024;
+    const size_t smem = sizeof(CorrSmem2<NC>) + 1024;
     auto kern = sp_corr_tc_kernel<T, NC>;
     cudaError_t e = smem_optin<sp_corr_tc_kernel<T, NC>>(smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThr, smem, st>>>((T*)y, dt, (const float2*)lam, (const float2*)Cp, (const float2*)x_ws, H, L, N,
+    kern<<<grid, kThrS, smem, st>>>((T*)y, dt, (const float2*)lam, (const float2*)Cp, (const float2*)x_ws, H, L, N,
                                    c_begin);
   }
   return cudaGetLastError();

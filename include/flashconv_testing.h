@@ -33,6 +33,13 @@ FC_TEST_API int fc_selftest_umma(const void* A, const void* B, float* D, int* er
 FC_TEST_API int fc_selftest_umma2(const void* A, const void* B, float* D, int* err, int N, int K, int bf16, int a_mn,
                                   int b_mn, int a_lbo, int a_sbo, int b_lbo, int b_sbo, void* stream);
 
+/* The same product with A held in tensor memory: each row of A (K 16-bit
+ * elements) is written with tcgen05.st, two elements per 32-bit column (even
+ * k in the low half), and the MMA reads A from there.  Same limits and
+ * returns as fc_selftest_umma. */
+FC_TEST_API int fc_selftest_umma_tmem_a(const void* A, const void* B, float* D, int* err, int N, int K, int bf16,
+                                        void* stream);
+
 /* Number of tensor-core CTAs (all tcgen05 kernels of the library, since load)
  * that gave up waiting for MMA completion after their bounded wait; each such
  * CTA skipped its remaining work and freed its tensor memory.  0 in normal
