@@ -65,7 +65,7 @@ cudaError_t run_ssm_conv(const void* u, const float* dt, const float* lambda, co
                          cudaStream_t st) {
   const SsmArgs none{nullptr, nullptr, nullptr, nullptr, 0};
   cudaError_t e;
-  if (fftconv_tc_supported(L, dtype)) {  // filter kernel, then the tensor-core convolution
+  if (fftconv_tc_supported(L, dtype, B)) {  // filter kernel, then the tensor-core convolution
     e = launch_ssm_gen(dt, lambda, Bp, Cp, H, N, L, f, st);
     if (e != cudaSuccess) return e;
     return launch_fftconv_tc(u, f, D, y, B, H, L, dtype, true, st);
@@ -138,7 +138,7 @@ FC_API fc_status fftconv_fwd(const void* u, const float* f, const float* D, void
   FC_REQUIRE(f && D, FC_EINVAL, "null f or D");
   FC_REQUIRE(aligned(f, 16) && aligned(D, 4), FC_EINVAL, "f must be 16-byte aligned, D 4-byte aligned");
   FC_REQUIRE(L >= 1 && L <= 8192, FC_EUNSUPPORTED, "fftconv_fwd: L must be in [1, 8192] (got %d)", L);
-  if (fc::fftconv_tc_supported(L, dtype))
+  if (fc::fftconv_tc_supported(L, dtype, B))
     return cuda_status(fc::launch_fftconv_tc(u, f, D, y, B, H, L, dtype, false, (cudaStream_t)stream),
                        "fftconv_fwd (tensor cores) launch");
   if (fc::fftconv_tcl_supported(L, dtype))
@@ -173,7 +173,7 @@ FC_API fc_status fftconv_bwd(const void* dy, const void* u, const float* f, cons
                "df needs u (16-byte aligned); df, dD 4-byte aligned");
   cudaStream_t st = (cudaStream_t)stream;
   if (du) {
-    s = fc::fftconv_tc_supported(L, dtype)
+    s = fc::fftconv_tc_supported(L, dtype, B)
             ? cuda_status(fc::launch_fftconv_tc(dy, f, D, du, B, H, L, dtype, false, st, true),
                           "fftconv_bwd: du (tensor cores) launch")
         : fc::fftconv_tcl_supported(L, dtype)

@@ -76,7 +76,7 @@ cudaError_t launch_sp_adjoint_state(const float* dt, const float* lam, const flo
                                     int N, cudaStream_t st);
 
 // Tensor-core fused FFT convolution (block-FFT stages as tcgen05 GEMMs).
-bool fftconv_tc_supported(int L, int dtype);
+bool fftconv_tc_supported(int L, int dtype, int B);
 // after_filter_kernel: f is written by the kernel launched just before on the
 // same stream (ssm_gen), which lets this launch start as its programmatic
 // dependent (prologue overlapped; the filter is read only after that kernel

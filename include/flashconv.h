@@ -112,14 +112,16 @@ FC_API fc_status ssm_kernel_gen(const float* dt, const float* lambda, const floa
  * leaves the causal outputs t < L exact); B, H >= 1.  u and y may not
  * overlap.
  * Precision: FC_F32 and every L without a tensor-core kernel (L < 1024 or
- * not a power of two): float32 FFTs on the CUDA cores, one rounding at the
- * store.  16-bit I/O at L = 1024, 2048, 4096, 8192 runs the block-FFT
- * stages on the tensor cores: the filter (with D added to its tap 0) is
- * rounded to the I/O type; the DFT-128 stages take their data operand in the
- * I/O type (exact for u); the column DFT stages take float16 operands scaled
- * so that they stay within 2 max|u| (finite for |u| <= 32752); the inverse
- * stage's input is rounded to the I/O type; accumulation is float32 and y is
- * rounded once at the store. */
+ * not a power of two, or L = 1024 with B <= 2): float32 FFTs on the CUDA
+ * cores, one rounding at the store.  16-bit I/O at L = 1024 (B >= 3) and at
+ * L = 2048, 4096, 8192 runs the block-FFT stages on the tensor cores: the
+ * filter (with D added to its tap 0) is rounded to the I/O type; the DFT-128
+ * stages take their data operand in the I/O type (exact for u); at L = 1024
+ * the length-16 column DFTs, twiddles and filter product are float32
+ * register arithmetic; at L = 2048..8192 the column DFT stages take float16
+ * operands scaled so that they stay within 2 max|u| (finite for
+ * |u| <= 32752); the inverse stage's input is rounded to the I/O type;
+ * accumulation is float32 and y is rounded once at the store. */
 FC_API fc_status fftconv_fwd(const void* u, const float* f, const float* D, void* y,
                              int B, int H, int L, fc_dtype dtype, void* stream);
 

@@ -78,11 +78,13 @@ def test_fftconv_all_sizes(L, dtype):
     assert err < TOL[dtype], err
 
 
-@pytest.mark.parametrize("B,H,dtype", [(10, 3, "f16"), (1, 4, "bf16"), (2, 300, "f16"), (7, 2, "bf16")])
+@pytest.mark.parametrize("B,H,dtype", [(10, 3, "f16"), (3, 4, "bf16"), (4, 300, "f16"), (7, 2, "bf16"),
+                                       (5, 1, "f16"), (2, 5, "bf16")])
 def test_fftconv_tensor_core_batches(B, H, dtype):
-    """L = 1024 fp16/bf16 runs the tensor-core block FFT: several row-pair
-    batches per channel (B = 10), a single row, more channels than resident
-    CTAs (H = 300), odd B."""
+    """L = 1024 fp16/bf16 with B >= 3 runs the tensor-core block FFT (rounds of
+    three row pairs that may span two channels): several pairs per channel
+    (B = 10), odd B (a pair without its second row), more rounds than SMs
+    (H = 300), a single channel; B = 2 takes the CUDA-core path."""
     L = 1024
     wl = W.make_conv(B=B, H=H, L=L, N=16, dtype=dtype, seed=B * 1000 + H, dt_range=("loguniform", -3.0, -1.0))
     f32 = W.round_to(O.ssm_filter(wl.dt, wl.lam, wl.Bp, wl.Cp, L), "f32")
