@@ -454,6 +454,27 @@ def secondary_configs(T, dev, api, args, local_rank):
                       avg_launch_ms=ms, flops_note="causal half of S = Q K~^T and O = P V per (b, head)"),
         hbm_frac=(4 * units * 2) / 1e9 / (ms / 1e3) / peak,
         clocks=clocks)
+    del q, k, v, o, ws
+
+    # ---- long arbitrary filter at an EEG-clip length (fp32, B=8, H=256, L=12000): fftconv_long_fwd
+    B, H, L = 8, 256, 12000
+    rng = np.random.default_rng(12000)
+    u = T(rng.normal(size=(B, H, L)).astype(np.float32))
+    f = T((rng.normal(size=(H, L)) * np.exp(-np.arange(L) / 4000.0)).astype(np.float32))
+    D = T(rng.normal(size=H).astype(np.float32))
+    y = torch.empty_like(u)
+    ws = torch.empty(max(1, api.long_conv_workspace_bytes(B, H, L)), dtype=torch.uint8, device=dev)
+    units = B * H * L
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    ms, _ = graph_time(lambda: api.fftconv_long_fwd(u, f, D, out=y, workspace=ws), n, flush, rflush, stream)
+    clocks = sampler.stop()
+    out["longconv_f32_B8_H256_L12000"] = dict(
+        step="fftconv_long_fwd (arbitrary filter as long as the clip, 8192-blocks, fp32)", step_ms=ms,
+        value=units / (ms / 1e3), unit="conv elements/s",
+        roofline=hbm_roof("the whole long-convolution call", units * 8 + H * L * 4, ms,
+                          "u read + y written (fp32) + fp32 filter read"),
+        clocks=clocks)
     return out
 
 

@@ -23,6 +23,8 @@ SIGNATURES = {
     "fc_tc_timeouts": (ctypes.c_uint, []),
     "ssm_kernel_gen": (_i, [_fp, _fp, _fp, _fp, _i, _i, _i, _fp, _vp]),
     "fftconv_fwd": (_i, [_vp, _fp, _fp, _vp, _i, _i, _i, _i, _vp]),
+    "fftconv_long_workspace": (_sz, [_i, _i, _i]),
+    "fftconv_long_fwd": (_i, [_vp, _fp, _fp, _vp, _i, _i, _i, _vp, _sz, _i, _vp]),
     "fftconv_bwd": (_i, [_vp, _vp, _fp, _fp, _vp, _fp, _fp, _i, _i, _i, _i, _vp]),
     "ssm_conv_workspace": (_sz, [_i, _i]),
     "ssm_decode_step": (_i, [_vp, _fp, _fp, _fp, _fp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _vp]),

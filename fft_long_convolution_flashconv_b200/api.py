@@ -91,6 +91,27 @@ def fftconv_fwd(u: torch.Tensor, f: torch.Tensor, D: torch.Tensor,
     return out
 
 
+def long_conv_workspace_bytes(B: int, H: int, L: int) -> int:
+    return int(_lib.load().fftconv_long_workspace(B, H, L))
+
+
+def fftconv_long_fwd(u: torch.Tensor, f: torch.Tensor, D: torch.Tensor, out: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y = causal_conv(u, f) + D u for L up to 65536 (arbitrary filter); u: B x H x L."""
+    lib = _lib.load()
+    B, H, L = u.shape
+    f, D = _f32(f), _f32(D)
+    if out is None:
+        out = torch.empty_like(u)
+    need = int(lib.fftconv_long_workspace(B, H, L))
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=u.device)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    check(lib.fftconv_long_fwd(_ptr(u), _ptr(f), _ptr(D), _ptr(out), B, H, L, _ptr(workspace), ws_bytes,
+                               _dtype(u), _stream()), "fftconv_long_fwd")
+    return out
+
+
 def fftconv_bwd(dy: torch.Tensor, u: torch.Tensor, f: torch.Tensor, D: torch.Tensor, need_du: bool = True,
                 need_dfilter: bool = True):
     """Gradients of y = causal_conv(u, f) + D u given dy; returns (du, df, dD)

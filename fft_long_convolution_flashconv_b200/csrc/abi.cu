@@ -150,6 +150,30 @@ FC_API fc_status fftconv_fwd(const void* u, const float* f, const float* D, void
       "fftconv_fwd launch");
 }
 
+FC_API size_t fftconv_long_workspace(int B, int H, int L) {
+  if (B < 1 || H < 1 || L <= 8192 || L > 65536) return 0;
+  return fc::fftconv_long_workspace_bytes(B, H, L);
+}
+
+FC_API fc_status fftconv_long_fwd(const void* u, const float* f, const float* D, void* y, int B, int H, int L,
+                                  void* workspace, size_t ws_bytes, fc_dtype dtype, void* stream) {
+  g_err[0] = 0;
+  FC_REQUIRE(L >= 1 && L <= 65536, FC_EUNSUPPORTED, "fftconv_long_fwd: L must be in [1, 65536] (got %d)", L);
+  if (L <= 8192) return fftconv_fwd(u, f, D, y, B, H, L, dtype, stream);
+  fc_status s = check_conv_io(u, y, B, H, L, dtype);
+  if (s != FC_OK) return s;
+  FC_REQUIRE(f && D, FC_EINVAL, "null f or D");
+  FC_REQUIRE(aligned(f, 16) && aligned(D, 4), FC_EINVAL, "f must be 16-byte aligned, D 4-byte aligned");
+  const long long K = (L + 8191) / 8192;
+  FC_REQUIRE((long long)B * H * K <= (1LL << 26), FC_EUNSUPPORTED, "B * H * ceil(L / 8192) = %lld > 2^26",
+             (long long)B * H * K);
+  FC_REQUIRE(workspace && aligned(workspace, 256), FC_EINVAL, "workspace must be non-null and 256-byte aligned");
+  const size_t need = fftconv_long_workspace(B, H, L);
+  FC_REQUIRE(ws_bytes >= need, FC_EINVAL, "workspace too small: %zu < %zu bytes", ws_bytes, need);
+  return cuda_status(fc::launch_fftconv_long(u, f, D, y, B, H, L, workspace, dtype, (cudaStream_t)stream),
+                     "fftconv_long_fwd launch");
+}
+
 FC_API fc_status fftconv_bwd(const void* dy, const void* u, const float* f, const float* D, void* du, float* df,
                              float* dD, int B, int H, int L, fc_dtype dtype, void* stream) {
   g_err[0] = 0;

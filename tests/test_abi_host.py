@@ -29,7 +29,8 @@ def test_header_declares_expected_entry_points():
               "fftconv_statepass_workspace", "h3_mixer_workspace", "ssm_conv_fwd", "ssm_conv_workspace",
               "fc_last_error", "fc_status_string", "fc_version", "fftconv_bwd", "fc_tc_timeouts",
               "ssm_decode_step", "h3_mixer_decode_step", "h3_decode_state_bytes",
-              "fftconv_statepass_bwd", "fftconv_statepass_bwd_workspace"):
+              "fftconv_statepass_bwd", "fftconv_statepass_bwd_workspace", "fftconv_long_fwd",
+              "fftconv_long_workspace"):
         assert s in syms
 
 
@@ -169,3 +170,20 @@ def test_backward_and_decode_reject_bad_arguments():
     assert lib.h3_mixer_decode_step(P, P, P, P, P2, P, P, P2, P3, P, P, o, 1, 2, 64, 8, 4, -1, 1,
                                     None) == _lib.FC_EINVAL
     assert lib.h3_decode_state_bytes(2, 3, 64, 8) == 2 * 3 * 64 * 64 * 8 * 8
+
+
+def test_long_conv_rejects_bad_arguments():
+    lib = _lib.load()
+    y = P + (1 << 28)
+    ws = lib.fftconv_long_workspace(2, 3, 12000)
+    assert ws >= 4 * 2 * 3 * 16384 * 4
+    assert lib.fftconv_long_workspace(2, 3, 8192) == 0 and lib.fftconv_long_workspace(2, 3, 70000) == 0
+    # L out of range, missing / misaligned / small workspace, overlap
+    assert lib.fftconv_long_fwd(P, P2, P3, y, 2, 3, 70000, P3, ws, 0, None) == _lib.FC_EUNSUPPORTED
+    assert lib.fftconv_long_fwd(P, P2, P3, y, 2, 3, 12000, None, ws, 0, None) == _lib.FC_EINVAL
+    assert lib.fftconv_long_fwd(P, P2, P3, y, 2, 3, 12000, P3 + 16, ws, 0, None) == _lib.FC_EINVAL
+    assert lib.fftconv_long_fwd(P, P2, P3, y, 2, 3, 12000, P3, ws - 1, 0, None) == _lib.FC_EINVAL
+    assert "workspace too small" in _err()
+    assert lib.fftconv_long_fwd(P, P2, P3, P + 64, 2, 3, 12000, P3, ws, 0, None) == _lib.FC_EINVAL
+    # L <= 8192 goes through fftconv_fwd's validation
+    assert lib.fftconv_long_fwd(P, P2, P3, y, 2, 3, 4096, None, 0, 7, None) == _lib.FC_EINVAL

@@ -482,6 +482,31 @@ def test_fftconv_any_length(L, dtype):
     assert O.row_rel_err(host(df), rdf) < 1e-4 * max(1.0, np.log2(L * B + 1) / 4)
 
 
+@pytest.mark.parametrize("B,H,L,dtype", [(2, 3, 12000, "f32"), (3, 2, 9001, "bf16"), (1, 2, 20000, "f16"),
+                                         (2, 2, 8193, "f32"), (1, 1, 65536, "f32")])
+def test_fftconv_long_matches_oracle(B, H, L, dtype):
+    """Filters as long as the input past 8192 (12,000-step EEG-clip length,
+    non-powers of two, three and eight blocks, the first length past one
+    block): block convolutions with reversed high halves, against the direct
+    fp64 convolution."""
+    rng = np.random.default_rng(L + B)
+    u = W.round_to(rng.normal(size=(B, H, L)), dtype)
+    f = W.round_to(rng.normal(size=(H, L)) * np.exp(-np.arange(L) / (L / 3.0)), "f32")  # arbitrary, long-reaching
+    D = rng.normal(size=H)
+    y = host(api.fftconv_long_fwd(dev(u, dtype), dev(f), dev(D)))
+    ref = cref.causal_conv(u, f, D)
+    assert O.row_rel_err(y.reshape(-1, L), ref.reshape(-1, L)) < TOL[dtype]
+
+
+def test_fftconv_long_short_lengths_are_fftconv_fwd():
+    B, H, L = 3, 4, 5000
+    rng = np.random.default_rng(5)
+    u = dev(W.round_to(rng.normal(size=(B, H, L)), "f16"), "f16")
+    f = dev(rng.normal(size=(H, L)) * np.exp(-np.arange(L) / 900.0))
+    D = dev(rng.normal(size=H))
+    assert np.array_equal(host(api.fftconv_long_fwd(u, f, D)), host(api.fftconv_fwd(u, f, D)))
+
+
 def test_ssm_conv_any_length():
     wl = W.make_conv(B=2, H=6, L=1234, N=80, dtype="f32", seed=9)  # N > 64: fused generation path
     y = host(api.ssm_conv_fwd(dev(wl.u), *params(wl)))
