@@ -180,19 +180,13 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         dom_ms.append(a.elapsed_time(b))
     conv_avg = sum(dom_ms) / len(dom_ms)
-    t = torch.tensor([tot_ms, conv_avg], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    tot_ms, conv_avg = float(t[0]), float(t[1])
+    tot_ms, conv_avg = max_over_ranks([tot_ms, conv_avg], world, dev)
     ms_per_step = tot_ms / args.steps
-    value = units * world / (tot_ms / 1e3 / args.steps)
+    value = job_value(units, world, ms_per_step)
 
     # end to end through the C ABI with pinned host buffers
-    e2e_ms = e2e_fn(args.e2e_steps)
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_val = units * world / (float(te[0]) / 1e3)
+    e2e_ms, = max_over_ranks([e2e_fn(args.e2e_steps)], world, dev)
+    e2e_val = job_value(units, world, e2e_ms)
 
     peak, peak_kind = hbm_peak()
     achieved = alg_bytes / (conv_avg / 1e3) / 1e9
@@ -223,6 +217,24 @@ def run_ours(args, rank, world, local_rank):
     if args.others and rank == 0:
         res["headline_split"] = split_headline(T, dev, api, args)
     return res
+
+
+def max_over_ranks(vals, world, device):
+    """Element-wise max over ranks of per-rank device timings (ms).  Every rank
+    takes this collective step at the same point, so the slowest replica sets
+    the job's time."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def job_value(units_per_rank, world, ms_per_step):
+    """Whole-job throughput: the units every rank processed per step over the
+    (max-over-ranks) step time."""
+    return units_per_rank * world / (ms_per_step / 1e3)
 
 
 def flush_l2(wbuf, rbuf):
