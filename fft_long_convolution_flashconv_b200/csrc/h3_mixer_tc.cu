@@ -42,7 +42,7 @@ struct MixSmem {
   uint8_t k[(kT / 8) * kQSbo];      // B of S-MMA  (rows s, K = i)
   uint8_t v[2][(kT / 8) * kVLbo];   // B of O-MMA  (N = j, K = s), MN-major, double-buffered
   uint8_t p[kT * kT * 2];           // A of O-MMA  (rows t, K = s)
-  float fs[2 * kT];
+  float fs[2][2 * kT];              // Toeplitz weights of the current and the next s tile
   uint64_t mbar;
   uint32_t tmem_base;
 };
@@ -201,6 +201,21 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
         *reinterpret_cast<uint4*>(sm.v[buf] + voff(r, c8)) = make_uint4(0, 0, 0, 0);
     }
   };
+  // Toeplitz weights f[t - s] (+ D on the diagonal) of tile (t0, s0) for idx = t - s + 127 - (t0 - s0):
+  // this thread's two entries, loaded from global memory a tile ahead and stored after the P pass
+  auto weights = [&](int s0, float& w0, float& w1) {
+    const int d0 = tid - (kT - 1) + (t0 - s0), d1 = d0 + kThr;
+    w0 = (d0 >= 0 && d0 < L) ? fh[d0] : 0.f;
+    w1 = (tid + kThr < 2 * kT - 1 && d1 >= 0 && d1 < L) ? fh[d1] : 0.f;
+    if (d0 == 0) w0 += dh;
+    if (d1 == 0) w1 += dh;
+  };
+  {
+    float w0, w1;
+    weights(0, w0, w1);
+    sm.fs[0][tid] = w0;
+    sm.fs[0][tid + kThr] = w1;
+  }
   issue_k(0);
   issue_v(0, 0);
   cp_async_commit();
@@ -210,12 +225,6 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
     // ---- this tile's K~ and V have been copied (issued during the previous tile);
     // the Toeplitz weights for (t0, s0)
     cp_async_wait_all();
-    for (int idx = tid; idx < 2 * kT - 1; idx += kThr) {
-      const int d = idx - (kT - 1) + (t0 - s0);  // t - s
-      float w = (d >= 0 && d < L) ? fh[d] : 0.f;
-      if (d == 0) w += dh;
-      sm.fs[idx] = w;
-    }
     tc::fence_smem_to_async();
     tc::fence_before_sync();
     __syncthreads();
@@ -240,9 +249,12 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
       break;
     }
     tc::fence_after_sync();
-    // ---- the S-MMA has read K~: the next tile's K~ can come in now
+    // ---- the S-MMA has read K~: the next tile's K~ can come in now, and its weights
     if (st + 1 <= tt) issue_k(s0 + kT);
     cp_async_commit();
+    float wn0 = 0.f, wn1 = 0.f;
+    if (st + 1 <= tt) weights(s0 + kT, wn0, wn1);
+    const float* fsc = sm.fs[st & 1];
     // ---- P = S (.) Toeplitz weights, rounded to the operand type, into the K-major A tile
 #pragma unroll 1
     for (int c = 0; c < kT; c += 16) {
@@ -251,14 +263,18 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
       uint32_t pw[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float a = sv[2 * i] * sm.fs[row - (c + 2 * i) + (kT - 1)];
-        const float bb = sv[2 * i + 1] * sm.fs[row - (c + 2 * i + 1) + (kT - 1)];
+        const float a = sv[2 * i] * fsc[row - (c + 2 * i) + (kT - 1)];
+        const float bb = sv[2 * i + 1] * fsc[row - (c + 2 * i + 1) + (kT - 1)];
         pw[i] = Bits<T>::pack(a, bb);
       }
       *reinterpret_cast<uint4*>(sm.p + (uint32_t)(row >> 3) * kPSbo + (uint32_t)(c >> 3) * kPLbo + (row & 7) * 16) =
           make_uint4(pw[0], pw[1], pw[2], pw[3]);
       *reinterpret_cast<uint4*>(sm.p + (uint32_t)(row >> 3) * kPSbo + (uint32_t)((c + 8) >> 3) * kPLbo + (row & 7) * 16) =
           make_uint4(pw[4], pw[5], pw[6], pw[7]);
+    }
+    if (st + 1 <= tt) {  // the other buffer was last read by the P pass of tile st - 1
+      sm.fs[(st + 1) & 1][tid] = wn0;
+      sm.fs[(st + 1) & 1][tid + kThr] = wn1;
     }
     tc::fence_smem_to_async();
     tc::fence_before_sync();
