@@ -5,18 +5,21 @@
 // q, is exactly the causal Toeplitz-weighted product
 //   o_j[t] = sum_{s<=t} (f_h[t-s] + D_h [s==t]) (q_t . k~_s) v_s[j]
 // (H3 summary appendix D.2 "H3 Complexity": matrix multiplications plus the
-// SSM convolution).  Per 128-row tile of t and each 128-row tile of s <= t:
-//   S  = Q_t K~_s^T            tcgen05.mma, M=128 N=128 K=64, fp32 in TMEM
+// SSM convolution).  Per 128-row tile of t and each 64-row step of s <= t:
+//   S  = Q_t K~_s^T            tcgen05.mma, M=128 N=64 K=64, fp32 in TMEM
 //   P  = S (.) T_f(t-s)        4 warps: tcgen05.ld, scale, round, store to SMEM
-//   O += P V_s                 tcgen05.mma, M=128 N=64 K=128, fp32 in TMEM
+//   O += P V_s                 tcgen05.mma, M=128 N=64 K=64, fp32 in TMEM
 // The shift SSM k~[s,c] = sum_j Cshift[c,j] k[s-j,c] runs once, in a small
 // elementwise kernel, into a workspace (rounded to the operand type).  Q and
 // K~ tiles are K-major with padded core-matrix offsets (LBO 144 bytes) so that
 // the row-wise 16-byte staging copies are free of bank conflicts; V is staged
 // as it lies in memory and read by the tensor cores as an MN-major operand.
-// The next s tile's K~ and V are copied in with cp.async while the current
-// tile is processed (K~ once the S-MMA has read the current one; V into a
-// second buffer).
+// 64-row s steps keep a CTA at 128 TMEM columns and ~55 KB of shared memory,
+// so four CTAs share an SM and hide each other's copy and MMA latency; the
+// next step's K~ is copied in as soon as the S-MMA has read the current one,
+// V once the O-MMA has, and the next step's Toeplitz weights are loaded a step
+// ahead.  CTAs are launched heaviest tile first (a t tile has t / 64 + 2 s
+// steps), so the causal imbalance stays inside the first waves.
 // Every wait on MMA completion is bounded; on a timeout the CTA records it in
 // a device counter, skips its remaining work and still frees its TMEM.
 #include "kernels.cuh"
@@ -28,21 +31,22 @@ static __device__ unsigned int g_mixer_timeouts;
 
 namespace {
 constexpr int kHD = 64;         // head_dim
-constexpr int kT = 128;         // rows per t / s tile
+constexpr int kT = 128;         // rows per t tile
+constexpr int kS = 64;          // rows per s step
 constexpr int kThr = 128;       // 4 warps: one TMEM lane quarter each
 constexpr int kMaxS = 8;        // shift taps
-constexpr uint32_t kTmemCols = 256;  // S: cols [0,128), O: [128,192)
+constexpr uint32_t kTmemCols = 128;  // S: cols [0,64), O: [64,128)
 constexpr uint64_t kWaitNs = 2000000000ull;
 
 constexpr uint32_t kQLbo = 144, kQSbo = (kHD / 8) * 144;   // Q, K~: 128 rows x 64 K, padded
-constexpr uint32_t kVSbo = 144, kVLbo = (kHD / 8) * 144;   // V: MN-major, 64 N (j) x 128 K (s), padded
-constexpr uint32_t kPLbo = 128, kPSbo = (kT / 8) * 128;    // P: 128 rows x 128 K
+constexpr uint32_t kVSbo = 144, kVLbo = (kHD / 8) * 144;   // V: MN-major, 64 N (j) x 64 K (s), padded
+constexpr uint32_t kPLbo = 128, kPSbo = (kS / 8) * 128;    // P: 128 rows x 64 K
 struct MixSmem {
   uint8_t q[(kT / 8) * kQSbo];      // A of S-MMA  (rows t, K = i)
-  uint8_t k[(kT / 8) * kQSbo];      // B of S-MMA  (rows s, K = i)
-  uint8_t v[2][(kT / 8) * kVLbo];   // B of O-MMA  (N = j, K = s), MN-major, double-buffered
-  uint8_t p[kT * kT * 2];           // A of O-MMA  (rows t, K = s)
-  float fs[2][2 * kT];              // Toeplitz weights of the current and the next s tile
+  uint8_t k[(kS / 8) * kQSbo];      // B of S-MMA  (rows s, K = i)
+  uint8_t v[(kS / 8) * kVLbo];      // B of O-MMA  (N = j, K = s), MN-major
+  uint8_t p[kT * kS * 2];           // A of O-MMA  (rows t, K = s)
+  float fs[2][2 * kT];              // Toeplitz weights of the current and the next s step
   uint64_t mbar;
   uint32_t tmem_base;
 };
@@ -136,14 +140,19 @@ __global__ void __launch_bounds__(256) shift_ssm_kernel(const T* __restrict__ k,
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restrict__ q, const T* __restrict__ kt,
+__global__ void __launch_bounds__(kThr, 4) h3_mixer_tc_kernel(const T* __restrict__ q, const T* __restrict__ kt,
                                                               const T* __restrict__ v,
                                                               const float* __restrict__ fdiag,
                                                               const float* __restrict__ D, T* __restrict__ o, int L,
-                                                              int heads) {
+                                                              int heads, int B) {
   extern __shared__ __align__(1024) uint8_t smraw[];
   MixSmem& sm = *reinterpret_cast<MixSmem*>(smraw);
-  const int tt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // heaviest t tiles first: CTA i takes tile nt - 1 - i / (heads B), then (head, b)
+  const int nt = (L + kT - 1) / kT;
+  const int hb = heads * B;
+  const int tt = nt - 1 - (int)(blockIdx.x / hb);
+  const int rem = (int)(blockIdx.x % hb);
+  const int h = rem % heads, b = rem / heads;
   const int tid = threadIdx.x, warp = tid >> 5;
   const int dm = heads * kHD;
   const int t0 = tt * kT;
@@ -169,19 +178,19 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = sm.tmem_base;
-  const uint32_t tS = tmem, tO = tmem + 128;
+  const uint32_t tS = tmem, tO = tmem + kS;
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  const uint32_t idS = tc::idesc_f16(128, 128, Bits<T>::bf16);
+  const uint32_t idS = tc::idesc_f16(128, kS, Bits<T>::bf16);
   const uint32_t idO = tc::idesc_f16(128, kHD, Bits<T>::bf16, 0, 1);
   const float dh = D[h];
   const float* fh = fdiag + (size_t)h * L;
   uint32_t phase = 0;
   bool failed = false;
   const int row = tid;  // TMEM lane / tile row owned by this thread
-  // K~ / V tile of rows s0 .. s0+127 -> shared memory with cp.async (rows past L zeroed)
+  // K~ / V rows s0 .. s0+63 -> shared memory with cp.async (rows past L zeroed)
   auto issue_k = [&](int s0) {
     const uint32_t ka = tc::smem_u32(sm.k);
-    for (int idx = tid; idx < kT * (kHD / 8); idx += kThr) {
+    for (int idx = tid; idx < kS * (kHD / 8); idx += kThr) {
       const int r = idx >> 3, c8 = (idx & 7) * 8;
       const int s = s0 + r;
       if (s < L)
@@ -190,23 +199,23 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
         *reinterpret_cast<uint4*>(sm.k + qoff(r, c8)) = make_uint4(0, 0, 0, 0);
     }
   };
-  auto issue_v = [&](int s0, int buf) {
-    const uint32_t va = tc::smem_u32(sm.v[buf]);
-    for (int idx = tid; idx < kT * (kHD / 8); idx += kThr) {
+  auto issue_v = [&](int s0) {
+    const uint32_t va = tc::smem_u32(sm.v);
+    for (int idx = tid; idx < kS * (kHD / 8); idx += kThr) {
       const int r = idx >> 3, c8 = (idx & 7) * 8;
       const int s = s0 + r;
       if (s < L)
         cp_async16(va + voff(r, c8), vb + (size_t)s * dm + c8);
       else
-        *reinterpret_cast<uint4*>(sm.v[buf] + voff(r, c8)) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(sm.v + voff(r, c8)) = make_uint4(0, 0, 0, 0);
     }
   };
-  // Toeplitz weights f[t - s] (+ D on the diagonal) of tile (t0, s0) for idx = t - s + 127 - (t0 - s0):
-  // this thread's two entries, loaded from global memory a tile ahead and stored after the P pass
+  // Toeplitz weights f[t - s] (+ D on the diagonal) of step (t0, s0) at idx = t - s + 63 - (t0 - s0)
+  // (t - s in [t0 - s0 - 63, t0 - s0 + 127]): this thread's two entries, loaded a step ahead
   auto weights = [&](int s0, float& w0, float& w1) {
-    const int d0 = tid - (kT - 1) + (t0 - s0), d1 = d0 + kThr;
+    const int d0 = tid - (kS - 1) + (t0 - s0), d1 = d0 + kThr;
     w0 = (d0 >= 0 && d0 < L) ? fh[d0] : 0.f;
-    w1 = (tid + kThr < 2 * kT - 1 && d1 >= 0 && d1 < L) ? fh[d1] : 0.f;
+    w1 = (tid + kThr < kT + kS - 1 && d1 >= 0 && d1 < L) ? fh[d1] : 0.f;
     if (d0 == 0) w0 += dh;
     if (d1 == 0) w1 += dh;
   };
@@ -217,22 +226,18 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
     sm.fs[0][tid + kThr] = w1;
   }
   issue_k(0);
-  issue_v(0, 0);
+  issue_v(0);
   cp_async_commit();
 
-  for (int st = 0; st <= tt && !failed; ++st) {
-    const int s0 = st * kT;
-    // ---- this tile's K~ and V have been copied (issued during the previous tile);
-    // the Toeplitz weights for (t0, s0)
+  const int nsteps = min((t0 + kT + kS - 1) / kS, (L + kS - 1) / kS);  // s0 = kS st <= t0 + 127, s0 < L
+  for (int st = 0; st < nsteps && !failed; ++st) {
+    const int s0 = st * kS;
+    // ---- this step's K~ and V have been copied (issued during the previous step)
     cp_async_wait_all();
     tc::fence_smem_to_async();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    // ---- the next tile's V goes to the other buffer (its last reader, the O-MMA of
-    // tile st - 1, has completed)
-    if (st + 1 <= tt) issue_v(s0 + kT, (st + 1) & 1);
-    cp_async_commit();
     // ---- S = Q K~^T
     if (tid == 0) {
       const uint32_t qa = tc::smem_u32(sm.q), ka = tc::smem_u32(sm.k);
@@ -249,22 +254,23 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
       break;
     }
     tc::fence_after_sync();
-    // ---- the S-MMA has read K~: the next tile's K~ can come in now, and its weights
-    if (st + 1 <= tt) issue_k(s0 + kT);
+    // ---- the S-MMA has read K~: the next step's K~ can come in now, and its weights
+    const bool more = st + 1 < nsteps;
+    if (more) issue_k(s0 + kS);
     cp_async_commit();
     float wn0 = 0.f, wn1 = 0.f;
-    if (st + 1 <= tt) weights(s0 + kT, wn0, wn1);
+    if (more) weights(s0 + kS, wn0, wn1);
     const float* fsc = sm.fs[st & 1];
     // ---- P = S (.) Toeplitz weights, rounded to the operand type, into the K-major A tile
 #pragma unroll 1
-    for (int c = 0; c < kT; c += 16) {
+    for (int c = 0; c < kS; c += 16) {
       float sv[16];
       tc::tmem_ld16_wait(tS + lane_off + (uint32_t)c, sv);
       uint32_t pw[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float a = sv[2 * i] * fsc[row - (c + 2 * i) + (kT - 1)];
-        const float bb = sv[2 * i + 1] * fsc[row - (c + 2 * i + 1) + (kT - 1)];
+        const float a = sv[2 * i] * fsc[row - (c + 2 * i) + (kS - 1)];
+        const float bb = sv[2 * i + 1] * fsc[row - (c + 2 * i + 1) + (kS - 1)];
         pw[i] = Bits<T>::pack(a, bb);
       }
       *reinterpret_cast<uint4*>(sm.p + (uint32_t)(row >> 3) * kPSbo + (uint32_t)(c >> 3) * kPLbo + (row & 7) * 16) =
@@ -272,7 +278,7 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
       *reinterpret_cast<uint4*>(sm.p + (uint32_t)(row >> 3) * kPSbo + (uint32_t)((c + 8) >> 3) * kPLbo + (row & 7) * 16) =
           make_uint4(pw[4], pw[5], pw[6], pw[7]);
     }
-    if (st + 1 <= tt) {  // the other buffer was last read by the P pass of tile st - 1
+    if (more) {  // the other buffer was last read by the P pass of step st - 1
       sm.fs[(st + 1) & 1][tid] = wn0;
       sm.fs[(st + 1) & 1][tid + kThr] = wn1;
     }
@@ -282,9 +288,9 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
     tc::fence_after_sync();
     // ---- O += P V
     if (tid == 0) {
-      const uint32_t pa = tc::smem_u32(sm.p), va = tc::smem_u32(sm.v[st & 1]);
+      const uint32_t pa = tc::smem_u32(sm.p), va = tc::smem_u32(sm.v);
 #pragma unroll
-      for (int kk = 0; kk < kT / 16; ++kk)
+      for (int kk = 0; kk < kS / 16; ++kk)
         tc::mma_f16(tO, tc::desc_kmajor(pa + kk * 2 * kPLbo, kPLbo, kPSbo),
                     tc::desc_kmajor(va + kk * 2 * kVLbo, kVLbo, kVSbo), idO, (st > 0 || kk > 0) ? 1u : 0u);
       tc::mma_commit(&sm.mbar);
@@ -296,6 +302,9 @@ __global__ void __launch_bounds__(kThr, 1) h3_mixer_tc_kernel(const T* __restric
       break;
     }
     tc::fence_after_sync();
+    // ---- the O-MMA has read V: the next step's V
+    if (more) issue_v(s0 + kS);
+    cp_async_commit();
   }
   cp_async_wait_all();
   if (!failed) {
@@ -352,8 +361,9 @@ static cudaError_t mixer_tc_t(const void* q, const void* k, const void* v, const
   auto kern = h3_mixer_tc_kernel<T>;
   e = smem_optin<h3_mixer_tc_kernel<T>>(smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((L + kT - 1) / kT, heads, B);
-  kern<<<grid, kThr, smem, st>>>((const T*)q, (const T*)kt, (const T*)v, f, D, (T*)o, L, heads);
+  const long long ctas = (long long)((L + kT - 1) / kT) * heads * B;
+  if (ctas > 0x7fffffffLL) return cudaErrorInvalidValue;
+  kern<<<(unsigned)ctas, kThr, smem, st>>>((const T*)q, (const T*)kt, (const T*)v, f, D, (T*)o, L, heads, B);
   return cudaGetLastError();
 }
 
