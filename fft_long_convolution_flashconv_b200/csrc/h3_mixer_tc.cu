@@ -59,6 +59,8 @@ __device__ __forceinline__ void cp_async16(uint32_t saddr, const void* g) {
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+// all but the most recently committed group of this thread's copies have landed
+__device__ __forceinline__ void cp_async_wait_but_last() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ uint32_t voff(int s, int j8) {  // 8 consecutive j at time s
   return (uint32_t)(j8 >> 3) * kVSbo + (uint32_t)(s >> 3) * kVLbo + (uint32_t)(s & 7) * 16;
 }
@@ -226,14 +228,16 @@ __global__ void __launch_bounds__(kThr, 4) h3_mixer_tc_kernel(const T* __restric
     sm.fs[0][tid + kThr] = w1;
   }
   issue_k(0);
+  cp_async_commit();
   issue_v(0);
   cp_async_commit();
 
   const int nsteps = min((t0 + kT + kS - 1) / kS, (L + kS - 1) / kS);  // s0 = kS st <= t0 + 127, s0 < L
   for (int st = 0; st < nsteps && !failed; ++st) {
     const int s0 = st * kS;
-    // ---- this step's K~ and V have been copied (issued during the previous step)
-    cp_async_wait_all();
+    // ---- this step's K~ has been copied (issued during the previous step; its V, committed
+    // after it, may still be in flight and is waited for before the O-MMA)
+    cp_async_wait_but_last();
     tc::fence_smem_to_async();
     tc::fence_before_sync();
     __syncthreads();
@@ -282,6 +286,7 @@ __global__ void __launch_bounds__(kThr, 4) h3_mixer_tc_kernel(const T* __restric
       sm.fs[(st + 1) & 1][tid] = wn0;
       sm.fs[(st + 1) & 1][tid + kThr] = wn1;
     }
+    cp_async_wait_but_last();  // this step's V (only the next step's K~ may still be in flight)
     tc::fence_smem_to_async();
     tc::fence_before_sync();
     __syncthreads();
