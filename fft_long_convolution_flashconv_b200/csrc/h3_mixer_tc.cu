@@ -266,21 +266,26 @@ __global__ void __launch_bounds__(kThr, 4) h3_mixer_tc_kernel(const T* __restric
     if (more) weights(s0 + kS, wn0, wn1);
     const float* fsc = sm.fs[st & 1];
     // ---- P = S (.) Toeplitz weights, rounded to the operand type, into the K-major A tile
-#pragma unroll 1
-    for (int c = 0; c < kS; c += 16) {
-      float sv[16];
-      tc::tmem_ld16_wait(tS + lane_off + (uint32_t)c, sv);
+#pragma unroll
+    for (int c = 0; c < kS; c += 32) {
+      float sv2[32];
+      tc::tmem_ld16x2_wait(tS + lane_off + (uint32_t)c, tS + lane_off + (uint32_t)c + 16u, sv2, sv2 + 16);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+      const float* sv = sv2 + 16 * hh;
+      const int c16 = c + 16 * hh;
       uint32_t pw[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float a = sv[2 * i] * fsc[row - (c + 2 * i) + (kS - 1)];
-        const float bb = sv[2 * i + 1] * fsc[row - (c + 2 * i + 1) + (kS - 1)];
+        const float a = sv[2 * i] * fsc[row - (c16 + 2 * i) + (kS - 1)];
+        const float bb = sv[2 * i + 1] * fsc[row - (c16 + 2 * i + 1) + (kS - 1)];
         pw[i] = Bits<T>::pack(a, bb);
       }
-      *reinterpret_cast<uint4*>(sm.p + (uint32_t)(row >> 3) * kPSbo + (uint32_t)(c >> 3) * kPLbo + (row & 7) * 16) =
+      *reinterpret_cast<uint4*>(sm.p + (uint32_t)(row >> 3) * kPSbo + (uint32_t)(c16 >> 3) * kPLbo + (row & 7) * 16) =
           make_uint4(pw[0], pw[1], pw[2], pw[3]);
-      *reinterpret_cast<uint4*>(sm.p + (uint32_t)(row >> 3) * kPSbo + (uint32_t)((c + 8) >> 3) * kPLbo + (row & 7) * 16) =
-          make_uint4(pw[4], pw[5], pw[6], pw[7]);
+      *reinterpret_cast<uint4*>(sm.p + (uint32_t)(row >> 3) * kPSbo + (uint32_t)((c16 + 8) >> 3) * kPLbo +
+                                (row & 7) * 16) = make_uint4(pw[4], pw[5], pw[6], pw[7]);
+      }
     }
     if (more) {  // the other buffer was last read by the P pass of step st - 1
       sm.fs[(st + 1) & 1][tid] = wn0;
