@@ -39,6 +39,8 @@
 // every pass: warp w serves TMEM lane quarter w % 4 and the column group
 // w / 4.  Waits on MMA completion are bounded; a CTA that gives up counts it
 // in a device word, skips its remaining work and frees its TMEM.
+#include <cuda.h>
+
 #include "fft_stockham.cuh"
 #include "kernels.cuh"
 #include "tc100.cuh"
@@ -68,7 +70,7 @@ struct LG {
   static constexpr uint32_t tcols = 4 * N2;         // TMEM: work [0, 2 N2) | filter [2 N2, 4 N2)
   static constexpr uint32_t o_ca = 0, o_cb = kCBytes, o_gf = 2 * kCBytes, o_gi = o_gf + R * 2048,
                             o_x = o_gi + R * 2048, o_yv = o_x + 2 * xplane, o_fst = o_yv + yv,
-                            o_mbar = o_fst + 4 * Lc, o_tmem = o_mbar + 8,
+                            o_mbar = o_fst + 4 * Lc, o_tmem = o_mbar + 16,  // MMA and row-copy barriers
                             bytes = o_tmem + 8;
   static_assert(256u * N2 * 2 == yv, "Z must fit the stage-B tiles");
 };
@@ -127,17 +129,18 @@ __device__ __forceinline__ float2 f2(uint32_t re, uint32_t im) { return make_flo
 template <typename T, int R>
 __global__ void __launch_bounds__(kThrL, 1)
     fftconv_tcl_kernel(const T* __restrict__ u, const float* __restrict__ f, int fstride, const float* __restrict__ D,
-                       T* __restrict__ y, int B, int H, long long Lrow, int C, int conj_filter) {
+                       T* __restrict__ y, int B, int H, long long Lrow, int C, int conj_filter,
+                       const __grid_constant__ CUtensorMap umap) {
   using G = LG<R>;
   constexpr int N2 = G::N2, Lc = G::Lc, M = G::M;
   extern __shared__ __align__(1024) uint8_t sm[];
   uint64_t* mbar = reinterpret_cast<uint64_t*>(sm + G::o_mbar);
+  uint64_t* mbar_ld = mbar + 1;  // a pair's rows landed in the X planes (tensor-map copies)
   uint32_t* tmem_p = reinterpret_cast<uint32_t*>(sm + G::o_tmem);
   const int tid = threadIdx.x, warp = tid >> 5;
   const int row = tid & 127;  // TMEM lane: k1 in the passes, output lane j in the epilogue
   const int set = warp >> 2;  // column group 0..3
   const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-  const uint16_t* ub = reinterpret_cast<const uint16_t*>(u);
   uint16_t* yb = reinterpret_cast<uint16_t*>(y);
   const uint32_t s_base = tc::smem_u32(sm);
   const uint32_t ca = s_base + G::o_ca, cb = s_base + G::o_cb, gf = s_base + G::o_gf, gi = s_base + G::o_gi;
@@ -146,6 +149,7 @@ __global__ void __launch_bounds__(kThrL, 1)
   if (warp == 0) tc::tmem_alloc(tmem_p, G::tcols);
   if (tid == 0) {
     tc::mbar_init(mbar, 1);
+    tc::mbar_init(mbar_ld, 1);
     tc::fence_mbar_init();
   }
   // constant blocks (tables built with the library, already in the operand layouts): CA, CB in the
@@ -190,22 +194,24 @@ __global__ void __launch_bounds__(kThrL, 1)
   auto row_off = [&](int h, int q) -> size_t {
     return ((size_t)(q / C) * H + h) * (size_t)Lrow + (size_t)(q % C) * Lc;
   };
-  // cp.async of a pair's rows into the X planes (missing second row: zeros)
+  // a pair's rows into the X planes: one tensor-map copy per row (thread 0), each box
+  // (8 n2, 8 n1 % 8, N2 / 8 column groups, 8 n1 / 8) landing in the operand layout; a
+  // missing second row lies past the last row of the map and arrives as zeros
+  uint32_t ph_ld = 0;
+  bool ld_pend = false;  // a pair's copies are in flight
   auto issue_pair = [&](long long it) {
-    const int h = (int)(it / NP), p = (int)(it - (long long)h * NP);
-    const int q0 = 2 * p, q1 = 2 * p + 1;
-    const uint16_t* r0 = ub + row_off(h, q0);
-    const uint16_t* r1 = q1 < Q ? ub + row_off(h, q1) : nullptr;
-    for (int idx = tid; idx < 64 * (N2 / 8); idx += kThrL) {
-      const int n1 = idx / (N2 / 8), c8 = idx - n1 * (N2 / 8);
-      const uint32_t off = (uint32_t)c8 * 128 + (uint32_t)(n1 >> 3) * G::lboX + (uint32_t)(n1 & 7) * 16;
-      const int t = n1 * N2 + c8 * 8;
-      cp_async16(xr + off, r0 + t);
-      if (r1)
-        cp_async16(xi + off, r1 + t);
-      else
-        *reinterpret_cast<uint4*>(sm + G::o_x + G::xplane + off) = make_uint4(0, 0, 0, 0);
+    if (tid == 0) {
+      const int h = (int)(it / NP), p = (int)(it - (long long)h * NP);
+      const int q0 = 2 * p, q1 = 2 * p + 1;
+      tc::mbar_expect_tx(mbar_ld, 2u * G::xplane);
+      tc::tma_load_5d(xr, &umap, 0, 0, 0, 8 * (q0 % C), (q0 / C) * H + h, mbar_ld);
+      tc::tma_load_5d(xi, &umap, 0, 0, 0, 8 * (q1 % C), (q1 / C) * H + h, mbar_ld);
     }
+  };
+  auto wait_pair = [&]() -> bool {  // all threads; bounded
+    const bool ok = tc::mbar_wait_bounded(mbar_ld, ph_ld, kWaitNsL);
+    ph_ld ^= 1u;
+    return ok;
   };
   auto issue_filter = [&](int h) {
     const float* fr = f + (size_t)h * fstride;
@@ -334,7 +340,7 @@ __global__ void __launch_bounds__(kThrL, 1)
       }
       if (!mma_wait()) { failed = true; break; }
       issue_pair(it);  // the X planes are free again
-      cp_async_commit();
+      ld_pend = true;
       pass1(tw);
       smem_to_mma();
       if (tid == 0) {
@@ -343,12 +349,10 @@ __global__ void __launch_bounds__(kThrL, 1)
       }
       if (!mma_wait()) { failed = true; break; }
       hcur = h;
-    } else if (it == it0) {
-      issue_pair(it);
-      cp_async_commit();
     }
-    // ---- the pair: stage A
-    cp_async_wait_all();
+    // ---- the pair: stage A (its rows were copied in during the previous item, or above)
+    if (__syncthreads_or(!wait_pair())) { failed = true; break; }
+    ld_pend = false;
     smem_to_mma();
     if (tid == 0) {
       issue_stage_a(tw, true);
@@ -358,8 +362,12 @@ __global__ void __launch_bounds__(kThrL, 1)
     // the X planes (and the filter staging) are free: prefetch the next item
     if (it + 1 < it1) {
       const int hn = (int)((it + 1) / NP);
-      if (hn == h) issue_pair(it + 1);
-      else issue_filter(hn);
+      if (hn == h) {
+        issue_pair(it + 1);
+        ld_pend = true;
+      } else {
+        issue_filter(hn);
+      }
     }
     cp_async_commit();
     pass1(tw);
@@ -457,34 +465,73 @@ __global__ void __launch_bounds__(kThrL, 1)
       if (q < Q) {
         uint16_t* yr = yb + row_off(h, q) + (size_t)n1 * N2;
         constexpr int CPS = N2 / 4;  // columns per warp group
+        uint32_t v[CPS / 8][8];
+#pragma unroll
+        for (int c8 = 0; c8 < CPS / 8; ++c8) tc::tmem_ld8(tw + lane_off + (uint32_t)(set * CPS + c8 * 8), v[c8]);
+        tc::tmem_wait_ld();  // one wait for all of this thread's columns
 #pragma unroll
         for (int c8 = 0; c8 < CPS / 8; ++c8) {
-          uint32_t v[8];
-          const int col = set * CPS + c8 * 8;
-          tc::tmem_ld8(tw + lane_off + (uint32_t)col, v);
-          tc::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 8; ++e) tc::tmem_regs_ready(v[e]);
-          *reinterpret_cast<uint4*>(yr + col) =
-              make_uint4(OpL<T>::pack(__uint_as_float(v[0]), __uint_as_float(v[1])),
-                         OpL<T>::pack(__uint_as_float(v[2]), __uint_as_float(v[3])),
-                         OpL<T>::pack(__uint_as_float(v[4]), __uint_as_float(v[5])),
-                         OpL<T>::pack(__uint_as_float(v[6]), __uint_as_float(v[7])));
+          for (int e = 0; e < 8; ++e) tc::tmem_regs_ready(v[c8][e]);
+          *reinterpret_cast<uint4*>(yr + set * CPS + c8 * 8) =
+              make_uint4(OpL<T>::pack(__uint_as_float(v[c8][0]), __uint_as_float(v[c8][1])),
+                         OpL<T>::pack(__uint_as_float(v[c8][2]), __uint_as_float(v[c8][3])),
+                         OpL<T>::pack(__uint_as_float(v[c8][4]), __uint_as_float(v[c8][5])),
+                         OpL<T>::pack(__uint_as_float(v[c8][6]), __uint_as_float(v[c8][7])));
         }
       }
     }
     tc::fence_before_sync();  // the epilogue's TMEM reads precede the next item's MMAs
   }
   cp_async_wait_all();
+  if (ld_pend) (void)tc::mbar_wait_bounded(mbar_ld, ph_ld, kWaitNsL);  // copies in flight land first
   if (failed && tid == 0) atomicAdd(&g_fftconv_tcl_timeouts, 1u);
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 0) tc::tmem_dealloc(tmem, G::tcols);
 }
 
+typedef CUresult (*TensorMapEncodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                         const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                         CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static TensorMapEncodeTiled encode_fn() {
+  static TensorMapEncodeTiled fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<TensorMapEncodeTiled>(p);
+  }();
+  return fn;
+}
+
+// Rows of u as 5-d boxes that land in the stage-A operand layout: element
+// (e, r, c8, a, row) is u[row * Lrow + (8 a + r) * N2 + 8 c8 + e] (n1 = 8 a + r,
+// chunk c = a / 8 of a row of C chunks), box (8, 8, N2 / 8, 8, 1) = one chunk's
+// 64 non-zero n1 rows.
+template <int R>
+static cudaError_t make_row_map(CUtensorMap* m, const void* u, int B, int H, long long Lrow, int C) {
+  constexpr int N2 = LG<R>::N2;
+  TensorMapEncodeTiled enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t dims[5] = {8, 8, (cuuint64_t)(N2 / 8), (cuuint64_t)(8 * C), (cuuint64_t)B * (cuuint64_t)H};
+  const cuuint64_t strides[4] = {(cuuint64_t)(2 * N2), 16, (cuuint64_t)(16 * N2), (cuuint64_t)(2 * Lrow)};
+  const cuuint32_t box[5] = {8, 8, (cuuint32_t)(N2 / 8), 8, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 5, const_cast<void*>(u), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <typename T, int R>
 static cudaError_t tcl_t(const void* u, const float* f, int fstride, const float* D, void* y, int B, int H,
                          long long Lrow, int C, bool pdl, int conj_filter, cudaStream_t st) {
+  CUtensorMap umap;
+  cudaError_t e0 = make_row_map<R>(&umap, u, B, H, Lrow, C);
+  if (e0 != cudaSuccess) return e0;
   const size_t smem = LG<R>::bytes;
   cudaError_t e = smem_optin<fftconv_tcl_kernel<T, R>>(smem);
   if (e != cudaSuccess) return e;
@@ -501,7 +548,7 @@ static cudaError_t tcl_t(const void* u, const float* f, int fstride, const float
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, fftconv_tcl_kernel<T, R>, (const T*)u, f, fstride, D, (T*)y, B, H, Lrow, C,
-                            conj_filter);
+                            conj_filter, umap);
 }
 
 bool fftconv_tcl_supported(int Lc, int dtype) { return (dtype == 1 || dtype == 2) && (Lc == 2048 || Lc == 4096 || Lc == 8192); }
