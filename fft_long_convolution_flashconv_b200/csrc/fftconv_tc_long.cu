@@ -34,16 +34,16 @@
 // imaginary outputs are the two convolutions).  When the channel changes,
 // the filter (with D added to its tap 0) goes through stages A and B into a
 // TMEM region that every pair of the channel then reads in pass 2.  The next
-// pair's rows (or the next channel's filter) are copied in with cp.async as
+// pair's rows (or the next channel's filter) are copied in (the rows by two
+// tensor-map copies from one thread, the filter with cp.async) as
 // soon as stage A has released the input buffer.  All 16 warps take part in
 // every pass: warp w serves TMEM lane quarter w % 4 and the column group
 // w / 4.  Waits on MMA completion are bounded; a CTA that gives up counts it
 // in a device word, skips its remaining work and frees its TMEM.
-#include <cuda.h>
-
 #include "fft_stockham.cuh"
 #include "kernels.cuh"
 #include "tc100.cuh"
+#include "tmap.cuh"
 
 #define FC_TABLES_DFT128
 #define FC_TABLES_LONG
@@ -491,39 +491,13 @@ __global__ void __launch_bounds__(kThrL, 1)
   if (warp == 0) tc::tmem_dealloc(tmem, G::tcols);
 }
 
-typedef CUresult (*TensorMapEncodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                         const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                         CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static TensorMapEncodeTiled encode_fn() {
-  static TensorMapEncodeTiled fn = [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      p = nullptr;
-    return reinterpret_cast<TensorMapEncodeTiled>(p);
-  }();
-  return fn;
-}
-
-// Rows of u as 5-d boxes that land in the stage-A operand layout: element
-// (e, r, c8, a, row) is u[row * Lrow + (8 a + r) * N2 + 8 c8 + e] (n1 = 8 a + r,
-// chunk c = a / 8 of a row of C chunks), box (8, 8, N2 / 8, 8, 1) = one chunk's
-// 64 non-zero n1 rows.
 template <int R>
 static cudaError_t make_row_map(CUtensorMap* m, const void* u, int B, int H, long long Lrow, int C) {
   constexpr int N2 = LG<R>::N2;
-  TensorMapEncodeTiled enc = encode_fn();
-  if (!enc) return cudaErrorNotSupported;
   const cuuint64_t dims[5] = {8, 8, (cuuint64_t)(N2 / 8), (cuuint64_t)(8 * C), (cuuint64_t)B * (cuuint64_t)H};
   const cuuint64_t strides[4] = {(cuuint64_t)(2 * N2), 16, (cuuint64_t)(16 * N2), (cuuint64_t)(2 * Lrow)};
   const cuuint32_t box[5] = {8, 8, (cuuint32_t)(N2 / 8), 8, 1};
-  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 5, const_cast<void*>(u), dims, strides, box, estr,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+  return encode_map_5d_u16(m, u, dims, strides, box);
 }
 
 template <typename T, int R>

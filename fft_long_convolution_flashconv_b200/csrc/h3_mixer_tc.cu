@@ -22,8 +22,11 @@
 // steps), so the causal imbalance stays inside the first waves.
 // Every wait on MMA completion is bounded; on a timeout the CTA records it in
 // a device counter, skips its remaining work and still frees its TMEM.
+#include <algorithm>
+
 #include "kernels.cuh"
 #include "tc100.cuh"
+#include "tmap.cuh"
 
 namespace fc {
 
@@ -346,6 +349,352 @@ __global__ void __launch_bounds__(kThr, 4) h3_mixer_tc_kernel(const T* __restric
   if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
+// ---------------------------------------------------------------------------
+// Warp-specialised persistent form (L a multiple of 8).  One CTA per SM walks
+// a list of (t tile, head, b) items, heaviest tiles first and dealt to the
+// CTAs in snake order so the causal work evens out.  Per item, 128-row s
+// steps s0 = 0, 128, ..., t0; the roles hand over through mbarriers:
+//   warp 0      copies K~ and V tiles of each step (two 5-d tensor-map copies
+//               straight into the operand layouts) into a 4-stage ring;
+//   warp 1      issues S = Q K~^T (M=128 N=128 K=64, Q from tensor memory)
+//               into one of two S buffers, then O += P V (M=128 N=64 K=128, P
+//               from tensor memory) of the previous step, so the weighting of
+//               step g overlaps the O-MMA of step g - 1;
+//   warps 4-7 / 8-11  weight the S tiles of even / odd steps: P = S (.) f[t-s]
+//               (+ D on the diagonal), rounded to the operand type and
+//               written back over the same tensor-memory columns;
+//   warps 12-15 put each item's Q tile into tensor memory and write its O.
+// Tensor memory: S/P [0,128) and [128,256), O [256,320) and [320,384),
+// Q [384,416) and [416,448).  Every wait is bounded; a role that gives up
+// raises a shared flag the others see in their own waits, and the CTA lets
+// its copies and MMAs in flight finish before freeing tensor memory.
+namespace {
+constexpr int kWsS = 128;                   // rows per s step
+constexpr int kWsStages = 4;                // K~ / V ring depth
+constexpr int kWsThr = 512;
+constexpr uint32_t kWsTile = 128 * kHD * 2;  // one 128 x 64 16-bit tile
+constexpr int kWinStride = 264;             // floats between the four shifted window copies
+constexpr uint32_t kColO = 256, kColQ = 384, kWsCols = 512;
+
+struct WsSmem {
+  uint8_t k[kWsStages][kWsTile];
+  uint8_t v[kWsStages][kWsTile];
+  float win[2][2][4 * kWinStride];          // [weighting group][buffer]: window copies shifted by 0..3
+  uint64_t k_full[kWsStages], v_full[kWsStages], kv_empty[kWsStages];
+  uint64_t s_full[2], p_full[2], q_full[2], o_full[2], o_empty[2], drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// The items of one CTA in order, and the 128-row s steps of each.
+struct WsIter {
+  int G, cta, nitems, nt, hb, heads;
+  int r, n, k, j, nst, g;  // round, ordinal of the item in this CTA, item, step, steps of the item, global step
+  int tt, h, b;
+  __device__ void set_item() {
+    k = r * G + ((r & 1) ? (G - 1 - cta) : cta);
+    if (k < nitems) {
+      tt = nt - 1 - k / hb;
+      const int rem = k - (k / hb) * hb;
+      h = rem % heads;
+      b = rem / heads;
+      nst = tt + 1;
+    }
+  }
+  __device__ void init(int G_, int cta_, int nitems_, int nt_, int heads_, int B) {
+    G = G_, cta = cta_, nitems = nitems_, nt = nt_, heads = heads_, hb = heads_ * B;
+    r = 0, n = 0, j = 0, g = 0;
+    set_item();
+  }
+  __device__ bool valid() const { return k < nitems; }
+  __device__ void next() {
+    ++g;
+    if (++j == nst) {
+      j = 0;
+      ++n;
+      ++r;
+      set_item();
+    }
+  }
+  __device__ void next_item() {
+    g += nst - j;
+    j = 0;
+    ++n;
+    ++r;
+    set_item();
+  }
+};
+
+__device__ __forceinline__ void nbar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// Named barrier over `count` threads that also ORs a predicate across them.
+__device__ __forceinline__ bool nbar_or(int id, int count, bool v) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(out)
+      : "r"((uint32_t)v), "r"(id), "r"(count)
+      : "memory");
+  return out != 0;
+}
+}  // namespace
+
+template <typename T>
+__global__ void __launch_bounds__(kWsThr, 1)
+    h3_mixer_ws_kernel(const T* __restrict__ q, const float* __restrict__ fdiag, const float* __restrict__ D,
+                       T* __restrict__ o, int L, int heads, int B, const __grid_constant__ CUtensorMap kmap,
+                       const __grid_constant__ CUtensorMap vmap) {
+  extern __shared__ __align__(1024) uint8_t smraw[];
+  WsSmem& sm = *reinterpret_cast<WsSmem*>(smraw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int dm = heads * kHD;
+  const int nt = (L + kT - 1) / kT;
+  const int nitems = nt * heads * B;
+  volatile int* abort_flag = &sm.abort;
+
+  if (tid == 0) {
+    for (int i = 0; i < kWsStages; ++i) {
+      tc::mbar_init(&sm.k_full[i], 1);
+      tc::mbar_init(&sm.v_full[i], 1);
+      tc::mbar_init(&sm.kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&sm.s_full[i], 1);
+      tc::mbar_init(&sm.p_full[i], 128);
+      tc::mbar_init(&sm.q_full[i], 128);
+      tc::mbar_init(&sm.o_full[i], 1);
+      tc::mbar_init(&sm.o_empty[i], 128);
+    }
+    tc::mbar_init(&sm.drain, 1);
+    sm.abort = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) tc::tmem_alloc(&sm.tmem_base, kWsCols);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = sm.tmem_base;
+
+  // bounded wait that also gives up as soon as another role has given up
+  auto wwait = [&](uint64_t* mb, uint32_t parity) -> bool {
+    if (tc::mbar_try_wait(mb, parity)) return true;
+    const uint64_t t0 = tc::globaltimer_ns();
+    while (!tc::mbar_try_wait(mb, parity)) {
+      if (*abort_flag) return false;
+      if (tc::globaltimer_ns() - t0 > kWaitNs) {
+        *abort_flag = 1;
+        return false;
+      }
+    }
+    return true;
+  };
+  WsIter it;
+  it.init((int)gridDim.x, (int)blockIdx.x, nitems, nt, heads, B);
+
+  if (warp == 0) {
+    // ---------------- K~ / V copies
+    for (; it.valid(); it.next()) {
+      const int stg = it.g % kWsStages;
+      const uint32_t use = (uint32_t)(it.g / kWsStages);
+      bool ok = true;
+      if (lane == 0 && use > 0) ok = wwait(&sm.kv_empty[stg], (use - 1) & 1u);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      if (lane == 0) {
+        const int r8 = (it.j * kWsS) / 8;
+        tc::mbar_expect_tx(&sm.k_full[stg], kWsTile);
+        tc::tma_load_5d(tc::smem_u32(sm.k[stg]), &kmap, 0, 0, 8 * it.h, r8, it.b, &sm.k_full[stg]);
+        tc::mbar_expect_tx(&sm.v_full[stg], kWsTile);
+        tc::tma_load_5d(tc::smem_u32(sm.v[stg]), &vmap, 0, 0, 8 * it.h, r8, it.b, &sm.v_full[stg]);
+      }
+    }
+    // copies still in flight (only after a give-up) land before the CTA leaves
+    if (lane == 0) {
+      for (int g = it.g - kWsStages; g < it.g; ++g) {
+        if (g < 0) continue;
+        const int stg = g % kWsStages;
+        const uint32_t par = (uint32_t)(g / kWsStages) & 1u;
+        (void)tc::mbar_wait_bounded(&sm.k_full[stg], par, kWaitNs);
+        (void)tc::mbar_wait_bounded(&sm.v_full[stg], par, kWaitNs);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issue (lane 0)
+    const uint32_t idS = tc::idesc_f16(128, kWsS, Bits<T>::bf16);
+    const uint32_t idO = tc::idesc_f16(128, kHD, Bits<T>::bf16, 0, 1);
+    int pg = -1, pstg = 0, pn = 0, pj = 0, plast = 0;  // the step whose O-MMA is still to be issued
+    auto issue_o = [&]() -> bool {
+      bool ok = true;
+      if (lane == 0) {
+        if (pj == 0 && pn >= 2) ok = wwait(&sm.o_empty[pn & 1], (uint32_t)((pn - 2) >> 1) & 1u);
+        if (ok) ok = wwait(&sm.p_full[pg & 1], (uint32_t)(pg >> 1) & 1u);
+        if (ok) ok = wwait(&sm.v_full[pstg], (uint32_t)(pg / kWsStages) & 1u);
+        if (ok) {
+          tc::fence_after_sync();
+          const uint32_t d = tmem + kColO + 64u * (uint32_t)(pn & 1), a = tmem + 128u * (uint32_t)(pg & 1);
+          const uint32_t vb = tc::smem_u32(sm.v[pstg]);
+#pragma unroll
+          for (int kk = 0; kk < kWsS / 16; ++kk)
+            tc::mma_f16_tmem_a(d, a + 8u * kk, tc::desc_kmajor(vb + kk * 2048, 1024, 128), idO,
+                               (pj > 0 || kk > 0) ? 1u : 0u);
+          tc::mma_commit(&sm.kv_empty[pstg]);
+          if (plast) tc::mma_commit(&sm.o_full[pn & 1]);
+        }
+      }
+      return __shfl_sync(0xffffffffu, ok, 0);
+    };
+    bool ok = true;
+    for (; it.valid(); it.next()) {
+      const int stg = it.g % kWsStages;
+      if (lane == 0) {
+        if (it.j == 0) ok = wwait(&sm.q_full[it.n & 1], (uint32_t)(it.n >> 1) & 1u);
+        if (ok) ok = wwait(&sm.k_full[stg], (uint32_t)(it.g / kWsStages) & 1u);
+        if (ok) {
+          tc::fence_after_sync();
+          const uint32_t d = tmem + 128u * (uint32_t)(it.g & 1), a = tmem + kColQ + 32u * (uint32_t)(it.n & 1);
+          const uint32_t kb = tc::smem_u32(sm.k[stg]);
+#pragma unroll
+          for (int kk = 0; kk < kHD / 16; ++kk)
+            tc::mma_f16_tmem_a(d, a + 8u * kk, tc::desc_kmajor(kb + kk * 256, 128, 1024), idS, kk > 0 ? 1u : 0u);
+          tc::mma_commit(&sm.s_full[it.g & 1]);
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      if (pg >= 0 && !issue_o()) {
+        ok = false;
+        break;
+      }
+      pg = it.g, pstg = stg, pn = it.n, pj = it.j, plast = (it.j + 1 == it.nst);
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok && pg >= 0) (void)issue_o();
+    if (lane == 0) {  // everything issued has completed before tensor memory is freed
+      tc::mma_commit(&sm.drain);
+      (void)tc::mbar_wait_bounded(&sm.drain, 0, kWaitNs);
+    }
+    __syncwarp();
+  } else if (warp >= 4 && warp < 12) {
+    // ---------------- weighting: P = S (.) f[t - s], even steps on warps 4-7, odd on 8-11
+    const int wg = (warp >> 2) - 1;
+    const int row = 32 * (warp & 3) + lane;  // TMEM lane = row of the t tile
+    const int wt = tid & 127;                // thread of the group
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    if (wg == 1) it.next();
+    WsIter nx = it;
+    nx.next();
+    nx.next();
+    // window of a step: W[x] = f[t0 - s0 - 127 + x] (+ D at 0, 0 below 0), x < 255;
+    // this thread loads x = wt and wt + 128
+    auto load_win = [&](const WsIter& s, float& w0, float& w1) {
+      const float* fh = fdiag + (size_t)s.h * L;
+      const float dh = D[s.h];
+      const int d0 = (s.tt - s.j) * kT - 127 + wt, d1 = d0 + 128;
+      w0 = (d0 >= 0 && d0 < L) ? fh[d0] + (d0 == 0 ? dh : 0.f) : 0.f;
+      w1 = (wt < 127 && d1 >= 0 && d1 < L) ? fh[d1] + (d1 == 0 ? dh : 0.f) : 0.f;
+    };
+    float w0 = 0.f, w1 = 0.f;
+    if (it.valid()) load_win(it, w0, w1);
+    int buf = 0;
+    while (it.valid()) {
+      // copy a of the window holds W[x + a] at x, so every 4-column group reads one aligned float4
+      float* wb = sm.win[wg][buf];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        if (wt - a >= 0) wb[a * kWinStride + wt - a] = w0;
+        wb[a * kWinStride + wt + 128 - a] = w1;
+      }
+      nbar_sync(1 + wg, 128);
+      if (nx.valid()) load_win(nx, w0, w1);
+      const bool ok = wwait(&sm.s_full[it.g & 1], (uint32_t)(it.g >> 1) & 1u);
+      if (nbar_or(1 + wg, 128, !ok)) break;
+      tc::fence_after_sync();
+      const uint32_t sb = tmem + 128u * (uint32_t)(it.g & 1) + lane_off;
+      // weights of columns c .. c+3 (c = 0 mod 4): W[r-c+124 .. r-c+127] = copy (r & 3) at (r - (r & 3)) - c + 124
+      const float* wq = wb + (row & 3) * kWinStride + (row - (row & 3)) + 124;
+#pragma unroll
+      for (int cb = 0; cb < kWsS / 32; ++cb) {
+        float s[32];
+        tc::tmem_ld16x2_wait(sb + (uint32_t)(32 * cb), sb + (uint32_t)(32 * cb + 16), s, s + 16);
+        uint32_t pk[16];
+#pragma unroll
+        for (int g4 = 0; g4 < 8; ++g4) {
+          const float4 w4 = *reinterpret_cast<const float4*>(wq - (32 * cb + 4 * g4));
+          pk[2 * g4] = Bits<T>::pack(s[4 * g4] * w4.w, s[4 * g4 + 1] * w4.z);
+          pk[2 * g4 + 1] = Bits<T>::pack(s[4 * g4 + 2] * w4.y, s[4 * g4 + 3] * w4.x);
+        }
+        // P columns [16 cb, 16 cb + 16) lie in S columns this thread has already read
+        tc::tmem_st8(sb + (uint32_t)(16 * cb), pk);
+        tc::tmem_st8(sb + (uint32_t)(16 * cb + 8), pk + 8);
+      }
+      tc::tmem_wait_st();
+      tc::fence_before_sync();
+      tc::mbar_arrive(&sm.p_full[it.g & 1]);
+      buf ^= 1;
+      it = nx;
+      nx.next();
+      nx.next();
+    }
+  } else if (warp >= 12) {
+    // ---------------- Q into tensor memory, O out
+    const int row = 32 * (warp & 3) + lane;
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint16_t* qb = reinterpret_cast<const uint16_t*>(q);
+    uint16_t* ob = reinterpret_cast<uint16_t*>(o);
+    auto load_q = [&](const WsIter& s) {
+      const int t = s.tt * kT + row;
+      uint32_t w[32];
+      if (t < L) {
+        const uint4* src = reinterpret_cast<const uint4*>(qb + ((size_t)s.b * L + t) * dm + (size_t)s.h * kHD);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint4 x = src[i];
+          w[4 * i] = x.x, w[4 * i + 1] = x.y, w[4 * i + 2] = x.z, w[4 * i + 3] = x.w;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) w[i] = 0u;
+      }
+      const uint32_t qa = tmem + kColQ + 32u * (uint32_t)(s.n & 1) + lane_off;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tc::tmem_st8(qa + 8u * i, w + 8 * i);
+      tc::tmem_wait_st();
+      tc::fence_before_sync();
+      tc::mbar_arrive(&sm.q_full[s.n & 1]);
+    };
+    if (it.valid()) load_q(it);
+    while (it.valid()) {
+      WsIter nx = it;
+      nx.next_item();
+      if (nx.valid()) load_q(nx);  // its buffer was last read by item n - 1, already written out
+      const bool ok = wwait(&sm.o_full[it.n & 1], (uint32_t)(it.n >> 1) & 1u);
+      if (nbar_or(3, 128, !ok)) break;
+      tc::fence_after_sync();
+      const uint32_t oa = tmem + kColO + 64u * (uint32_t)(it.n & 1) + lane_off;
+      float ov[64];
+      tc::tmem_ld16x2_wait(oa, oa + 16u, ov, ov + 16);
+      tc::tmem_ld16x2_wait(oa + 32u, oa + 48u, ov + 32, ov + 48);
+      tc::fence_before_sync();
+      tc::mbar_arrive(&sm.o_empty[it.n & 1]);
+      const int t = it.tt * kT + row;
+      if (t < L) {
+        uint4* dst = reinterpret_cast<uint4*>(ob + ((size_t)it.b * L + t) * dm + (size_t)it.h * kHD);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          dst[i] = make_uint4(Bits<T>::pack(ov[8 * i], ov[8 * i + 1]), Bits<T>::pack(ov[8 * i + 2], ov[8 * i + 3]),
+                              Bits<T>::pack(ov[8 * i + 4], ov[8 * i + 5]), Bits<T>::pack(ov[8 * i + 6], ov[8 * i + 7]));
+      }
+      it = nx;
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (tid == 0 && sm.abort) atomicAdd(&g_mixer_timeouts, 1u);
+  if (warp == 1) tc::tmem_dealloc(tmem, kWsCols);
+}
+
 template <typename T>
 static cudaError_t mixer_tc_t(const void* q, const void* k, const void* v, const float* Cs, const float* f,
                               const float* D, void* o, void* kt, int B, int L, int heads, int S, cudaStream_t st) {
@@ -367,6 +716,22 @@ static cudaError_t mixer_tc_t(const void* q, const void* k, const void* v, const
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (L % 8 == 0) {
+    // warp-specialised form: K~ and V tiles through tensor maps (rows in groups of 8)
+    CUtensorMap kmap, vmap;
+    const cuuint64_t dims[5] = {8, 8, (cuuint64_t)(dm / 8), (cuuint64_t)(L / 8), (cuuint64_t)B};
+    const cuuint64_t strides[4] = {(cuuint64_t)dm * 2, 16, (cuuint64_t)dm * 16, (cuuint64_t)L * dm * 2};
+    const cuuint32_t box[5] = {8, 8, 8, 16, 1};
+    if ((e = encode_map_5d_u16(&kmap, kt, dims, strides, box)) != cudaSuccess) return e;
+    if ((e = encode_map_5d_u16(&vmap, v, dims, strides, box)) != cudaSuccess) return e;
+    const size_t wsmem = sizeof(WsSmem);
+    if ((e = smem_optin<h3_mixer_ws_kernel<T>>(wsmem)) != cudaSuccess) return e;
+    const long long items = (long long)((L + kT - 1) / kT) * heads * B;
+    if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const int grid = (int)std::min<long long>(items, (long long)num_sms());
+    h3_mixer_ws_kernel<T><<<grid, kWsThr, wsmem, st>>>((const T*)q, f, D, (T*)o, L, heads, B, kmap, vmap);
+    return cudaGetLastError();
+  }
   const size_t smem = sizeof(MixSmem) + 1024;
   auto kern = h3_mixer_tc_kernel<T>;
   e = smem_optin<h3_mixer_tc_kernel<T>>(smem);

@@ -264,10 +264,12 @@ def _head_err(o, ref, mw, rows, ts):
 
 @pytest.mark.parametrize("dtype,L,S,heads", [("f32", 200, 4, 2), ("f16", 130, 4, 2), ("f32", 64, 1, 2),
                                              ("bf16", 96, 3, 2), ("f16", 256, 8, 3), ("bf16", 129, 1, 1),
-                                             ("f16", 300, 2, 2)])
+                                             ("f16", 300, 2, 2), ("f16", 1000, 4, 3), ("bf16", 512, 2, 5),
+                                             ("f16", 1024, 1, 1)])
 def test_h3_mixer_small(dtype, L, S, heads):
-    """fp32 I/O runs the CUDA-core kernel, fp16/bf16 the tensor-core one
-    (128-row tiles: ragged, exact and multi-tile lengths)."""
+    """fp32 I/O runs the CUDA-core kernel, fp16/bf16 the tensor-core ones
+    (128-row tiles: ragged, exact and multi-tile lengths; L a multiple of 8
+    takes the warp-specialised kernel, other L the one-tile-per-CTA kernel)."""
     mw = W.make_mixer(B=2, L=L, heads=heads, head_dim=64, N=8, shift_len=S, dtype=dtype, seed=L)
     o = _mixer_gpu(mw)
     ref = _mixer_ref(mw)
