@@ -49,6 +49,22 @@ __device__ __forceinline__ uint64_t desc_kmajor(uint32_t saddr, uint32_t lbo_byt
   return d;                 // base offset 0, no swizzle
 }
 
+// Descriptor of an operand tile stored with the 128-byte swizzle (rows of 64
+// 16-bit elements, 8-row atoms of 1024 bytes, atoms 1024-byte aligned).
+// K-major: rows are M/N, consecutive 8-row atoms sbo bytes apart, the leading
+// offset unused; a K step of 16 elements inside the atom advances the start
+// address by 32 bytes.  MN-major: rows are K, 64 M/N elements per row, K atoms
+// sbo bytes apart, lbo the distance between 64-wide M/N blocks.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;  // descriptor version for sm_100
+  d |= (uint64_t)2u << 61;  // 128-byte swizzle
+  return d;
+}
+
 // kind::f16 instruction descriptor: fp32 accumulator, A and B both fp16
 // (ab_bf16 = 0) or both bf16 (1), dense; a_mn / b_mn select MN-major operands.
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int ab_bf16, int a_mn = 0, int b_mn = 0) {
@@ -131,6 +147,15 @@ __device__ __forceinline__ void tma_load_5d(uint32_t dst, const void* tmap, int 
       "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5, "
       "%6}], [%7];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(smem_u32(mbar))
+      : "memory");
+}
+
+// Tiled (tensor-map) TMA load of one 3-d box, counted on mbar as it lands.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int c0, int c1, int c2, uint64_t* mbar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(mbar))
       : "memory");
 }
 
