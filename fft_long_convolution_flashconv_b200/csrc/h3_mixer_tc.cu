@@ -143,9 +143,10 @@ struct WsSmem {
   uint8_t v[kWsStages][kWsTile];
   uint8_t q[2][kWsTile];
   float win[2][2][4 * kWinStride];          // [weighting group][buffer]: window copies shifted by 0..3
-  uint64_t k_full[kWsStages], v_full[kWsStages], kv_empty[kWsStages];
+  uint64_t k_full[kWsStages], v_full[kWsStages];
+  uint64_t o_done[kWsStages];  // O-MMA of step g done: frees ring stage g % 4 and S buffer g % 3
   uint64_t q_full[2], q_empty[2];
-  uint64_t s_full[kWsSBuf], p_full[kWsSBuf], s_free[kWsSBuf];
+  uint64_t s_full[kWsSBuf], p_full[kWsSBuf];
   uint64_t o_full[2], o_empty[2], drain[2];
   uint32_t tmem_base;
   int abort;
@@ -226,12 +227,11 @@ __global__ void __launch_bounds__(kWsThr, 1)
     for (int i = 0; i < kWsStages; ++i) {
       tc::mbar_init(&sm.k_full[i], 1);
       tc::mbar_init(&sm.v_full[i], 1);
-      tc::mbar_init(&sm.kv_empty[i], 1);
+      tc::mbar_init(&sm.o_done[i], 1);
     }
     for (int i = 0; i < kWsSBuf; ++i) {
       tc::mbar_init(&sm.s_full[i], 1);
       tc::mbar_init(&sm.p_full[i], 128);
-      tc::mbar_init(&sm.s_free[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&sm.q_full[i], 1);
@@ -282,7 +282,7 @@ __global__ void __launch_bounds__(kWsThr, 1)
             last_q = it.n;
           }
         }
-        if (ok && use > 0) ok = wwait(&sm.kv_empty[stg], (use - 1) & 1u);
+        if (ok && use > 0) ok = wwait(&sm.o_done[stg], (use - 1) & 1u);  // O-MMA of step g - 4
         if (ok) {
           const int s0 = it.j * kWsS;
           tc::mbar_expect_tx(&sm.k_full[stg], kWsTile);
@@ -316,7 +316,10 @@ __global__ void __launch_bounds__(kWsThr, 1)
       if (lane == 0) {
         if (it.j == 0) ok = wwait(&sm.q_full[it.n & 1], (uint32_t)(it.n >> 1) & 1u);
         if (ok) ok = wwait(&sm.k_full[stg], (uint32_t)(it.g / kWsStages) & 1u);
-        if (ok && it.g >= kWsSBuf) ok = wwait(&sm.s_free[sb], (uint32_t)(it.g / kWsSBuf - 1) & 1u);
+        if (ok && it.g >= kWsSBuf) {  // O-MMA of step g - 3 (never two phases behind: step g + 1 needs this S)
+          const int gp = it.g - kWsSBuf;
+          ok = wwait(&sm.o_done[gp % kWsStages], (uint32_t)(gp / kWsStages) & 1u);
+        }
         if (ok) {
           tc::fence_after_sync();
           const uint32_t d = tmem + 128u * (uint32_t)sb;
@@ -355,8 +358,7 @@ __global__ void __launch_bounds__(kWsThr, 1)
 #pragma unroll
           for (int kk = 1; kk < kWsS / 16; ++kk)
             tc::mma_f16_tmem_a(d, a + 8u * kk, va + 128u * kk, idO, 1u);  // +2048 bytes: two K atoms
-          tc::mma_commit(&sm.kv_empty[stg]);
-          tc::mma_commit(&sm.s_free[sb]);
+          tc::mma_commit(&sm.o_done[stg]);
           if (it.j + 1 == it.nst) tc::mma_commit(&sm.o_full[it.n & 1]);
         }
       }
