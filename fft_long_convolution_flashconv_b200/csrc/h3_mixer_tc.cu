@@ -54,12 +54,14 @@ template <> struct Bits<__nv_bfloat16> {
 
 // k~ = shift SSM of k (B x L x dm, same type as k).  A thread owns 8 adjacent
 // channels (their taps stay in registers) and kSeg consecutive time steps of
-// one sequence: it loads those rows plus the S - 1 rows before them once, all
-// up front, then forms the kSeg outputs from registers.  A warp covers 256
-// adjacent channels of one time step (512-byte coalesced rows).
-constexpr int kSeg = 16;
+// one sequence, read in batches of kBatch rows through a register window that
+// carries the last S - 1 rows over, so each input row is loaded once per
+// segment (plus S - 1 halo rows).  Consecutive threads take consecutive
+// channel groups of the same rows: every load and store is a coalesced 16-byte
+// access, and all segments are resident at once (one wave).
+constexpr int kSeg = 32, kBatch = 8;
 template <typename T, int S>
-__global__ void __launch_bounds__(256) shift_ssm_kernel(const T* __restrict__ k, const float* __restrict__ Cshift,
+__global__ void __launch_bounds__(128) shift_ssm_kernel(const T* __restrict__ k, const float* __restrict__ Cshift,
                                                         T* __restrict__ kt, int B, int L, int dm) {
   const int ng = dm / 8;
   const int nseg = (L + kSeg - 1) / kSeg;
@@ -72,38 +74,48 @@ __global__ void __launch_bounds__(256) shift_ssm_kernel(const T* __restrict__ k,
   const uint16_t* kb = reinterpret_cast<const uint16_t*>(k) + (size_t)b * L * dm + c8;
   uint16_t* ob = reinterpret_cast<uint16_t*>(kt) + (size_t)b * L * dm + c8;
   const int t0 = seg * kSeg;
-  // rows t0 - (S-1) .. t0 + kSeg - 1, all loads issued before any use (zero outside [0, L))
-  uint4 rows[kSeg + S - 1];
-#pragma unroll
-  for (int i = 0; i < kSeg + S - 1; ++i) {
-    const int t = t0 - (S - 1) + i;
-    rows[i] = (t >= 0 && t < L) ? *reinterpret_cast<const uint4*>(kb + (size_t)t * dm) : make_uint4(0, 0, 0, 0);
-  }
   float cs[S][8];
 #pragma unroll
   for (int j = 0; j < S; ++j)
 #pragma unroll
     for (int i = 0; i < 8; ++i) cs[j][i] = __ldg(Cshift + (size_t)(c8 + i) * S + j);
+  // w[S - 1 + i] = row t0 + i0 + i of the batch, w[0 .. S - 2] the S - 1 rows before it (zero before 0)
+  uint4 w[S - 1 + kBatch];
 #pragma unroll
-  for (int i = 0; i < kSeg; ++i) {
-    const int t = t0 + i;
-    if (t < L) {
+  for (int i = 0; i < S - 1; ++i) {
+    const int t = t0 - (S - 1) + i;
+    w[i] = t >= 0 ? *reinterpret_cast<const uint4*>(kb + (size_t)t * dm) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll 1
+  for (int i0 = 0; i0 < kSeg && t0 + i0 < L; i0 += kBatch) {
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int t = t0 + i0 + i;
+      w[S - 1 + i] = t < L ? *reinterpret_cast<const uint4*>(kb + (size_t)t * dm) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int t = t0 + i0 + i;
       float acc[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) acc[c] = 0.f;
 #pragma unroll
       for (int j = 0; j < S; ++j) {  // tap j reads row t - j
-        const uint16_t* e = reinterpret_cast<const uint16_t*>(&rows[i + S - 1 - j]);
+        const uint16_t* e = reinterpret_cast<const uint16_t*>(&w[S - 1 + i - j]);
 #pragma unroll
         for (int c = 0; c < 8; ++c) acc[c] = fmaf(cs[j][c], Bits<T>::tof(e[c]), acc[c]);
       }
-      uint4 out;
-      out.x = Bits<T>::pack(acc[0], acc[1]);
-      out.y = Bits<T>::pack(acc[2], acc[3]);
-      out.z = Bits<T>::pack(acc[4], acc[5]);
-      out.w = Bits<T>::pack(acc[6], acc[7]);
-      *reinterpret_cast<uint4*>(ob + (size_t)t * dm) = out;
+      if (t < L) {
+        uint4 out;
+        out.x = Bits<T>::pack(acc[0], acc[1]);
+        out.y = Bits<T>::pack(acc[2], acc[3]);
+        out.z = Bits<T>::pack(acc[4], acc[5]);
+        out.w = Bits<T>::pack(acc[6], acc[7]);
+        *reinterpret_cast<uint4*>(ob + (size_t)t * dm) = out;
+      }
     }
+#pragma unroll
+    for (int i = 0; i < S - 1; ++i) w[i] = w[kBatch + i];
   }
 }
 
@@ -468,18 +480,18 @@ static cudaError_t mixer_tc_t(const void* q, const void* k, const void* v, const
                               const float* D, void* o, void* kt, int B, int L, int heads, int S, cudaStream_t st) {
   const int dm = heads * kHD;
   const long long items = (long long)B * ((L + kSeg - 1) / kSeg) * (dm / 8);
-  const unsigned sg = (unsigned)((items + 255) / 256);
+  const unsigned sg = (unsigned)((items + 127) / 128);
   const T* kk = (const T*)k;
   T* ko = (T*)kt;
   switch (S) {
-    case 1: shift_ssm_kernel<T, 1><<<sg, 256, 0, st>>>(kk, Cs, ko, B, L, dm); break;
-    case 2: shift_ssm_kernel<T, 2><<<sg, 256, 0, st>>>(kk, Cs, ko, B, L, dm); break;
-    case 3: shift_ssm_kernel<T, 3><<<sg, 256, 0, st>>>(kk, Cs, ko, B, L, dm); break;
-    case 4: shift_ssm_kernel<T, 4><<<sg, 256, 0, st>>>(kk, Cs, ko, B, L, dm); break;
-    case 5: shift_ssm_kernel<T, 5><<<sg, 256, 0, st>>>(kk, Cs, ko, B, L, dm); break;
-    case 6: shift_ssm_kernel<T, 6><<<sg, 256, 0, st>>>(kk, Cs, ko, B, L, dm); break;
-    case 7: shift_ssm_kernel<T, 7><<<sg, 256, 0, st>>>(kk, Cs, ko, B, L, dm); break;
-    case 8: shift_ssm_kernel<T, 8><<<sg, 256, 0, st>>>(kk, Cs, ko, B, L, dm); break;
+    case 1: shift_ssm_kernel<T, 1><<<sg, 128, 0, st>>>(kk, Cs, ko, B, L, dm); break;
+    case 2: shift_ssm_kernel<T, 2><<<sg, 128, 0, st>>>(kk, Cs, ko, B, L, dm); break;
+    case 3: shift_ssm_kernel<T, 3><<<sg, 128, 0, st>>>(kk, Cs, ko, B, L, dm); break;
+    case 4: shift_ssm_kernel<T, 4><<<sg, 128, 0, st>>>(kk, Cs, ko, B, L, dm); break;
+    case 5: shift_ssm_kernel<T, 5><<<sg, 128, 0, st>>>(kk, Cs, ko, B, L, dm); break;
+    case 6: shift_ssm_kernel<T, 6><<<sg, 128, 0, st>>>(kk, Cs, ko, B, L, dm); break;
+    case 7: shift_ssm_kernel<T, 7><<<sg, 128, 0, st>>>(kk, Cs, ko, B, L, dm); break;
+    case 8: shift_ssm_kernel<T, 8><<<sg, 128, 0, st>>>(kk, Cs, ko, B, L, dm); break;
     default: return cudaErrorInvalidValue;
   }
   cudaError_t e = cudaGetLastError();
