@@ -58,15 +58,22 @@ template <> struct Bits<__nv_bfloat16> {
 // carries the last S - 1 rows over, so each input row is loaded once per
 // segment (plus S - 1 halo rows).  Consecutive threads take consecutive
 // channel groups of the same rows: every load and store is a coalesced 16-byte
-// access, and all segments are resident at once (one wave).
-constexpr int kSeg = 32, kBatch = 8;
+// access.  The kernel runs as a programmatic dependent of the filter
+// generator, whose output it does not read: it lets the mixer launch early,
+// does its own work while the generator runs, and waits for the generator only
+// before it exits, so its completion implies the generator's.
+constexpr int kSeg = 32, kBatch = 16;
 template <typename T, int S>
-__global__ void __launch_bounds__(128) shift_ssm_kernel(const T* __restrict__ k, const float* __restrict__ Cshift,
+__global__ void __launch_bounds__(128, 3) shift_ssm_kernel(const T* __restrict__ k, const float* __restrict__ Cshift,
                                                         T* __restrict__ kt, int B, int L, int dm) {
   const int ng = dm / 8;
   const int nseg = (L + kSeg - 1) / kSeg;
+  asm volatile("griddepcontrol.launch_dependents;");
   const long long item = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (item >= (long long)B * nseg * ng) return;
+  if (item >= (long long)B * nseg * ng) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    return;
+  }
   const int g = (int)(item % ng);
   const long long bs = item / ng;
   const int seg = (int)(bs % nseg), b = (int)(bs / nseg);
@@ -117,6 +124,7 @@ __global__ void __launch_bounds__(128) shift_ssm_kernel(const T* __restrict__ k,
 #pragma unroll
     for (int i = 0; i < S - 1; ++i) w[i] = w[kBatch + i];
   }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -256,6 +264,9 @@ __global__ void __launch_bounds__(kWsThr, 1)
     tc::fence_mbar_init();
   }
   if (warp == 1) tc::tmem_alloc(&sm.tmem_base, kWsCols);
+  // launched as a programmatic dependent of the shift SSM: k~ (and, through it, the
+  // filters) are read only after that kernel has completed
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -483,17 +494,29 @@ static cudaError_t mixer_tc_t(const void* q, const void* k, const void* v, const
   const unsigned sg = (unsigned)((items + 127) / 128);
   const T* kk = (const T*)k;
   T* ko = (T*)kt;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(sg);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e0;
   switch (S) {
-    case 1: shift_ssm_kernel<T, 1><<<sg, 128, 0, st>>>(kk, Cs, ko, B, L, dm); break;
-    case 2: shift_ssm_kernel<T, 2><<<sg, 128, 0, st>>>(kk, Cs, ko, B, L, dm); break;
-    case 3: shift_ssm_kernel<T, 3><<<sg, 128, 0, st>>>(kk, Cs, ko, B, L, dm); break;
-    case 4: shift_ssm_kernel<T, 4><<<sg, 128, 0, st>>>(kk, Cs, ko, B, L, dm); break;
-    case 5: shift_ssm_kernel<T, 5><<<sg, 128, 0, st>>>(kk, Cs, ko, B, L, dm); break;
-    case 6: shift_ssm_kernel<T, 6><<<sg, 128, 0, st>>>(kk, Cs, ko, B, L, dm); break;
-    case 7: shift_ssm_kernel<T, 7><<<sg, 128, 0, st>>>(kk, Cs, ko, B, L, dm); break;
-    case 8: shift_ssm_kernel<T, 8><<<sg, 128, 0, st>>>(kk, Cs, ko, B, L, dm); break;
+    case 1: e0 = cudaLaunchKernelEx(&cfg, shift_ssm_kernel<T, 1>, kk, Cs, ko, B, L, dm); break;
+    case 2: e0 = cudaLaunchKernelEx(&cfg, shift_ssm_kernel<T, 2>, kk, Cs, ko, B, L, dm); break;
+    case 3: e0 = cudaLaunchKernelEx(&cfg, shift_ssm_kernel<T, 3>, kk, Cs, ko, B, L, dm); break;
+    case 4: e0 = cudaLaunchKernelEx(&cfg, shift_ssm_kernel<T, 4>, kk, Cs, ko, B, L, dm); break;
+    case 5: e0 = cudaLaunchKernelEx(&cfg, shift_ssm_kernel<T, 5>, kk, Cs, ko, B, L, dm); break;
+    case 6: e0 = cudaLaunchKernelEx(&cfg, shift_ssm_kernel<T, 6>, kk, Cs, ko, B, L, dm); break;
+    case 7: e0 = cudaLaunchKernelEx(&cfg, shift_ssm_kernel<T, 7>, kk, Cs, ko, B, L, dm); break;
+    case 8: e0 = cudaLaunchKernelEx(&cfg, shift_ssm_kernel<T, 8>, kk, Cs, ko, B, L, dm); break;
     default: return cudaErrorInvalidValue;
   }
+  if (e0 != cudaSuccess) return e0;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // Q, K~ and V tiles (128 rows x one head's 64 columns) through swizzled tensor maps
@@ -509,8 +532,14 @@ static cudaError_t mixer_tc_t(const void* q, const void* k, const void* v, const
   const long long tiles = (long long)((L + kT - 1) / kT) * heads * B;
   if (tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
   const int grid = (int)std::min<long long>(tiles, (long long)num_sms());
-  h3_mixer_ws_kernel<T><<<grid, kWsThr, wsmem, st>>>(f, D, (T*)o, L, heads, B, qmap, kmap, vmap);
-  return cudaGetLastError();
+  cudaLaunchConfig_t mcfg = {};
+  mcfg.gridDim = dim3(grid);
+  mcfg.blockDim = dim3(kWsThr);
+  mcfg.dynamicSmemBytes = wsmem;
+  mcfg.stream = st;
+  mcfg.attrs = attr;
+  mcfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&mcfg, h3_mixer_ws_kernel<T>, f, D, (T*)o, L, heads, B, qmap, kmap, vmap);
 }
 
 cudaError_t launch_h3_mixer_tc(const void* q, const void* k, const void* v, const float* Cshift, const float* fdiag,
