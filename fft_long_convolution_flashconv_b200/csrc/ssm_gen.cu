@@ -296,6 +296,192 @@ __global__ void __launch_bounds__(kGThr, SHORT ? 4 : 2) ssm_gen_tc_kernel(const 
   if (warp == 0) tc::tmem_dealloc(*sm.tmem_p, 32);
 }
 
+// Long filters (L > 2048): 64-tap rows, t = 64 th + tl (tl < 64), one GEMM per 8192 taps,
+//   f[64 th + tl] = sum_k AH[th][k] Q[tl][k]        (M = 128 rows th, N = 64, K = 128)
+//   AH[th][2n] + i AH[th][2n+1] = A_n^(64 th),  Q[tl][2n] - i Q[tl][2n+1] = 2 C_n B_n A_n^tl,
+// split hi/lo as above.  Four times the taps per MMA group and per table of the 16-tap form, so
+// the tables, the 24 MMAs and the waits are paid once per 8192 taps instead of per 2048.
+// AH[th] = A^(8192 u) A^(2048 r) A^(512 gq) A^(64 m) for th = 8 (gq + 4 r) + m (exact powers A,
+// A^16, A^64, A^512, A^2048; at most 7 products each); Q[tl] = w A^(16 gq) A^j, tl = 16 gq + j.
+namespace {
+constexpr int kG64Units = 2;                    // 8192-tap units per CTA
+constexpr int kG64Cols = 64, kG64UnitTaps = kGRows * kG64Cols;
+constexpr uint32_t kG64Q = (kG64Cols / 8) * kGSbo;
+struct Gen64Layout {
+  static constexpr uint32_t ahh = 0, ahl = kGTab, qh = 2 * kGTab, ql = qh + kG64Q, pw = ql + kG64Q;
+  static constexpr uint32_t red = pw + 64 * 5 * 8, mbar = red + 32, tmem = mbar + 8, bytes = tmem + 8;
+};
+}  // namespace
+
+__global__ void __launch_bounds__(kGThr, 2) ssm_gen_tc64_kernel(const float* __restrict__ dt,
+                                                                const float2* __restrict__ lam,
+                                                                const float2* __restrict__ Bp,
+                                                                const float2* __restrict__ Cp, int H, int N, int L,
+                                                                float* __restrict__ f) {
+  asm volatile("griddepcontrol.launch_dependents;");  // see ssm_gen_tc_kernel
+  using LY = Gen64Layout;
+  extern __shared__ __align__(1024) uint8_t gtsm[];
+  uint8_t* ahh = gtsm + LY::ahh;
+  uint8_t* ahl = gtsm + LY::ahl;
+  uint8_t* qh = gtsm + LY::qh;
+  uint8_t* ql = gtsm + LY::ql;
+  float2* pw = reinterpret_cast<float2*>(gtsm + LY::pw);
+  float* red = reinterpret_cast<float*>(gtsm + LY::red);
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(gtsm + LY::mbar);
+  uint32_t* tmem_p = reinterpret_cast<uint32_t*>(gtsm + LY::tmem);
+  const int h = blockIdx.y;
+  const int units = (L + kG64UnitTaps - 1) / kG64UnitTaps;
+  const int u0 = blockIdx.x * kG64Units, u1 = min(units, u0 + kG64Units);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int n = tid & 63, gq = tid >> 6;  // this thread's mode and row-group phase (0..3)
+  const float d = dt[h];
+  if (warp == 0) tc::tmem_alloc(tmem_p, 64);
+  if (tid == 0) {
+    tc::mbar_init(mbar, 1);
+    tc::fence_mbar_init();
+  }
+  for (int idx = tid; idx < 64 * 5; idx += kGThr) {
+    const int m = idx / 5, e = idx - 5 * m;
+    float2 v = make_float2(0.f, 0.f);
+    if (m < N) {
+      const float2 l = lam[(size_t)h * N + m];
+      v = ssm_pow(d, l.x, l.y, e == 0 ? 1.0 : e == 1 ? 16.0 : e == 2 ? 64.0 : e == 3 ? 512.0 : 2048.0);
+    }
+    pw[idx] = v;
+  }
+  float2 lm = make_float2(0.f, 0.f), w = make_float2(0.f, 0.f);
+  if (n < N) {
+    lm = lam[(size_t)h * N + n];
+    const float2 cb = cmul(Cp[(size_t)h * N + n], Bp[(size_t)h * N + n]);
+    w = make_float2(2.f * cb.x, 2.f * cb.y);
+  }
+  // power-of-two scale: the largest |Re|, |Im| of any 2 C B just below 2^13
+  float mx = fmaxf(fabsf(w.x), fabsf(w.y));
+  mx = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(mx)));
+  if ((tid & 31) == 0) red[warp] = mx;
+  __syncthreads();
+  mx = 0.f;
+#pragma unroll
+  for (int i = 0; i < kGThr / 32; ++i) mx = fmaxf(mx, red[i]);
+  float scale = 1.f, inv = 1.f;
+  if (mx > 0.f && mx <= 3.0e38f) {
+    int ex = 0;
+    (void)frexpf(mx, &ex);
+    scale = ldexpf(1.f, 13 - ex);
+    inv = ldexpf(1.f, ex - 13);
+  }
+  const float2 a1 = pw[n * 5 + 0], a16 = pw[n * 5 + 1], a64 = pw[n * 5 + 2];
+  const float2 a512 = pw[n * 5 + 3], a2048 = pw[n * 5 + 4];
+  const float2 one = n < N ? make_float2(1.f, 0.f) : make_float2(0.f, 0.f);
+  float2 m8[8], G[4];
+  m8[0] = one;
+#pragma unroll
+  for (int m = 1; m < 8; ++m) m8[m] = cmul(m8[m - 1], a64);
+  float2 g512 = one, p16 = one;
+#pragma unroll
+  for (int i = 0; i < 3; ++i)
+    if (i < gq) {
+      g512 = cmul(g512, a512);
+      p16 = cmul(p16, a16);
+    }
+  G[0] = g512;
+#pragma unroll
+  for (int r = 1; r < 4; ++r) G[r] = cmul(G[r - 1], a2048);
+  // Q rows tl = 16 gq .. 16 gq + 15
+  {
+    float2 p = cmul(make_float2(w.x * scale, w.y * scale), p16);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      uint32_t lo;
+      const uint32_t hi = gsplit(p.x, -p.y, lo);
+      *reinterpret_cast<uint32_t*>(qh + goff(16 * gq + j, n)) = hi;
+      *reinterpret_cast<uint32_t*>(ql + goff(16 * gq + j, n)) = lo;
+      p = cmul(p, a1);
+    }
+  }
+  const uint32_t idesc = tc::idesc_f16(kGRows, kG64Cols, 0);
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+  const int half = warp >> 2;  // output columns 32 half .. 32 half + 31
+  const bool vec_ok = (L & 3) == 0;
+  uint32_t phase = 0;
+  bool failed = false;
+  for (int u = u0; u < u1; ++u) {
+    const int th0 = u * kGRows;
+    const int rows = min(kGRows, (L - th0 * kG64Cols + kG64Cols - 1) / kG64Cols);
+    const float2 base = n >= N ? make_float2(0.f, 0.f)
+                        : th0 == 0 ? make_float2(1.f, 0.f) : ssm_pow(d, lm.x, lm.y, 64.0 * th0);
+    if (u > u0) {  // the previous unit's MMAs have read the tables (its wait is behind us)
+      tc::fence_before_sync();
+      __syncthreads();
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int g = gq + 4 * r;
+      const float2 pg = cmul(base, G[r]);
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        // rows past the end feed only never-stored outputs: zero them
+        const float2 v = 8 * g + m < rows ? cmul(pg, m8[m]) : make_float2(0.f, 0.f);
+        uint32_t lo;
+        const uint32_t hi = gsplit(v.x, v.y, lo);
+        *reinterpret_cast<uint32_t*>(ahh + goff(8 * g + m, n)) = hi;
+        *reinterpret_cast<uint32_t*>(ahl + goff(8 * g + m, n)) = lo;
+      }
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_p;
+    if (tid == 0) {
+      const uint32_t ah = tc::smem_u32(ahh), al = tc::smem_u32(ahl);
+      const uint32_t bh = tc::smem_u32(qh), bl = tc::smem_u32(ql);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        tc::mma_f16(tmem, tc::desc_kmajor(ah + kk * 2 * kGLbo, kGLbo, kGSbo),
+                    tc::desc_kmajor(bh + kk * 2 * kGLbo, kGLbo, kGSbo), idesc, kk > 0 ? 1u : 0u);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        tc::mma_f16(tmem, tc::desc_kmajor(ah + kk * 2 * kGLbo, kGLbo, kGSbo),
+                    tc::desc_kmajor(bl + kk * 2 * kGLbo, kGLbo, kGSbo), idesc, 1u);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        tc::mma_f16(tmem, tc::desc_kmajor(al + kk * 2 * kGLbo, kGLbo, kGSbo),
+                    tc::desc_kmajor(bh + kk * 2 * kGLbo, kGLbo, kGSbo), idesc, 1u);
+      tc::mma_commit(mbar);
+    }
+    const bool ok = tc::mbar_wait_bounded(mbar, phase, kGWaitNs);
+    phase ^= 1u;
+    if (__syncthreads_or(!ok)) {
+      failed = true;
+      break;
+    }
+    tc::fence_after_sync();
+    float v[32];
+    tc::tmem_ld16x2_wait(tmem + lane_off + (uint32_t)(32 * half), tmem + lane_off + (uint32_t)(32 * half + 16), v,
+                         v + 16);
+    const int r = (warp & 3) * 32 + (tid & 31);  // TMEM lane = row
+    if (r < rows) {
+      const long long t0 = (long long)(th0 + r) * kG64Cols + 32 * half;
+      float* fp = f + (size_t)h * L + t0;
+      if (vec_ok && t0 + 32 <= L) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          reinterpret_cast<float4*>(fp)[q] =
+              make_float4(v[4 * q] * inv, v[4 * q + 1] * inv, v[4 * q + 2] * inv, v[4 * q + 3] * inv);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (t0 + j < L) fp[j] = v[j] * inv;
+      }
+    }
+  }
+  if (failed && tid == 0) atomicAdd(&g_gen_tc_timeouts, 1u);
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(*tmem_p, 64);
+}
+
 unsigned int gen_tc_timeouts() {
   unsigned int v = 0;
   cudaMemcpyFromSymbol(&v, g_gen_tc_timeouts, sizeof(v));
@@ -304,6 +490,16 @@ unsigned int gen_tc_timeouts() {
 
 cudaError_t launch_ssm_gen(const float* dt, const float* lam, const float* Bp, const float* Cp, int H, int N,
                            int L, float* f, cudaStream_t st) {
+  if (N <= 64 && L > 2 * kGUnitTaps) {
+    const int units = (L + kG64UnitTaps - 1) / kG64UnitTaps;
+    cudaError_t e = smem_optin<ssm_gen_tc64_kernel>(Gen64Layout::bytes);
+    if (e != cudaSuccess) return e;
+    dim3 grid((units + kG64Units - 1) / kG64Units, H);
+    ssm_gen_tc64_kernel<<<grid, kGThr, Gen64Layout::bytes, st>>>(
+        dt, reinterpret_cast<const float2*>(lam), reinterpret_cast<const float2*>(Bp),
+        reinterpret_cast<const float2*>(Cp), H, N, L, f);
+    return cudaGetLastError();
+  }
   if (N <= 64) {
     const int units = (L + kGUnitTaps - 1) / kGUnitTaps;
     const bool short_rows = L <= kGUnitTaps / 2;

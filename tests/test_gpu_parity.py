@@ -55,6 +55,9 @@ def oracle_A(wl, hs=None):
     (2, 1, 100, ("loguniform", -1.0, -1.0)),            # N = 1 (real A for n = 0)
     (3, 64, 1001, ("loguniform", -3.0, -1.0)),          # L % 16 != 0: ragged last row, scalar stores
     (2, 96, 3000, ("loguniform", -3.0, -1.0)),          # N > 64: CUDA-core generator
+    (3, 64, 12345, ("loguniform", -3.0, -1.0)),         # 64-tap rows: two units, ragged, scalar stores
+    (2, 32, 20000, ("loguniform", -3.0, -2.0)),         # 64-tap rows: three units over two CTAs
+    (4, 64, 4100, ("loguniform", -3.0, -1.0)),          # 64-tap rows: one partial unit
 ])
 def test_ssm_kernel_gen(H, N, L, dt):
     wl = W.make_conv(B=1, H=H, L=8, N=N, dtype="f32", seed=7, dt_range=dt)
