@@ -176,10 +176,12 @@ __global__ void __launch_bounds__(kThrS, 2) sp_state_tc_kernel(const T* __restri
 
   // this lane's mode: row r = lane -> mode lane / 2, real (even) or imaginary (odd) part
   const int n = lane >> 1, part = lane & 1;
-  float2 w128 = make_float2(0.f, 0.f), whalf = make_float2(0.f, 0.f), bn = make_float2(0.f, 0.f);
+  float2 w128 = make_float2(0.f, 0.f), w256 = make_float2(0.f, 0.f), whalf = make_float2(0.f, 0.f),
+         bn = make_float2(0.f, 0.f);
   if (n < N) {
     const float2 lm = lam[(size_t)h * N + n];
     w128 = ssm_pow(d, lm.x, lm.y, (double)kKS);
+    w256 = ssm_pow(d, lm.x, lm.y, 2.0 * kKS);
     whalf = ssm_pow(d, lm.x, lm.y, (double)kKS * HC);
     bn = Bp[(size_t)h * N + n];
   }
@@ -230,25 +232,26 @@ __global__ void __launch_bounds__(kThrS, 2) sp_state_tc_kernel(const T* __restri
     }
     // Horner in A^128 over this half's columns ih = HC half .. HC half + HC - 1
     const uint32_t tm = sm.tmem_base + (uint32_t)((c & 1) * tmem_cols<NC>());
-    float z[HC];
+    uint32_t zv[HC];
 #pragma unroll
-    for (int j = 0; j < HC; j += 8) {
-      uint32_t v[8];
-      tc::tmem_ld8(tm + lane_off + (uint32_t)(HC * half + j), v);
-      tc::tmem_wait_ld();
+    for (int j = 0; j < HC; j += 8) tc::tmem_ld8(tm + lane_off + (uint32_t)(HC * half + j), zv + j);
+    tc::tmem_wait_ld();  // one wait for all of this thread's columns
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        tc::tmem_regs_ready(v[e]);
-        z[j + e] = __uint_as_float(v[e]);
-      }
+    for (int j = 0; j < HC; ++j) tc::tmem_regs_ready(zv[j]);
+    // two interleaved Horner chains in A^256 (even and odd columns), then even * A^128 + odd
+    float er = 0.f, ei = 0.f, orr = 0.f, oi = 0.f;
+#pragma unroll
+    for (int ih = 0; ih < HC; ih += 2) {
+      const float ze = __uint_as_float(zv[ih]), zo = __uint_as_float(zv[ih + 1]);
+      const float ner = fmaf(er, w256.x, fmaf(-ei, w256.y, ze));
+      ei = fmaf(er, w256.y, ei * w256.x);
+      er = ner;
+      const float nor = fmaf(orr, w256.x, fmaf(-oi, w256.y, zo));
+      oi = fmaf(orr, w256.y, oi * w256.x);
+      orr = nor;
     }
-    float ar = 0.f, ai = 0.f;
-#pragma unroll
-    for (int ih = 0; ih < HC; ++ih) {
-      const float nr = fmaf(ar, w128.x, fmaf(-ai, w128.y, z[ih]));
-      ai = fmaf(ar, w128.y, ai * w128.x);
-      ar = nr;
-    }
+    float ar = fmaf(er, w128.x, fmaf(-ei, w128.y, orr));
+    float ai = fmaf(er, w128.y, fmaf(ei, w128.x, oi));
     // lower half: times A^(128 HC) (its columns come HC blocks earlier), plus the upper half
     if (half == 1) sm.part[lane] = make_float2(ar, ai);
     tc::fence_before_sync();
