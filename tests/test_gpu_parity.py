@@ -58,6 +58,7 @@ def oracle_A(wl, hs=None):
     (3, 64, 12345, ("loguniform", -3.0, -1.0)),         # 64-tap rows: two units, ragged, scalar stores
     (2, 32, 20000, ("loguniform", -3.0, -2.0)),         # 64-tap rows: three units over two CTAs
     (4, 64, 4100, ("loguniform", -3.0, -1.0)),          # 64-tap rows: one partial unit
+    (2, 1, 5000, ("loguniform", -2.0, -1.0)),           # 64-tap rows, N = 1
 ])
 def test_ssm_kernel_gen(H, N, L, dt):
     wl = W.make_conv(B=1, H=H, L=8, N=N, dtype="f32", seed=7, dt_range=dt)
@@ -268,7 +269,8 @@ def _head_err(o, ref, mw, rows, ts):
 @pytest.mark.parametrize("dtype,L,S,heads", [("f32", 200, 4, 2), ("f16", 130, 4, 2), ("f32", 64, 1, 2),
                                              ("bf16", 96, 3, 2), ("f16", 256, 8, 3), ("bf16", 129, 1, 1),
                                              ("f16", 300, 2, 2), ("f16", 1000, 4, 3), ("bf16", 512, 2, 5),
-                                             ("f16", 1024, 1, 1)])
+                                             ("f16", 1024, 1, 1), ("f16", 1, 4, 1), ("bf16", 7, 8, 2),
+                                             ("f16", 2048, 3, 1)])
 def test_h3_mixer_small(dtype, L, S, heads):
     """fp32 I/O runs the CUDA-core kernel, fp16/bf16 the tensor-core ones
     (128-row tiles: ragged, exact and multi-tile lengths; L a multiple of 8
