@@ -66,12 +66,12 @@ cudaError_t run_ssm_conv(const void* u, const float* dt, const float* lambda, co
   const SsmArgs none{nullptr, nullptr, nullptr, nullptr, 0};
   cudaError_t e;
   if (fftconv_tc_supported(L, dtype, B)) {  // filter kernel, then the tensor-core convolution
-    e = launch_ssm_gen(dt, lambda, Bp, Cp, H, N, L, f, st);
+    e = launch_ssm_gen(dt, lambda, Bp, Cp, H, N, L, f, st, true);
     if (e != cudaSuccess) return e;
     return launch_fftconv_tc(u, f, D, y, B, H, L, dtype, true, st);
   }
   if (fftconv_tcl_supported(L, dtype)) {
-    e = launch_ssm_gen(dt, lambda, Bp, Cp, H, N, L, f, st);
+    e = launch_ssm_gen(dt, lambda, Bp, Cp, H, N, L, f, st, true);
     if (e != cudaSuccess) return e;
     return launch_fftconv_tcl(u, f, L, D, y, B, H, L, L, 1, dtype, true, false, st);
   }
@@ -245,7 +245,9 @@ static fc_status statepass_run(const void* u, const float* dt, const float* lamb
                                const float* D, void* y, int B, int H, int L, int N, int chunk, const float* state_in,
                                float* state_out, float* fT, float* s_ws, float* x_ws, int dtype, cudaStream_t st) {
   const int C = L / chunk;
-  fc_status s = cuda_status(fc::launch_ssm_gen(dt, lambda, Bp, Cp, H, N, chunk, fT, st), "statepass: filter launch");
+  fc_status s = cuda_status(fc::launch_ssm_gen(dt, lambda, Bp, Cp, H, N, chunk, fT, st,
+                                               fc::fftconv_tcl_supported(chunk, dtype)),
+                            "statepass: filter launch");
   if (s != FC_OK) return s;
   const fc::SsmArgs none{nullptr, nullptr, nullptr, nullptr, 0};
   s = fc::fftconv_tcl_supported(chunk, dtype)
@@ -396,7 +398,8 @@ FC_API fc_status h3_mixer_fwd(const void* q, const void* k, const void* v, const
   FC_REQUIRE(ws_bytes >= need, FC_EINVAL, "workspace too small: %zu < %zu bytes", ws_bytes, need);
   float* f = (float*)workspace;
   cudaStream_t st = (cudaStream_t)stream;
-  s = cuda_status(fc::launch_ssm_gen(dt, lambda, Bp, Cp, heads, N, L, f, st), "h3_mixer: filter launch");
+  s = cuda_status(fc::launch_ssm_gen(dt, lambda, Bp, Cp, heads, N, L, f, st, dtype == FC_F16 || dtype == FC_BF16),
+                  "h3_mixer: filter launch");
   if (s != FC_OK) return s;
   if (dtype == FC_F16 || dtype == FC_BF16) {
     void* kt = (char*)workspace + round_up((size_t)heads * L * sizeof(float), 256);

@@ -15,8 +15,11 @@ cudaError_t run_ssm_conv(const void* u, const float* dt, const float* lambda, co
                          const float* D, void* y, int B, int H, int L, int N, float* f, int dtype,
                          cudaStream_t st);
 
+// hi_only (N <= 64): single fp16 tables, about 11 significant bits, for a filter that a 16-bit
+// tensor-core convolution or the 16-bit mixer rounds to its operand type anyway; otherwise the
+// tables are split hi + lo (about 22 bits).
 cudaError_t launch_ssm_gen(const float* dt, const float* lam, const float* Bp, const float* Cp, int H, int N, int L,
-                           float* f, cudaStream_t st);
+                           float* f, cudaStream_t st, bool hi_only = false);
 
 // dtype: 0 f32, 1 f16, 2 bf16.  Lc = transform half-length (chunk), C chunks per row.
 // sp.dt != nullptr: generate the filter from the SSM parameters inside the

@@ -120,7 +120,7 @@ __device__ __forceinline__ uint32_t goff(int r, int n) {  // K elements (2n, 2n+
 }
 }  // namespace
 
-template <bool SHORT>
+template <bool SHORT, bool HI>
 __global__ void __launch_bounds__(kGThr, SHORT ? 4 : 2) ssm_gen_tc_kernel(const float* __restrict__ dt,
                                                                           const float2* __restrict__ lam,
                                                                           const float2* __restrict__ Bp,
@@ -213,7 +213,7 @@ __global__ void __launch_bounds__(kGThr, SHORT ? 4 : 2) ssm_gen_tc_kernel(const 
       uint32_t lo;
       const uint32_t hi = gsplit(p.x, -p.y, lo);
       *reinterpret_cast<uint32_t*>(sm.qh + goff(4 * gq + j, n)) = hi;
-      *reinterpret_cast<uint32_t*>(sm.ql + goff(4 * gq + j, n)) = lo;
+      if constexpr (!HI) *reinterpret_cast<uint32_t*>(sm.ql + goff(4 * gq + j, n)) = lo;
       p = cmul(p, a1);
     }
   }
@@ -238,7 +238,7 @@ __global__ void __launch_bounds__(kGThr, SHORT ? 4 : 2) ssm_gen_tc_kernel(const 
         uint32_t lo;
         const uint32_t hi = gsplit(v.x, v.y, lo);
         *reinterpret_cast<uint32_t*>(sm.ahh + goff(8 * g + m, n)) = hi;
-        *reinterpret_cast<uint32_t*>(sm.ahl + goff(8 * g + m, n)) = lo;
+        if constexpr (!HI) *reinterpret_cast<uint32_t*>(sm.ahl + goff(8 * g + m, n)) = lo;
       }
     }
     tc::fence_smem_to_async();
@@ -253,14 +253,16 @@ __global__ void __launch_bounds__(kGThr, SHORT ? 4 : 2) ssm_gen_tc_kernel(const 
       for (int kk = 0; kk < 8; ++kk)
         tc::mma_f16(tmem, tc::desc_kmajor(ah + kk * 2 * kGLbo, kGLbo, kGSbo),
                     tc::desc_kmajor(qh + kk * 2 * kGLbo, kGLbo, kGSbo), idesc, kk > 0 ? 1u : 0u);
+      if constexpr (!HI) {
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        tc::mma_f16(tmem, tc::desc_kmajor(ah + kk * 2 * kGLbo, kGLbo, kGSbo),
-                    tc::desc_kmajor(ql + kk * 2 * kGLbo, kGLbo, kGSbo), idesc, 1u);
+        for (int kk = 0; kk < 8; ++kk)
+          tc::mma_f16(tmem, tc::desc_kmajor(ah + kk * 2 * kGLbo, kGLbo, kGSbo),
+                      tc::desc_kmajor(ql + kk * 2 * kGLbo, kGLbo, kGSbo), idesc, 1u);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        tc::mma_f16(tmem, tc::desc_kmajor(al + kk * 2 * kGLbo, kGLbo, kGSbo),
-                    tc::desc_kmajor(qh + kk * 2 * kGLbo, kGLbo, kGSbo), idesc, 1u);
+        for (int kk = 0; kk < 8; ++kk)
+          tc::mma_f16(tmem, tc::desc_kmajor(al + kk * 2 * kGLbo, kGLbo, kGSbo),
+                      tc::desc_kmajor(qh + kk * 2 * kGLbo, kGLbo, kGSbo), idesc, 1u);
+      }
       tc::mma_commit(sm.mbar);
     }
     const bool ok = tc::mbar_wait_bounded(sm.mbar, phase, kGWaitNs);
@@ -313,6 +315,7 @@ struct Gen64Layout {
 };
 }  // namespace
 
+template <bool HI>
 __global__ void __launch_bounds__(kGThr, 2) ssm_gen_tc64_kernel(const float* __restrict__ dt,
                                                                 const float2* __restrict__ lam,
                                                                 const float2* __restrict__ Bp,
@@ -395,7 +398,7 @@ __global__ void __launch_bounds__(kGThr, 2) ssm_gen_tc64_kernel(const float* __r
       uint32_t lo;
       const uint32_t hi = gsplit(p.x, -p.y, lo);
       *reinterpret_cast<uint32_t*>(qh + goff(16 * gq + j, n)) = hi;
-      *reinterpret_cast<uint32_t*>(ql + goff(16 * gq + j, n)) = lo;
+      if constexpr (!HI) *reinterpret_cast<uint32_t*>(ql + goff(16 * gq + j, n)) = lo;
       p = cmul(p, a1);
     }
   }
@@ -425,7 +428,7 @@ __global__ void __launch_bounds__(kGThr, 2) ssm_gen_tc64_kernel(const float* __r
         uint32_t lo;
         const uint32_t hi = gsplit(v.x, v.y, lo);
         *reinterpret_cast<uint32_t*>(ahh + goff(8 * g + m, n)) = hi;
-        *reinterpret_cast<uint32_t*>(ahl + goff(8 * g + m, n)) = lo;
+        if constexpr (!HI) *reinterpret_cast<uint32_t*>(ahl + goff(8 * g + m, n)) = lo;
       }
     }
     tc::fence_smem_to_async();
@@ -440,14 +443,16 @@ __global__ void __launch_bounds__(kGThr, 2) ssm_gen_tc64_kernel(const float* __r
       for (int kk = 0; kk < 8; ++kk)
         tc::mma_f16(tmem, tc::desc_kmajor(ah + kk * 2 * kGLbo, kGLbo, kGSbo),
                     tc::desc_kmajor(bh + kk * 2 * kGLbo, kGLbo, kGSbo), idesc, kk > 0 ? 1u : 0u);
+      if constexpr (!HI) {
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        tc::mma_f16(tmem, tc::desc_kmajor(ah + kk * 2 * kGLbo, kGLbo, kGSbo),
-                    tc::desc_kmajor(bl + kk * 2 * kGLbo, kGLbo, kGSbo), idesc, 1u);
+        for (int kk = 0; kk < 8; ++kk)
+          tc::mma_f16(tmem, tc::desc_kmajor(ah + kk * 2 * kGLbo, kGLbo, kGSbo),
+                      tc::desc_kmajor(bl + kk * 2 * kGLbo, kGLbo, kGSbo), idesc, 1u);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        tc::mma_f16(tmem, tc::desc_kmajor(al + kk * 2 * kGLbo, kGLbo, kGSbo),
-                    tc::desc_kmajor(bh + kk * 2 * kGLbo, kGLbo, kGSbo), idesc, 1u);
+        for (int kk = 0; kk < 8; ++kk)
+          tc::mma_f16(tmem, tc::desc_kmajor(al + kk * 2 * kGLbo, kGLbo, kGSbo),
+                      tc::desc_kmajor(bh + kk * 2 * kGLbo, kGLbo, kGSbo), idesc, 1u);
+      }
       tc::mma_commit(mbar);
     }
     const bool ok = tc::mbar_wait_bounded(mbar, phase, kGWaitNs);
@@ -488,30 +493,36 @@ unsigned int gen_tc_timeouts() {
   return v;
 }
 
-cudaError_t launch_ssm_gen(const float* dt, const float* lam, const float* Bp, const float* Cp, int H, int N,
-                           int L, float* f, cudaStream_t st) {
-  if (N <= 64 && L > 2 * kGUnitTaps) {
+template <bool HI>
+static cudaError_t gen_tc(const float* dt, const float* lam, const float* Bp, const float* Cp, int H, int N, int L,
+                          float* f, cudaStream_t st) {
+  const float2* l2 = reinterpret_cast<const float2*>(lam);
+  const float2* b2 = reinterpret_cast<const float2*>(Bp);
+  const float2* c2 = reinterpret_cast<const float2*>(Cp);
+  if (L > 2 * kGUnitTaps) {
     const int units = (L + kG64UnitTaps - 1) / kG64UnitTaps;
-    cudaError_t e = smem_optin<ssm_gen_tc64_kernel>(Gen64Layout::bytes);
+    cudaError_t e = smem_optin<ssm_gen_tc64_kernel<HI>>(Gen64Layout::bytes);
     if (e != cudaSuccess) return e;
     dim3 grid((units + kG64Units - 1) / kG64Units, H);
-    ssm_gen_tc64_kernel<<<grid, kGThr, Gen64Layout::bytes, st>>>(
-        dt, reinterpret_cast<const float2*>(lam), reinterpret_cast<const float2*>(Bp),
-        reinterpret_cast<const float2*>(Cp), H, N, L, f);
+    ssm_gen_tc64_kernel<HI><<<grid, kGThr, Gen64Layout::bytes, st>>>(dt, l2, b2, c2, H, N, L, f);
     return cudaGetLastError();
   }
-  if (N <= 64) {
-    const int units = (L + kGUnitTaps - 1) / kGUnitTaps;
-    const bool short_rows = L <= kGUnitTaps / 2;
-    auto kern = short_rows ? ssm_gen_tc_kernel<true> : ssm_gen_tc_kernel<false>;
-    const size_t smem = short_rows ? GenLayout<true>::bytes : GenLayout<false>::bytes;
-    cudaError_t e = short_rows ? smem_optin<ssm_gen_tc_kernel<true>>(smem) : smem_optin<ssm_gen_tc_kernel<false>>(smem);
-    if (e != cudaSuccess) return e;
-    dim3 grid((units + kGUnits - 1) / kGUnits, H);
-    kern<<<grid, kGThr, smem, st>>>(dt, reinterpret_cast<const float2*>(lam), reinterpret_cast<const float2*>(Bp),
-                                    reinterpret_cast<const float2*>(Cp), H, N, L, f);
-    return cudaGetLastError();
-  }
+  const int units = (L + kGUnitTaps - 1) / kGUnitTaps;
+  const bool short_rows = L <= kGUnitTaps / 2;
+  auto kern = short_rows ? ssm_gen_tc_kernel<true, HI> : ssm_gen_tc_kernel<false, HI>;
+  const size_t smem = short_rows ? GenLayout<true>::bytes : GenLayout<false>::bytes;
+  cudaError_t e = short_rows ? smem_optin<ssm_gen_tc_kernel<true, HI>>(smem)
+                             : smem_optin<ssm_gen_tc_kernel<false, HI>>(smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((units + kGUnits - 1) / kGUnits, H);
+  kern<<<grid, kGThr, smem, st>>>(dt, l2, b2, c2, H, N, L, f);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ssm_gen(const float* dt, const float* lam, const float* Bp, const float* Cp, int H, int N,
+                           int L, float* f, cudaStream_t st, bool hi_only) {
+  if (N <= 64)
+    return hi_only ? gen_tc<true>(dt, lam, Bp, Cp, H, N, L, f, st) : gen_tc<false>(dt, lam, Bp, Cp, H, N, L, f, st);
 
   const int tiles = (L + kGenTile - 1) / kGenTile;
   cudaError_t e = smem_optin<ssm_gen_kernel>(kGenSmem);

@@ -172,7 +172,11 @@ FC_API fc_status fftconv_bwd(const void* dy, const void* u, const float* f, cons
 /* ssm_conv_fwd -- ssm_kernel_gen followed by fftconv_fwd in one call (the
  * filter is regenerated on the device every call).  workspace must hold
  * ssm_conv_workspace(H, L) bytes (the H x L filter).  Precision: that of
- * ssm_kernel_gen followed by that of fftconv_fwd. */
+ * ssm_kernel_gen followed by that of fftconv_fwd, except that when the
+ * convolution runs on the tensor cores (16-bit I/O, L = 1024 with B >= 3 or
+ * L in {2048, 4096, 8192}) and N <= 64, the filter comes from single fp16
+ * tables (about 11 significant bits instead of 22): the convolution rounds
+ * f + D to the 16-bit operand type anyway. */
 FC_API size_t ssm_conv_workspace(int H, int L);
 FC_API fc_status ssm_conv_fwd(const void* u, const float* dt, const float* lambda, const float* Bp,
                               const float* Cp, const float* D, void* y, int B, int H, int L, int N,
@@ -194,13 +198,16 @@ FC_API fc_status ssm_conv_fwd(const void* u, const float* dt, const float* lambd
  * call's state_in.  workspace: at least fftconv_statepass_workspace(...)
  * bytes, 256-byte aligned.  Limits: chunk a power of two, 16 <= chunk <=
  * 8192, L % chunk == 0, 1 <= N <= 256.
- * Precision: the chunk convolutions run on the CUDA cores in float32 and are
- * stored in the I/O type; the initial-state term is then added to the stored
- * values and the sum rounded again (two roundings for chunks after the
- * first).  With 16-bit I/O, chunk in {2048, 4096, 8192} and N <= 64, the end
- * states and the initial-state term are tensor-core GEMMs against tables
- * split hi/lo into 16-bit parts (about 22 significant bits; 16 for the
- * bfloat16 u-side table), with u as an exact 16-bit operand. */
+ * Precision: the chunk convolutions are stored in the I/O type; the
+ * initial-state term is then added to the stored values and the sum rounded
+ * again (two roundings for chunks after the first).  They run on the CUDA
+ * cores in float32, except with 16-bit I/O and chunk in {2048, 4096, 8192},
+ * where they are fftconv_fwd's tensor-core kernel (the chunk filter then
+ * comes from single fp16 tables, about 11 significant bits, for N <= 64).
+ * With 16-bit I/O, those chunks and N <= 64, the end states and the
+ * initial-state term are tensor-core GEMMs against tables split hi/lo into
+ * 16-bit parts (about 22 significant bits; 16 for the bfloat16 u-side
+ * table), with u as an exact 16-bit operand. */
 FC_API size_t fftconv_statepass_workspace(int B, int H, int L, int N, int chunk);
 FC_API fc_status fftconv_statepass(const void* u, const float* dt, const float* lambda, const float* Bp,
                                    const float* Cp, const float* D, void* y, int B, int H, int L, int N,
@@ -246,7 +253,8 @@ FC_API fc_status fftconv_statepass_bwd(const void* dy, const float* dt, const fl
  * Precision: FC_F32 runs in float32 on the CUDA cores.  16-bit I/O runs the
  * two GEMMs per tile on the tensor cores: k~ is stored in the I/O type, the
  * Toeplitz-weighted scores (f[t-s] + D [s == t]) (q_t . k~_s) are rounded to
- * the I/O type before they multiply v; accumulation is float32. */
+ * the I/O type before they multiply v; accumulation is float32; for N <= 64
+ * the filters come from single fp16 tables (about 11 significant bits). */
 FC_API size_t h3_mixer_workspace(int B, int L, int heads, int head_dim, int N);
 FC_API fc_status h3_mixer_fwd(const void* q, const void* k, const void* v, const float* Cshift,
                               const float* dt, const float* lambda, const float* Bp, const float* Cp,
