@@ -20,12 +20,14 @@
 //   Q[tl][2n]  - i Q[tl][2n+1]  = 2 C_n x_n A_n^(tl+1)          (per chunk)
 // is one M=128 N=NC K=128 GEMM per chunk.
 //
-// Precision: every table operand is split into a 16-bit high part and a
-// 16-bit remainder (hi + lo), and the MMAs sum hi*hi + hi*lo + lo*hi in fp32,
-// so each table carries ~22 significant bits (16 for bf16 u-side tables);
-// u itself is an exact 16-bit operand.  The correction's per-chunk operand is
-// scaled by a power of two so that its largest entry sits near 2^13 (fp16
-// range); the epilogue multiplies the scale back out exactly.  The powers
+// Precision: the per-head tables (P, AH) are split into a 16-bit high part and
+// a 16-bit remainder (hi + lo), ~22 significant bits (16 for the bf16 P
+// table); u itself is an exact 16-bit operand, so the end states sum
+// Phi*u + Plo*u.  The correction's per-chunk operand Q is a single fp16 table
+// (~11 bits, below the rounding of y itself) and the correction sums
+// AHhi*Q + AHlo*Q; Q is scaled by a power of two so that its largest entry
+// sits near 2^13 (fp16 range) and the epilogue multiplies the scale back out
+// exactly.  The powers
 // assume |A_n| <= 1 (Re lambda <= 0), as for any stable SSM.
 //
 // One CTA owns one (b, h) row and walks its chunks; the next chunk of u is
@@ -287,8 +289,7 @@ template <int NC>
 struct CorrSmem2 {
   uint8_t ahh[kTab];               // A: AH hi, 128 rows (th) x 128 K (2n + re/im)
   uint8_t ahl[kTab];               // A: AH lo
-  uint8_t qh[(NC / 8) * kSbo];     // B: Q hi, NC rows (tl) x 128 K
-  uint8_t ql[(NC / 8) * kSbo];     // B: Q lo
+  uint8_t qh[(NC / 8) * kSbo];     // B: Q (fp16), NC rows (tl) x 128 K
   float red[kThrS / 32];
   uint64_t mbar[2];
   uint32_t tmem_base;
@@ -388,11 +389,8 @@ __global__ void __launch_bounds__(kThrS, 2) sp_corr_tc_kernel(T* __restrict__ y,
       float2 p = cmul(w, st[r]);
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
-        uint32_t hi, lo;
-        split2<__half>(p.x, -p.y, hi, lo);
         const uint32_t off = toff(8 * tg + m, n >> 2) + (uint32_t)(n & 3) * 4u;
-        *reinterpret_cast<uint32_t*>(sm.qh + off) = hi;
-        *reinterpret_cast<uint32_t*>(sm.ql + off) = lo;
+        *reinterpret_cast<uint32_t*>(sm.qh + off) = Op16<__half>::bits(p.x) | (Op16<__half>::bits(-p.y) << 16);
         p = cmul(p, a1);
       }
     }
@@ -400,16 +398,12 @@ __global__ void __launch_bounds__(kThrS, 2) sp_corr_tc_kernel(T* __restrict__ y,
   };
   auto issue = [&](int c) {
     const uint32_t ah = tc::smem_u32(sm.ahh), al = tc::smem_u32(sm.ahl);
-    const uint32_t qh = tc::smem_u32(sm.qh), ql = tc::smem_u32(sm.ql);
+    const uint32_t qh = tc::smem_u32(sm.qh);
     const uint32_t tm = sm.tmem_base + (uint32_t)((c & 1) * tmem_cols<NC>());
 #pragma unroll
     for (int kk = 0; kk < kKS / 16; ++kk)
       tc::mma_f16(tm, tc::desc_kmajor(ah + kk * 2 * kLbo, kLbo, kSbo), tc::desc_kmajor(qh + kk * 2 * kLbo, kLbo, kSbo),
                   idesc, kk > 0 ? 1u : 0u);
-#pragma unroll
-    for (int kk = 0; kk < kKS / 16; ++kk)
-      tc::mma_f16(tm, tc::desc_kmajor(ah + kk * 2 * kLbo, kLbo, kSbo), tc::desc_kmajor(ql + kk * 2 * kLbo, kLbo, kSbo),
-                  idesc, 1u);
 #pragma unroll
     for (int kk = 0; kk < kKS / 16; ++kk)
       tc::mma_f16(tm, tc::desc_kmajor(al + kk * 2 * kLbo, kLbo, kSbo), tc::desc_kmajor(qh + kk * 2 * kLbo, kLbo, kSbo),
