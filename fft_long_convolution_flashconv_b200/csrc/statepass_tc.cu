@@ -23,7 +23,8 @@
 // Precision: the per-head tables (P, AH) are split into a 16-bit high part and
 // a 16-bit remainder (hi + lo), ~22 significant bits (16 for the bf16 P
 // table); u itself is an exact 16-bit operand, so the end states sum
-// Phi*u + Plo*u.  The correction's per-chunk operand Q is a single fp16 table
+// Phi*u + Plo*u -- with fp16 I/O only Phi*u: fp16 P alone carries 11 bits,
+// and the state's rounding stays far below the state tolerance.  The correction's per-chunk operand Q is a single fp16 table
 // (~11 bits, below the rounding of y itself) and the correction sums
 // AHhi*Q + AHlo*Q; Q is scaled by a power of two so that its largest entry
 // sits near 2^13 (fp16 range) and the epilogue multiplies the scale back out
@@ -198,10 +199,12 @@ __global__ void __launch_bounds__(kThrS, 2) sp_state_tc_kernel(const T* __restri
     for (int kk = 0; kk < kKS / 16; ++kk)
       tc::mma_f16(tm, tc::desc_kmajor(pa + kk * 2 * kLbo, kLbo, kSbo), tc::desc_kmajor(ua + kk * 2 * kLbo, kLbo, kSbo),
                   idesc, kk > 0 ? 1u : 0u);
+    if constexpr (Op16<T>::bf16) {  // fp16 P alone carries 11 bits; bf16 P needs its remainder
 #pragma unroll
-    for (int kk = 0; kk < kKS / 16; ++kk)
-      tc::mma_f16(tm, tc::desc_kmajor(pb + kk * 2 * kLbo, kLbo, kSbo), tc::desc_kmajor(ua + kk * 2 * kLbo, kLbo, kSbo),
-                  idesc, 1u);
+      for (int kk = 0; kk < kKS / 16; ++kk)
+        tc::mma_f16(tm, tc::desc_kmajor(pb + kk * 2 * kLbo, kLbo, kSbo), tc::desc_kmajor(ua + kk * 2 * kLbo, kLbo, kSbo),
+                    idesc, 1u);
+    }
     tc::mma_commit(&sm.mbar[c & 1]);
   };
   // chunk 0 landed (chunk 1 may still be in flight)
