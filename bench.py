@@ -482,7 +482,7 @@ def secondary_configs(T, dev, api, args, local_rank):
     ms, _ = graph_time(lambda: api.fftconv_long_fwd(u, f, D, out=y, workspace=ws), n, flush, rflush, stream)
     clocks = sampler.stop()
     out["longconv_f32_B8_H256_L12000"] = dict(
-        step="fftconv_long_fwd (arbitrary filter as long as the clip, 8192-blocks, fp32)", step_ms=ms,
+        step="fftconv_long_fwd (arbitrary filter as long as the clip, four-step FFT, fp32)", step_ms=ms,
         value=units / (ms / 1e3), unit="conv elements/s",
         roofline=hbm_roof("the whole long-convolution call", units * 8 + H * L * 4, ms,
                           "u read + y written (fp32) + fp32 filter read"),

@@ -1,28 +1,33 @@
 // Causal convolution with an arbitrary real filter as long as the input
-// (L up to 65536, any length), built from block convolutions of length T = 8192.
+// (8192 < L <= 65536, any length), as one zero-padded FFT convolution per row.
 //
 // H3 summary, appendix F "Raw speech and EEG": long convolutions over
 // 12,000-step EEG clips; §2 "Convolutional view": y = f * u + D u with the
-// causal crop of the zero-padded (linear) convolution.  A length-2L transform
-// of L > 8192 does not fit one SM's shared memory in fp32, so the row is cut
-// into K = ceil(L / T) blocks u_i and the filter into blocks f_j, and
-//   y_m = sum_{i + j = m} low(u_i, f_j) + sum_{i + j = m - 1} high(u_i, f_j)
-// where low(a, b) = causal(a, b) (the first T outputs of the linear
-// convolution a * b) and high(a, b)[t] = (a * b)[T + t] (t < T - 1, and 0 at
-// t = T - 1).  With ra, rb the blocks reversed in time,
-//   high(a, b)[t] = causal(ra, rb)[T - 2 - t],
-// so both parts come from the same fused chunk-convolution kernel
-// (launch_fftconv with K chunks of T per row, fp32 I/O): for each filter
-// block j one launch over all input blocks for the low parts and one over
-// the reversed blocks for the high parts, accumulated in fp32, then
-// y = acc + D u rounded once to the I/O type.
+// causal crop of the zero-padded (linear) convolution.  The transform length
+// M = 2^ceil(log2(2L - 1)) (32768 .. 131072) does not fit one SM's shared
+// memory in fp32, so it is split four-step: M = M1 x M2 with M2 = 256 and
+// M1 = M / 256, n = n1 + M1 n2, k = M2 k1 + k2 (n1, k1 < M1; n2, k2 < M2),
+//   X[M2 k1 + k2] = sum_n1 w_M1^(n1 k1) [ w_M^(n1 k2) sum_n2 w_M2^(n2 k2) x[n1 + M1 n2] ].
+// Three passes per pair of rows (two real rows packed as u0 + i u1; f is
+// real, so the real and imaginary outputs are the two convolutions), with
+// the spectrum in fp32 global memory between them:
+//   pass 1  per n1: the M2-point DFT over n2, then the twiddle w_M^(n1 k2)
+//   pass 2  per k2: the M1-point DFT over n1, the product with F^ / M, the
+//           inverse M1-point DFT and the conjugate twiddle
+//   pass 3  per n1: the inverse M2-point DFT, the crop to n < L, + D u
+// F^ comes from passes 1 and 2 run on the filter once per channel.  Every DFT
+// is the register/shared-memory Stockham FFT of fft_stockham.cuh, one group of
+// TG threads per sequence; each pass stages its tile through shared memory so
+// that global reads and writes run along the contiguous index.
+#include "fftconv_impl.cuh"
 #include "kernels.cuh"
 
 namespace fc {
 
 namespace {
-constexpr int kBT = 8192;  // block length
+constexpr int kLM2 = 8, kM2 = 1 << kLM2;  // inner DFT length
 constexpr int kThr = 256;
+constexpr int kNB = 16;                   // n1 values per CTA in passes 1 and 3 (one per thread group)
 
 template <typename T> __device__ __forceinline__ float ld_io(const T* p) { return (float)*p; }
 template <> __device__ __forceinline__ float ld_io<__half>(const __half* p) { return __half2float(*p); }
@@ -31,126 +36,296 @@ template <typename T> __device__ __forceinline__ T st_io(float v) { return (T)v;
 template <> __device__ __forceinline__ __half st_io<__half>(float v) { return __float2half_rn(v); }
 template <> __device__ __forceinline__ __nv_bfloat16 st_io<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
 
-// U[r][t] = u[r][t] (0 for t >= L), Ur = the same with every block reversed; rows of K T floats.
-template <typename T>
-__global__ void __launch_bounds__(kThr) lc_stage_u(const T* __restrict__ u, float* __restrict__ U,
-                                                   float* __restrict__ Ur, long long rows, int L, int K) {
-  const long long KT = (long long)K * kBT;
-  for (long long e = blockIdx.x * (long long)kThr + threadIdx.x; e < rows * KT; e += (long long)gridDim.x * kThr) {
-    const long long r = e / KT;
-    const int t = (int)(e - r * KT);
-    const float v = t < L ? ld_io(u + r * L + t) : 0.f;
-    const int i = t / kBT, p = t - i * kBT;
-    U[e] = v;
-    Ur[r * KT + (long long)i * kBT + (kBT - 1 - p)] = v;
+// w_M^(-t) = exp(-2 pi i t / M) for an exact integer t (reduced mod M by the caller)
+__device__ __forceinline__ float2 tw_exact(long long t, int M) {
+  float s, c;
+  sincospif(-2.0f * (float)t / (float)M, &s, &c);
+  return make_float2(c, s);
+}
+
+template <int LOGN>
+struct Grp {  // one length-N sequence per group of TG threads
+  using P = FftPlan<LOGN>;
+  static constexpr int N = P::M, TG = P::TG, R0 = P::R0, RL = P::RLAST, RM = P::RMAX;
+  static constexpr int G = kThr / TG;                       // sequences per CTA
+  static constexpr int SH = ILog2<R0>::v;
+  static constexpr int BUF = N + (N >> SH);
+  static constexpr int PER0 = RM / R0, PER_L = RM / RL;
+  // row stride (in float2) of a [position][G] staging tile: with G + 32 / TG
+  // the 32 lanes of a warp (32 / TG sequences x TG positions) spread evenly
+  // over the shared-memory banks
+  static constexpr int TS = G + 32 / TG;
+};
+
+template <int LOGN>
+__device__ __forceinline__ void fill_twiddles(float2* tw, int tid) {
+  using P = FftPlan<LOGN>;
+  for (int j = tid; j < P::TWN; j += kThr) {
+    float sn, cs;
+    sincospif(-2.0f * (float)j / (float)P::M, &sn, &cs);
+    tw[j] = make_float2(cs, sn);
   }
 }
 
-// F[j][h][p] = f[h][j T + p] (0 past L), Fr[j][h] = F[j][h] reversed.
-__global__ void __launch_bounds__(kThr) lc_stage_f(const float* __restrict__ f, float* __restrict__ F,
-                                                   float* __restrict__ Fr, int H, int L, int K) {
-  const long long n = (long long)K * H * kBT;
-  for (long long e = blockIdx.x * (long long)kThr + threadIdx.x; e < n; e += (long long)gridDim.x * kThr) {
-    const long long jh = e / kBT;
-    const int p = (int)(e - jh * kBT);
-    const int j = (int)(jh / H), h = (int)(jh - (long long)j * H);
-    const int t = j * kBT + p;
-    const float v = t < L ? f[(long long)h * L + t] : 0.f;
-    F[e] = v;
-    Fr[jh * kBT + (kBT - 1 - p)] = v;
+// Row q of channel h in a B x H x L array.
+__device__ __forceinline__ size_t row_of(int b, int h, int H, int L) { return ((size_t)b * H + h) * (size_t)L; }
+
+}  // namespace
+
+// ---------------------------------------------------------------- pass 1
+// grid (M1 / kNB, pairs): CTA = 16 consecutive n1 of one row pair (or, with
+// f != nullptr, of one channel's filter).  Y[pair][n1][k2] = w_M^(n1 k2) DFT_M2(x[n1 + M1 n2]).
+template <typename T, int LOGM1>
+__global__ void __launch_bounds__(kThr) lc_pass1(const T* __restrict__ u, const float* __restrict__ f,
+                                                 float2* __restrict__ Y, int B, int H, int L, int p0) {
+  using G2 = Grp<kLM2>;
+  static_assert(G2::G == kNB, "one thread group per n1 of the CTA");
+  constexpr int M1 = 1 << LOGM1, M = M1 * kM2;
+  extern __shared__ float2 lsm[];
+  float2* tile = lsm;                        // [n2][TS]
+  float2* gbuf = tile + kM2 * G2::TS;        // per group FFT buffers
+  float2* tw = gbuf + G2::G * G2::BUF;
+  const int tid = threadIdx.x, g = tid / G2::TG, tg = tid - g * G2::TG;
+  const int n10 = blockIdx.x * kNB, p = p0 + (int)blockIdx.y;
+  fill_twiddles<kLM2>(tw, tid);
+  // the two real rows of the pair (channel h, batches 2 bp and 2 bp + 1), or the filter
+  const float* fr = nullptr;
+  const T* u0 = nullptr;
+  const T* u1 = nullptr;
+  if (f) {
+    fr = f + (size_t)p * L;
+  } else {
+    const int nbp = (B + 1) / 2, h = p / nbp, bp = p - h * nbp;
+    u0 = u + row_of(2 * bp, h, H, L);
+    if (2 * bp + 1 < B) u1 = u + row_of(2 * bp + 1, h, H, L);
   }
+  for (int idx = tid; idx < kM2 * kNB; idx += kThr) {
+    const int n2 = idx / kNB, c = idx - n2 * kNB;
+    const long long n = (long long)(n10 + c) + (long long)M1 * n2;
+    float2 v = make_float2(0.f, 0.f);
+    if (n < L) {
+      if (fr) {
+        v.x = fr[n];
+      } else {
+        v.x = ld_io(u0 + n);
+        if (u1) v.y = ld_io(u1 + n);
+      }
+    }
+    tile[n2 * G2::TS + c] = v;
+  }
+  __syncthreads();
+  float2 v[G2::RM];
+#pragma unroll
+  for (int i = 0; i < G2::PER0; ++i)
+#pragma unroll
+    for (int r = 0; r < G2::R0; ++r) v[i * G2::R0 + r] = tile[(tg + i * G2::TG + r * (kM2 / G2::R0)) * G2::TS + g];
+  fft_fwd<kLM2>(v, gbuf + g * G2::BUF, tg, tw);
+  // v[i RL + r] = bin k2 = j + r M2 / RL, j = tg + i TG; twiddle and store row n1 of Y
+  const int n1 = n10 + g;
+  float2* yrow = Y + ((size_t)p * M1 + n1) * kM2;
+#pragma unroll
+  for (int i = 0; i < G2::PER_L; ++i)
+#pragma unroll
+    for (int r = 0; r < G2::RL; ++r) {
+      const int k2 = tg + i * G2::TG + r * (kM2 / G2::RL);
+      const float2 w = tw_exact(((long long)n1 * k2) & (M - 1), M);
+      yrow[k2] = cmul(v[i * G2::RL + r], w);
+    }
 }
 
-// acc block i + j (+1 for the high parts) += the block-i result of filter block j.
-__global__ void __launch_bounds__(kThr) lc_accumulate(float* __restrict__ acc, const float* __restrict__ tmp,
-                                                      long long rows, int K, int j, int high) {
-  const long long KT = (long long)K * kBT;
-  for (long long e = blockIdx.x * (long long)kThr + threadIdx.x; e < rows * KT; e += (long long)gridDim.x * kThr) {
-    const long long r = e / KT;
-    const int t = (int)(e - r * KT);
-    const int m = t / kBT, p = t - m * kBT;  // destination block and position
-    const int i = m - j - high;              // source block
-    if (i < 0) continue;
-    if (!high) {
-      acc[e] += tmp[r * KT + (long long)i * kBT + p];
-    } else if (p <= kBT - 2) {
-      acc[e] += tmp[r * KT + (long long)i * kBT + (kBT - 2 - p)];
+// ---------------------------------------------------------------- pass 2
+// grid (M2 / G1, pairs): CTA = G1 consecutive k2 of one row pair.  SPECTRUM:
+// the forward M1-point DFT of the filter's pass-1 output, written as
+// Fs[h][k2][k1] = X[M2 k1 + k2] / M.  Otherwise: forward DFT, product with
+// Fs of the pair's channel, inverse DFT, conjugate twiddle, back into Y.
+template <int LOGM1, bool SPECTRUM>
+__global__ void __launch_bounds__(kThr) lc_pass2(float2* __restrict__ Y, float2* __restrict__ Fs, int B, int p0,
+                                                 int conj_filter) {
+  using G1 = Grp<LOGM1>;
+  constexpr int M1 = 1 << LOGM1, M = M1 * kM2, GK = G1::G;
+  extern __shared__ float2 lsm[];
+  float2* tile = lsm;                        // [n1][TS]
+  float2* gbuf = tile + M1 * G1::TS;
+  float2* tw = gbuf + G1::G * G1::BUF;
+  const int tid = threadIdx.x, g = tid / G1::TG, tg = tid - g * G1::TG;
+  const int k20 = blockIdx.x * GK, p = p0 + (int)blockIdx.y;
+  fill_twiddles<LOGM1>(tw, tid);
+  float2* yp = Y + (size_t)p * M1 * kM2;
+  for (int idx = tid; idx < M1 * GK; idx += kThr) {
+    const int n1 = idx / GK, c = idx - n1 * GK;
+    tile[n1 * G1::TS + c] = yp[(size_t)n1 * kM2 + k20 + c];
+  }
+  __syncthreads();
+  float2 v[G1::RM];
+#pragma unroll
+  for (int i = 0; i < G1::PER0; ++i)
+#pragma unroll
+    for (int r = 0; r < G1::R0; ++r) v[i * G1::R0 + r] = tile[(tg + i * G1::TG + r * (M1 / G1::R0)) * G1::TS + g];
+  fft_fwd<LOGM1>(v, gbuf + g * G1::BUF, tg, tw);
+  const int k2 = k20 + g;
+  if constexpr (SPECTRUM) {
+    // v[i RL + r] = X[M2 k1 + k2], k1 = j + r M1 / RL
+    float2* fs = Fs + ((size_t)p * kM2 + k2) * M1;
+    constexpr float inv_m = 1.0f / (float)M;
+#pragma unroll
+    for (int i = 0; i < G1::PER_L; ++i)
+#pragma unroll
+      for (int r = 0; r < G1::RL; ++r) {
+        const int k1 = tg + i * G1::TG + r * (M1 / G1::RL);
+        fs[k1] = make_float2(v[i * G1::RL + r].x * inv_m, v[i * G1::RL + r].y * inv_m);
+      }
+  } else {
+    const int nbp = (B + 1) / 2, h = p / nbp;
+    const float2* fs = Fs + ((size_t)h * kM2 + k2) * M1;
+    const float sgn = conj_filter ? -1.f : 1.f;
+#pragma unroll
+    for (int i = 0; i < G1::PER_L; ++i)
+#pragma unroll
+      for (int r = 0; r < G1::RL; ++r) {
+        const int k1 = tg + i * G1::TG + r * (M1 / G1::RL);
+        const float2 F = fs[k1];
+        v[i * G1::RL + r] = cmul(v[i * G1::RL + r], make_float2(F.x, sgn * F.y));
+      }
+    __syncthreads();  // every group is past its forward transform (gbuf reuse in the inverse)
+    fft_inv<LOGM1>(v, gbuf + g * G1::BUF, tg, tw);
+    // v[i R0 + r] = n1 = j + r M1 / R0: conjugate twiddle, then back through the tile
+#pragma unroll
+    for (int i = 0; i < G1::PER0; ++i)
+#pragma unroll
+      for (int r = 0; r < G1::R0; ++r) {
+        const int n1 = tg + i * G1::TG + r * (M1 / G1::R0);
+        const float2 w = tw_exact(((long long)n1 * k2) & (M - 1), M);
+        tile[n1 * G1::TS + g] = cmul(v[i * G1::R0 + r], cconj(w));
+      }
+    __syncthreads();
+    for (int idx = tid; idx < M1 * GK; idx += kThr) {
+      const int n1 = idx / GK, c = idx - n1 * GK;
+      yp[(size_t)n1 * kM2 + k20 + c] = tile[n1 * G1::TS + c];
     }
   }
 }
 
-template <typename T>
-__global__ void __launch_bounds__(kThr) lc_finalize(const float* __restrict__ acc, const T* __restrict__ u,
-                                                    const float* __restrict__ D, T* __restrict__ y, long long rows,
-                                                    int H, int L, int K) {
-  const long long KT = (long long)K * kBT;
-  for (long long e = blockIdx.x * (long long)kThr + threadIdx.x; e < rows * L; e += (long long)gridDim.x * kThr) {
-    const long long r = e / L;
-    const int t = (int)(e - r * L);
-    const int h = (int)(r % H);
-    y[e] = st_io<T>(acc[r * KT + t] + D[h] * ld_io(u + e));
+// ---------------------------------------------------------------- pass 3
+// grid (M1 / kNB, pairs): CTA = 16 consecutive n1 of one row pair.  The
+// inverse M2-point DFT of Y'[n1][.] gives x[n1 + M1 n2]; rows n < L are
+// stored with + D u.
+template <typename T, int LOGM1>
+__global__ void __launch_bounds__(kThr) lc_pass3(const float2* __restrict__ Y, const T* __restrict__ u,
+                                                 const float* __restrict__ D, T* __restrict__ y, int B, int H,
+                                                 int L, int p0) {
+  using G2 = Grp<kLM2>;
+  constexpr int M1 = 1 << LOGM1;
+  extern __shared__ float2 lsm[];
+  float2* tile = lsm;                        // [n2][TS]
+  float2* gbuf = tile + kM2 * G2::TS;
+  float2* tw = gbuf + G2::G * G2::BUF;
+  const int tid = threadIdx.x, g = tid / G2::TG, tg = tid - g * G2::TG;
+  const int n10 = blockIdx.x * kNB, p = p0 + (int)blockIdx.y;
+  fill_twiddles<kLM2>(tw, tid);
+  __syncthreads();
+  const int n1 = n10 + g;
+  const float2* yrow = Y + ((size_t)p * M1 + n1) * kM2;
+  float2 v[G2::RM];
+  // input in the forward's last-stage layout: v[i RL + r] = k2 = j + r M2 / RL
+#pragma unroll
+  for (int i = 0; i < G2::PER_L; ++i)
+#pragma unroll
+    for (int r = 0; r < G2::RL; ++r) v[i * G2::RL + r] = yrow[tg + i * G2::TG + r * (kM2 / G2::RL)];
+  fft_inv<kLM2>(v, gbuf + g * G2::BUF, tg, tw);
+#pragma unroll
+  for (int i = 0; i < G2::PER0; ++i)
+#pragma unroll
+    for (int r = 0; r < G2::R0; ++r) tile[(tg + i * G2::TG + r * (kM2 / G2::R0)) * G2::TS + g] = v[i * G2::R0 + r];
+  __syncthreads();
+  const int nbp = (B + 1) / 2, h = p / nbp, bp = p - h * nbp;
+  const size_t r0 = row_of(2 * bp, h, H, L);
+  const bool has1 = 2 * bp + 1 < B;
+  const size_t r1 = has1 ? row_of(2 * bp + 1, h, H, L) : r0;
+  const float dh = D[h];
+  for (int idx = tid; idx < kM2 * kNB; idx += kThr) {
+    const int n2 = idx / kNB, c = idx - n2 * kNB;
+    const long long n = (long long)(n10 + c) + (long long)M1 * n2;
+    if (n < L) {
+      const float2 z = tile[n2 * G2::TS + c];
+      y[r0 + n] = st_io<T>(fmaf(dh, ld_io(u + r0 + n), z.x));
+      if (has1) y[r1 + n] = st_io<T>(fmaf(dh, ld_io(u + r1 + n), z.y));
+    }
   }
+}
+
+namespace {
+template <int LOGN>
+constexpr size_t pass_smem(int tile_rows) {
+  return sizeof(float2) * ((size_t)tile_rows * Grp<LOGN>::TS + (size_t)Grp<LOGN>::G * Grp<LOGN>::BUF +
+                           (size_t)FftPlan<LOGN>::TWN);
 }
 
 size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
 
-int grid_for(long long n) {
-  const long long g = (n + kThr - 1) / kThr;
-  const long long cap = (long long)num_sms() * 16;
-  return (int)(g < cap ? g : cap);
+int log2_transform(int L) {  // M = 2^m >= 2L - 1
+  int m = 0;
+  while ((1LL << m) < 2LL * L - 1) ++m;
+  return m;
+}
+
+template <typename T, int LOGM1>
+cudaError_t long_conv_t(const void* u, const float* f, const float* D, void* y, int B, int H, int L, char* ws,
+                        cudaStream_t st) {
+  constexpr int M1 = 1 << LOGM1, M = M1 * kM2;
+  const long long pairs = (long long)H * ((B + 1) / 2);
+  float2* Y = reinterpret_cast<float2*>(ws);
+  float2* Fs = reinterpret_cast<float2*>(ws + round256((size_t)pairs * M * sizeof(float2)));
+  constexpr size_t s13 = pass_smem<kLM2>(kM2);
+  constexpr size_t s2 = pass_smem<LOGM1>(M1);
+  cudaError_t e;
+  if ((e = smem_optin<lc_pass1<T, LOGM1>>(s13)) != cudaSuccess) return e;
+  if ((e = smem_optin<lc_pass1<float, LOGM1>>(s13)) != cudaSuccess) return e;
+  if ((e = smem_optin<lc_pass2<LOGM1, true>>(s2)) != cudaSuccess) return e;
+  if ((e = smem_optin<lc_pass2<LOGM1, false>>(s2)) != cudaSuccess) return e;
+  if ((e = smem_optin<lc_pass3<T, LOGM1>>(s13)) != cudaSuccess) return e;
+  const unsigned g13 = M1 / kNB, g2 = kM2 / Grp<LOGM1>::G;
+  // filter spectra (H "pairs" of the filter rows), through the Y area
+  for (long long c0 = 0; c0 < H; c0 += 65535) {
+    const unsigned n = (unsigned)std::min<long long>(65535, H - c0);
+    lc_pass1<float, LOGM1><<<dim3(g13, n), kThr, s13, st>>>(nullptr, f, Y, B, H, L, (int)c0);
+    lc_pass2<LOGM1, true><<<dim3(g2, n), kThr, s2, st>>>(Y, Fs, B, (int)c0, 0);
+  }
+  for (long long c0 = 0; c0 < pairs; c0 += 65535) {
+    const unsigned n = (unsigned)std::min<long long>(65535, pairs - c0);
+    lc_pass1<T, LOGM1><<<dim3(g13, n), kThr, s13, st>>>((const T*)u, nullptr, Y, B, H, L, (int)c0);
+    lc_pass2<LOGM1, false><<<dim3(g2, n), kThr, s2, st>>>(Y, Fs, B, (int)c0, 0);
+    lc_pass3<T, LOGM1><<<dim3(g13, n), kThr, s13, st>>>(Y, (const T*)u, D, (T*)y, B, H, L, (int)c0);
+  }
+  return cudaGetLastError();
 }
 
 template <typename T>
-cudaError_t long_conv_t(const void* u, const float* f, const float* D, void* y, int B, int H, int L, char* ws,
-                        int dtype, cudaStream_t st) {
-  const int K = (L + kBT - 1) / kBT;
-  const long long rows = (long long)B * H, KT = (long long)K * kBT;
-  const size_t row_bytes = round256((size_t)rows * KT * sizeof(float));
-  const size_t fil_bytes = round256((size_t)K * H * kBT * sizeof(float));
-  float* U = (float*)ws;
-  float* Ur = (float*)(ws + row_bytes);
-  float* tmp = (float*)(ws + 2 * row_bytes);
-  float* acc = (float*)(ws + 3 * row_bytes);
-  float* F = (float*)(ws + 4 * row_bytes);
-  float* Fr = (float*)(ws + 4 * row_bytes + fil_bytes);
-  float* zeroD = (float*)(ws + 4 * row_bytes + 2 * fil_bytes);
-  cudaError_t e;
-  if ((e = cudaMemsetAsync(acc, 0, (size_t)rows * KT * sizeof(float), st)) != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(zeroD, 0, (size_t)H * sizeof(float), st)) != cudaSuccess) return e;
-  lc_stage_u<T><<<grid_for(rows * KT), kThr, 0, st>>>((const T*)u, U, Ur, rows, L, K);
-  lc_stage_f<<<grid_for((long long)K * H * kBT), kThr, 0, st>>>(f, F, Fr, H, L, K);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const SsmArgs none{nullptr, nullptr, nullptr, nullptr, 0};
-  for (int j = 0; j < K; ++j) {
-    for (int high = 0; high < 2; ++high) {
-      if (high && j + 1 >= K) continue;  // the high parts of filter block j land in blocks >= j + 1
-      e = launch_fftconv(high ? Ur : U, (high ? Fr : F) + (size_t)j * H * kBT, kBT, none, zeroD, tmp, B, H, KT, kBT,
-                         K, /*dtype=*/0, st);
-      if (e != cudaSuccess) return e;
-      lc_accumulate<<<grid_for(rows * KT), kThr, 0, st>>>(acc, tmp, rows, K, j, high);
-      if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
+cudaError_t long_conv_m(const void* u, const float* f, const float* D, void* y, int B, int H, int L, char* ws,
+                        cudaStream_t st) {
+  switch (log2_transform(L) - kLM2) {
+    case 7: return long_conv_t<T, 7>(u, f, D, y, B, H, L, ws, st);
+    case 8: return long_conv_t<T, 8>(u, f, D, y, B, H, L, ws, st);
+    case 9: return long_conv_t<T, 9>(u, f, D, y, B, H, L, ws, st);
+    default: return cudaErrorInvalidValue;
   }
-  lc_finalize<T><<<grid_for(rows * L), kThr, 0, st>>>(acc, (const T*)u, D, (T*)y, rows, H, L, K);
-  (void)dtype;
-  return cudaGetLastError();
 }
 }  // namespace
 
+// [Y: pairs x M complex][Fs: H x M complex], 256-aligned; 0 for L outside (8192, 65536]
 size_t fftconv_long_workspace_bytes(int B, int H, int L) {
-  const int K = (L + kBT - 1) / kBT;
-  const long long rows = (long long)B * H, KT = (long long)K * kBT;
-  return 4 * round256((size_t)rows * KT * sizeof(float)) + 2 * round256((size_t)K * H * kBT * sizeof(float)) +
-         round256((size_t)H * sizeof(float));
+  if (B < 1 || H < 1 || L <= 8192 || L > 65536) return 0;
+  const size_t M = (size_t)1 << log2_transform(L);
+  const size_t pairs = (size_t)H * (size_t)((B + 1) / 2);
+  return round256(pairs * M * sizeof(float2)) + round256((size_t)H * M * sizeof(float2));
 }
 
 cudaError_t launch_fftconv_long(const void* u, const float* f, const float* D, void* y, int B, int H, int L,
                                 void* workspace, int dtype, cudaStream_t st) {
   char* ws = (char*)workspace;
   switch (dtype) {
-    case 0: return long_conv_t<float>(u, f, D, y, B, H, L, ws, dtype, st);
-    case 1: return long_conv_t<__half>(u, f, D, y, B, H, L, ws, dtype, st);
-    default: return long_conv_t<__nv_bfloat16>(u, f, D, y, B, H, L, ws, dtype, st);
+    case 0: return long_conv_m<float>(u, f, D, y, B, H, L, ws, st);
+    case 1: return long_conv_m<__half>(u, f, D, y, B, H, L, ws, st);
+    default: return long_conv_m<__nv_bfloat16>(u, f, D, y, B, H, L, ws, st);
   }
 }
 

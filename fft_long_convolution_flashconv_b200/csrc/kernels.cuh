@@ -105,8 +105,8 @@ cudaError_t launch_fftconv_tcl(const void* u, const float* f, int fstride, const
 unsigned int fftconv_tcl_timeouts();
 
 // Causal convolution with an arbitrary filter for L > 8192 (any length up to
-// 65536) from block convolutions of length 8192 (fftconv_long.cu); the
-// workspace holds four fp32 row buffers and the filter blocks.
+// 65536) as one four-step FFT convolution per row pair (fftconv_long.cu); the
+// workspace holds the row-pair and filter spectra in complex fp32.
 size_t fftconv_long_workspace_bytes(int B, int H, int L);
 cudaError_t launch_fftconv_long(const void* u, const float* f, const float* D, void* y, int B, int H, int L,
                                 void* workspace, int dtype, cudaStream_t st);

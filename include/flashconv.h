@@ -126,10 +126,11 @@ FC_API fc_status fftconv_fwd(const void* u, const float* f, const float* D, void
                              int B, int H, int L, fc_dtype dtype, void* stream);
 
 /* fftconv_long_workspace -- device workspace bytes fftconv_long_fwd needs
- * for L > 8192: four float32 buffers of B x H x K*8192 values and two of
- * K x H x 8192 filter values plus H floats (K = ceil(L / 8192)), each rounded
- * up to 256 bytes.  Returns 0 when no workspace is used (L <= 8192) and for
- * arguments the call would reject (B, H < 1, L > 65536). */
+ * for L > 8192: the complex float32 spectra of H * ceil(B / 2) row pairs
+ * and of the H filters at the transform length M = 2^ceil(log2(2L - 1)),
+ * i.e. 8 M (H ceil(B / 2) + H) bytes, each part rounded up to 256 bytes.
+ * Returns 0 when no workspace is used (L <= 8192) and for arguments the call
+ * would reject (B, H < 1, L > 65536). */
 FC_API size_t fftconv_long_workspace(int B, int H, int L);
 
 /* fftconv_long_fwd -- y = causal_conv(u, f) + D u for filters as long as the
@@ -138,14 +139,15 @@ FC_API size_t fftconv_long_workspace(int B, int H, int L);
  * EEG clips with filters as long as the clip; §2 "Convolutional view": the
  * causal crop of the linear convolution, y[t] = sum_{s<=t} f[t-s] u[s] + D u[t].
  * u, y: B x H x L in `dtype`; f: H x L floats; D: H floats.  Limits:
- * 1 <= L <= 65536 (any length); B * H * ceil(L / 8192) <= 2^26.  For
- * L <= 8192 this is fftconv_fwd (workspace unused, may be null).  For
- * L > 8192: workspace (256-byte aligned, caller-owned, >=
- * fftconv_long_workspace bytes; contents overwritten) holds the row cut into
- * K blocks of 8192; every output block is the sum of low and high halves of
- * block convolutions (block i of u with block j of f, i + j = m or m - 1;
- * high halves come from the time-reversed blocks), each run by the fused
- * float32 FFT convolution kernel, accumulated in float32.
+ * 1 <= L <= 65536 (any length); H * ceil(B / 2) <= 2^30.  For L <= 8192
+ * this is fftconv_fwd (workspace unused, may be null).  For L > 8192:
+ * workspace (256-byte aligned, caller-owned, >= fftconv_long_workspace
+ * bytes; contents overwritten) holds the spectra of one zero-padded FFT
+ * convolution per pair of rows (two real rows of a channel packed as one
+ * complex row), the M-point transform split four-step into M / 256 x 256
+ * (three passes through the workspace: 256-point DFTs with the twiddle,
+ * M / 256-point DFTs with the product by the filter spectrum and their
+ * inverses, inverse 256-point DFTs with the crop and + D u).
  * Precision: float32 arithmetic throughout, y rounded once to `dtype`.
  * Errors: as fftconv_fwd, plus FC_EINVAL for a missing, misaligned or too
  * small workspace; nothing is launched then. */

@@ -490,12 +490,13 @@ def test_fftconv_any_length(L, dtype):
 
 
 @pytest.mark.parametrize("B,H,L,dtype", [(2, 3, 12000, "f32"), (3, 2, 9001, "bf16"), (1, 2, 20000, "f16"),
-                                         (2, 2, 8193, "f32"), (1, 1, 65536, "f32")])
+                                         (2, 2, 8193, "f32"), (1, 1, 65536, "f32"), (5, 2, 40000, "f32"),
+                                         (2, 1, 32769, "bf16")])
 def test_fftconv_long_matches_oracle(B, H, L, dtype):
     """Filters as long as the input past 8192 (12,000-step EEG-clip length,
-    non-powers of two, three and eight blocks, the first length past one
-    block): block convolutions with reversed high halves, against the direct
-    fp64 convolution."""
+    non-powers of two, the first length past 8192, the maximum; transform
+    lengths 32768, 65536 and 131072, i.e. every four-step split; odd B
+    leaves a pair with one row): against the direct fp64 convolution."""
     rng = np.random.default_rng(L + B)
     u = W.round_to(rng.normal(size=(B, H, L)), dtype)
     f = W.round_to(rng.normal(size=(H, L)) * np.exp(-np.arange(L) / (L / 3.0)), "f32")  # arbitrary, long-reaching
