@@ -36,11 +36,26 @@ template <typename T> __device__ __forceinline__ T st_io(float v) { return (T)v;
 template <> __device__ __forceinline__ __half st_io<__half>(float v) { return __float2half_rn(v); }
 template <> __device__ __forceinline__ __nv_bfloat16 st_io<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
 
-// w_M^(-t) = exp(-2 pi i t / M) for an exact integer t (reduced mod M by the caller)
-__device__ __forceinline__ float2 tw_exact(long long t, int M) {
-  float s, c;
-  sincospif(-2.0f * (float)t / (float)M, &s, &c);
-  return make_float2(c, s);
+// The four-step twiddle w_M^(n1 k2) (n1 < M1, k2 < 256, so n1 k2 < M needs no
+// reduction) as the product of two table entries: with t = 256 a + b,
+// w_M^t = w_M1^a w_M^b.  hi[a] = w_M1^a (M1 entries), lo[b] = w_M^b (256).
+template <int LOGM1>
+__device__ __forceinline__ void fill_step_twiddles(float2* hi, float2* lo, int tid) {
+  constexpr int M1 = 1 << LOGM1, M = M1 * kM2;
+  for (int j = tid; j < M1 + kM2; j += kThr) {
+    float sn, cs;
+    if (j < M1) {
+      sincospif(-2.0f * (float)j / (float)M1, &sn, &cs);
+      hi[j] = make_float2(cs, sn);
+    } else {
+      sincospif(-2.0f * (float)(j - M1) / (float)M, &sn, &cs);
+      lo[j - M1] = make_float2(cs, sn);
+    }
+  }
+}
+__device__ __forceinline__ float2 step_twiddle(const float2* hi, const float2* lo, int n1, int k2) {
+  const int t = n1 * k2;
+  return cmul(hi[t >> kLM2], lo[t & (kM2 - 1)]);
 }
 
 template <int LOGN>
@@ -55,6 +70,13 @@ struct Grp {  // one length-N sequence per group of TG threads
   // the 32 lanes of a warp (32 / TG sequences x TG positions) spread evenly
   // over the shared-memory banks
   static constexpr int TS = G + 32 / TG;
+  // a staging tile of `rows` positions and the group FFT buffers share one
+  // region: the tile is read into registers before the first buffer store
+  // (after a CTA barrier inside the transform) and written only after a
+  // barrier that follows the last buffer load
+  static constexpr size_t region(int rows) {
+    return (size_t)rows * TS > (size_t)G * BUF ? (size_t)rows * TS : (size_t)G * BUF;
+  }
 };
 
 template <int LOGN>
@@ -80,14 +102,17 @@ __global__ void __launch_bounds__(kThr) lc_pass1(const T* __restrict__ u, const 
                                                  float2* __restrict__ Y, int B, int H, int L, int p0) {
   using G2 = Grp<kLM2>;
   static_assert(G2::G == kNB, "one thread group per n1 of the CTA");
-  constexpr int M1 = 1 << LOGM1, M = M1 * kM2;
+  constexpr int M1 = 1 << LOGM1;
   extern __shared__ float2 lsm[];
   float2* tile = lsm;                        // [n2][TS]
-  float2* gbuf = tile + kM2 * G2::TS;        // per group FFT buffers
-  float2* tw = gbuf + G2::G * G2::BUF;
+  float2* gbuf = lsm;                        // per group FFT buffers (same region)
+  float2* tw = lsm + G2::region(kM2);
+  float2* thi = tw + FftPlan<kLM2>::TWN;     // four-step twiddle tables
+  float2* tlo = thi + M1;
   const int tid = threadIdx.x, g = tid / G2::TG, tg = tid - g * G2::TG;
   const int n10 = blockIdx.x * kNB, p = p0 + (int)blockIdx.y;
   fill_twiddles<kLM2>(tw, tid);
+  fill_step_twiddles<LOGM1>(thi, tlo, tid);
   // the two real rows of the pair (channel h, batches 2 bp and 2 bp + 1), or the filter
   const float* fr = nullptr;
   const T* u0 = nullptr;
@@ -128,8 +153,7 @@ __global__ void __launch_bounds__(kThr) lc_pass1(const T* __restrict__ u, const 
 #pragma unroll
     for (int r = 0; r < G2::RL; ++r) {
       const int k2 = tg + i * G2::TG + r * (kM2 / G2::RL);
-      const float2 w = tw_exact(((long long)n1 * k2) & (M - 1), M);
-      yrow[k2] = cmul(v[i * G2::RL + r], w);
+      yrow[k2] = cmul(v[i * G2::RL + r], step_twiddle(thi, tlo, n1, k2));
     }
 }
 
@@ -145,11 +169,14 @@ __global__ void __launch_bounds__(kThr) lc_pass2(float2* __restrict__ Y, float2*
   constexpr int M1 = 1 << LOGM1, M = M1 * kM2, GK = G1::G;
   extern __shared__ float2 lsm[];
   float2* tile = lsm;                        // [n1][TS]
-  float2* gbuf = tile + M1 * G1::TS;
-  float2* tw = gbuf + G1::G * G1::BUF;
+  float2* gbuf = lsm;                        // (same region)
+  float2* tw = lsm + G1::region(M1);
+  float2* thi = tw + FftPlan<LOGM1>::TWN;    // four-step twiddle tables
+  float2* tlo = thi + M1;
   const int tid = threadIdx.x, g = tid / G1::TG, tg = tid - g * G1::TG;
   const int k20 = blockIdx.x * GK, p = p0 + (int)blockIdx.y;
   fill_twiddles<LOGM1>(tw, tid);
+  if constexpr (!SPECTRUM) fill_step_twiddles<LOGM1>(thi, tlo, tid);
   float2* yp = Y + (size_t)p * M1 * kM2;
   for (int idx = tid; idx < M1 * GK; idx += kThr) {
     const int n1 = idx / GK, c = idx - n1 * GK;
@@ -188,14 +215,14 @@ __global__ void __launch_bounds__(kThr) lc_pass2(float2* __restrict__ Y, float2*
       }
     __syncthreads();  // every group is past its forward transform (gbuf reuse in the inverse)
     fft_inv<LOGM1>(v, gbuf + g * G1::BUF, tg, tw);
+    __syncthreads();  // every group is done with its buffer (the tile's region)
     // v[i R0 + r] = n1 = j + r M1 / R0: conjugate twiddle, then back through the tile
 #pragma unroll
     for (int i = 0; i < G1::PER0; ++i)
 #pragma unroll
       for (int r = 0; r < G1::R0; ++r) {
         const int n1 = tg + i * G1::TG + r * (M1 / G1::R0);
-        const float2 w = tw_exact(((long long)n1 * k2) & (M - 1), M);
-        tile[n1 * G1::TS + g] = cmul(v[i * G1::R0 + r], cconj(w));
+        tile[n1 * G1::TS + g] = cmul(v[i * G1::R0 + r], cconj(step_twiddle(thi, tlo, n1, k2)));
       }
     __syncthreads();
     for (int idx = tid; idx < M1 * GK; idx += kThr) {
@@ -217,8 +244,8 @@ __global__ void __launch_bounds__(kThr) lc_pass3(const float2* __restrict__ Y, c
   constexpr int M1 = 1 << LOGM1;
   extern __shared__ float2 lsm[];
   float2* tile = lsm;                        // [n2][TS]
-  float2* gbuf = tile + kM2 * G2::TS;
-  float2* tw = gbuf + G2::G * G2::BUF;
+  float2* gbuf = lsm;                        // (same region)
+  float2* tw = lsm + G2::region(kM2);
   const int tid = threadIdx.x, g = tid / G2::TG, tg = tid - g * G2::TG;
   const int n10 = blockIdx.x * kNB, p = p0 + (int)blockIdx.y;
   fill_twiddles<kLM2>(tw, tid);
@@ -232,6 +259,7 @@ __global__ void __launch_bounds__(kThr) lc_pass3(const float2* __restrict__ Y, c
 #pragma unroll
     for (int r = 0; r < G2::RL; ++r) v[i * G2::RL + r] = yrow[tg + i * G2::TG + r * (kM2 / G2::RL)];
   fft_inv<kLM2>(v, gbuf + g * G2::BUF, tg, tw);
+  __syncthreads();  // every group is done with its buffer (the tile's region)
 #pragma unroll
   for (int i = 0; i < G2::PER0; ++i)
 #pragma unroll
@@ -255,9 +283,8 @@ __global__ void __launch_bounds__(kThr) lc_pass3(const float2* __restrict__ Y, c
 
 namespace {
 template <int LOGN>
-constexpr size_t pass_smem(int tile_rows) {
-  return sizeof(float2) * ((size_t)tile_rows * Grp<LOGN>::TS + (size_t)Grp<LOGN>::G * Grp<LOGN>::BUF +
-                           (size_t)FftPlan<LOGN>::TWN);
+constexpr size_t pass_smem(int tile_rows, int step_tw) {
+  return sizeof(float2) * (Grp<LOGN>::region(tile_rows) + (size_t)FftPlan<LOGN>::TWN + (size_t)step_tw);
 }
 
 size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
@@ -275,8 +302,8 @@ cudaError_t long_conv_t(const void* u, const float* f, const float* D, void* y, 
   const long long pairs = (long long)H * ((B + 1) / 2);
   float2* Y = reinterpret_cast<float2*>(ws);
   float2* Fs = reinterpret_cast<float2*>(ws + round256((size_t)pairs * M * sizeof(float2)));
-  constexpr size_t s13 = pass_smem<kLM2>(kM2);
-  constexpr size_t s2 = pass_smem<LOGM1>(M1);
+  constexpr size_t s13 = pass_smem<kLM2>(kM2, M1 + kM2);
+  constexpr size_t s2 = pass_smem<LOGM1>(M1, M1 + kM2);
   cudaError_t e;
   if ((e = smem_optin<lc_pass1<T, LOGM1>>(s13)) != cudaSuccess) return e;
   if ((e = smem_optin<lc_pass1<float, LOGM1>>(s13)) != cudaSuccess) return e;
