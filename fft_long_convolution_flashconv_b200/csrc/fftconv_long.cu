@@ -158,26 +158,30 @@ __global__ void __launch_bounds__(kThr) lc_pass1(const T* __restrict__ u, const 
 }
 
 // ---------------------------------------------------------------- pass 2
-// grid (M2 / G1, pairs): CTA = G1 consecutive k2 of one row pair.  SPECTRUM:
-// the forward M1-point DFT of the filter's pass-1 output, written as
-// Fs[h][k2][k1] = X[M2 k1 + k2] / M.  Otherwise: forward DFT, product with
-// Fs of the pair's channel, inverse DFT, conjugate twiddle, back into Y.
-template <int LOGM1, bool SPECTRUM>
-__global__ void __launch_bounds__(kThr) lc_pass2(float2* __restrict__ Y, float2* __restrict__ Fs, int B, int p0,
-                                                 int conj_filter) {
+// 16-byte asynchronous global -> shared copies (two float2 at a time)
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Filter spectra: grid (M2 / G1, channels), CTA = G1 consecutive k2 of one
+// filter.  The forward M1-point DFT of the filter's pass-1 output, written as
+// Fs[h][k2][k1] = X[M2 k1 + k2] / M.
+template <int LOGM1>
+__global__ void __launch_bounds__(kThr) lc_spectrum(const float2* __restrict__ Y, float2* __restrict__ Fs, int h0) {
   using G1 = Grp<LOGM1>;
   constexpr int M1 = 1 << LOGM1, M = M1 * kM2, GK = G1::G;
   extern __shared__ float2 lsm[];
   float2* tile = lsm;                        // [n1][TS]
   float2* gbuf = lsm;                        // (same region)
   float2* tw = lsm + G1::region(M1);
-  float2* thi = tw + FftPlan<LOGM1>::TWN;    // four-step twiddle tables
-  float2* tlo = thi + M1;
   const int tid = threadIdx.x, g = tid / G1::TG, tg = tid - g * G1::TG;
-  const int k20 = blockIdx.x * GK, p = p0 + (int)blockIdx.y;
+  const int k20 = blockIdx.x * GK, h = h0 + (int)blockIdx.y;
   fill_twiddles<LOGM1>(tw, tid);
-  if constexpr (!SPECTRUM) fill_step_twiddles<LOGM1>(thi, tlo, tid);
-  float2* yp = Y + (size_t)p * M1 * kM2;
+  const float2* yp = Y + (size_t)h * M1 * kM2;
   for (int idx = tid; idx < M1 * GK; idx += kThr) {
     const int n1 = idx / GK, c = idx - n1 * GK;
     tile[n1 * G1::TS + c] = yp[(size_t)n1 * kM2 + k20 + c];
@@ -189,31 +193,93 @@ __global__ void __launch_bounds__(kThr) lc_pass2(float2* __restrict__ Y, float2*
 #pragma unroll
     for (int r = 0; r < G1::R0; ++r) v[i * G1::R0 + r] = tile[(tg + i * G1::TG + r * (M1 / G1::R0)) * G1::TS + g];
   fft_fwd<LOGM1>(v, gbuf + g * G1::BUF, tg, tw);
+  // v[i RL + r] = X[M2 k1 + k2], k1 = j + r M1 / RL
   const int k2 = k20 + g;
-  if constexpr (SPECTRUM) {
-    // v[i RL + r] = X[M2 k1 + k2], k1 = j + r M1 / RL
-    float2* fs = Fs + ((size_t)p * kM2 + k2) * M1;
-    constexpr float inv_m = 1.0f / (float)M;
+  float2* fs = Fs + ((size_t)h * kM2 + k2) * M1;
+  constexpr float inv_m = 1.0f / (float)M;
+#pragma unroll
+  for (int i = 0; i < G1::PER_L; ++i)
+#pragma unroll
+    for (int r = 0; r < G1::RL; ++r) {
+      const int k1 = tg + i * G1::TG + r * (M1 / G1::RL);
+      fs[k1] = make_float2(v[i * G1::RL + r].x * inv_m, v[i * G1::RL + r].y * inv_m);
+    }
+}
+
+// grid (M2 / G1, channels): CTA = G1 consecutive k2 of every row pair of one
+// channel h (pairs p = h ceil(B / 2) + bp).  Per pair: the forward M1-point
+// DFT over n1, the product with Fs[h], the inverse DFT, the conjugate
+// twiddle, back into Y.  The next pair's columns are copied into the second
+// staging tile while this one is transformed; the channel's spectrum slice
+// stays in registers across the pairs where it fits (M1 <= 256).
+template <int LOGM1>
+__global__ void __launch_bounds__(kThr) lc_pass2(float2* __restrict__ Y, const float2* __restrict__ Fs, int B,
+                                                 int h0, int conj_filter) {
+  using G1 = Grp<LOGM1>;
+  constexpr int M1 = 1 << LOGM1, GK = G1::G;
+  constexpr bool kFreg = G1::RM <= 16;
+  constexpr int kReg = (int)G1::region(M1);
+  extern __shared__ float2 lsm[];
+  float2* tw = lsm + 2 * kReg;               // [tile 0][tile 1][FFT twiddles][four-step tables]
+  float2* thi = tw + FftPlan<LOGM1>::TWN;
+  float2* tlo = thi + M1;
+  const int tid = threadIdx.x, g = tid / G1::TG, tg = tid - g * G1::TG;
+  const int k20 = blockIdx.x * GK, h = h0 + (int)blockIdx.y, k2 = k20 + g;
+  const int nbp = (B + 1) / 2;
+  fill_twiddles<LOGM1>(tw, tid);
+  fill_step_twiddles<LOGM1>(thi, tlo, tid);
+  auto prefetch = [&](int bp) {  // columns k20 .. k20 + GK of pair bp into tile bp % 2
+    float2* tile = lsm + (bp & 1) * kReg;
+    const float2* yp = Y + ((size_t)h * nbp + bp) * M1 * kM2 + k20;
+    for (int idx = 2 * tid; idx < M1 * GK; idx += 2 * kThr) {
+      const int n1 = idx / GK, c = idx - n1 * GK;
+      cp_async16(tile + n1 * G1::TS + c, yp + (size_t)n1 * kM2 + c);
+    }
+    cp_async_commit();
+  };
+  prefetch(0);
+  const float2* fs = Fs + ((size_t)h * kM2 + k2) * M1;
+  const float sgn = conj_filter ? -1.f : 1.f;
+  float2 F[kFreg ? G1::RM : 1];
+  if constexpr (kFreg) {
 #pragma unroll
     for (int i = 0; i < G1::PER_L; ++i)
 #pragma unroll
       for (int r = 0; r < G1::RL; ++r) {
-        const int k1 = tg + i * G1::TG + r * (M1 / G1::RL);
-        fs[k1] = make_float2(v[i * G1::RL + r].x * inv_m, v[i * G1::RL + r].y * inv_m);
+        const float2 f = fs[tg + i * G1::TG + r * (M1 / G1::RL)];
+        F[i * G1::RL + r] = make_float2(f.x, sgn * f.y);
       }
-  } else {
-    const int nbp = (B + 1) / 2, h = p / nbp;
-    const float2* fs = Fs + ((size_t)h * kM2 + k2) * M1;
-    const float sgn = conj_filter ? -1.f : 1.f;
+  }
+  for (int bp = 0; bp < nbp; ++bp) {
+    float2* tile = lsm + (bp & 1) * kReg;
+    float2* gbuf = tile;                     // the FFT buffers share the current tile's region
+    if (bp + 1 < nbp) {
+      prefetch(bp + 1);  // tile (bp + 1) % 2 was released by the barrier that ended pair bp - 1
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    float2 v[G1::RM];
+#pragma unroll
+    for (int i = 0; i < G1::PER0; ++i)
+#pragma unroll
+      for (int r = 0; r < G1::R0; ++r) v[i * G1::R0 + r] = tile[(tg + i * G1::TG + r * (M1 / G1::R0)) * G1::TS + g];
+    fft_fwd<LOGM1>(v, gbuf + g * G1::BUF, tg, tw);
 #pragma unroll
     for (int i = 0; i < G1::PER_L; ++i)
 #pragma unroll
       for (int r = 0; r < G1::RL; ++r) {
-        const int k1 = tg + i * G1::TG + r * (M1 / G1::RL);
-        const float2 F = fs[k1];
-        v[i * G1::RL + r] = cmul(v[i * G1::RL + r], make_float2(F.x, sgn * F.y));
+        float2 f;
+        if constexpr (kFreg) {
+          f = F[i * G1::RL + r];
+        } else {
+          f = fs[tg + i * G1::TG + r * (M1 / G1::RL)];
+          f.y *= sgn;
+        }
+        v[i * G1::RL + r] = cmul(v[i * G1::RL + r], f);
       }
-    __syncthreads();  // every group is past its forward transform (gbuf reuse in the inverse)
+    __syncthreads();  // every group is past its forward transform (buffer reuse in the inverse)
     fft_inv<LOGM1>(v, gbuf + g * G1::BUF, tg, tw);
     __syncthreads();  // every group is done with its buffer (the tile's region)
     // v[i R0 + r] = n1 = j + r M1 / R0: conjugate twiddle, then back through the tile
@@ -225,10 +291,12 @@ __global__ void __launch_bounds__(kThr) lc_pass2(float2* __restrict__ Y, float2*
         tile[n1 * G1::TS + g] = cmul(v[i * G1::R0 + r], cconj(step_twiddle(thi, tlo, n1, k2)));
       }
     __syncthreads();
+    float2* yp = Y + ((size_t)h * nbp + bp) * M1 * kM2 + k20;
     for (int idx = tid; idx < M1 * GK; idx += kThr) {
       const int n1 = idx / GK, c = idx - n1 * GK;
-      yp[(size_t)n1 * kM2 + k20 + c] = tile[n1 * G1::TS + c];
+      yp[(size_t)n1 * kM2 + c] = tile[n1 * G1::TS + c];
     }
+    __syncthreads();  // tile bp % 2 is free for the prefetch of pair bp + 2
   }
 }
 
@@ -303,24 +371,32 @@ cudaError_t long_conv_t(const void* u, const float* f, const float* D, void* y, 
   float2* Y = reinterpret_cast<float2*>(ws);
   float2* Fs = reinterpret_cast<float2*>(ws + round256((size_t)pairs * M * sizeof(float2)));
   constexpr size_t s13 = pass_smem<kLM2>(kM2, M1 + kM2);
-  constexpr size_t s2 = pass_smem<LOGM1>(M1, M1 + kM2);
+  constexpr size_t ssp = pass_smem<LOGM1>(M1, 0);
+  constexpr size_t s2 = sizeof(float2) * (2 * Grp<LOGM1>::region(M1) + FftPlan<LOGM1>::TWN + M1 + kM2);
   cudaError_t e;
   if ((e = smem_optin<lc_pass1<T, LOGM1>>(s13)) != cudaSuccess) return e;
   if ((e = smem_optin<lc_pass1<float, LOGM1>>(s13)) != cudaSuccess) return e;
-  if ((e = smem_optin<lc_pass2<LOGM1, true>>(s2)) != cudaSuccess) return e;
-  if ((e = smem_optin<lc_pass2<LOGM1, false>>(s2)) != cudaSuccess) return e;
+  if ((e = smem_optin<lc_spectrum<LOGM1>>(ssp)) != cudaSuccess) return e;
+  if ((e = smem_optin<lc_pass2<LOGM1>>(s2)) != cudaSuccess) return e;
   if ((e = smem_optin<lc_pass3<T, LOGM1>>(s13)) != cudaSuccess) return e;
   const unsigned g13 = M1 / kNB, g2 = kM2 / Grp<LOGM1>::G;
-  // filter spectra (H "pairs" of the filter rows), through the Y area
+  // filter spectra (pass 1 on the H filter rows, through the Y area), then
+  // passes 1 and 3 per row pair and pass 2 per channel
   for (long long c0 = 0; c0 < H; c0 += 65535) {
     const unsigned n = (unsigned)std::min<long long>(65535, H - c0);
     lc_pass1<float, LOGM1><<<dim3(g13, n), kThr, s13, st>>>(nullptr, f, Y, B, H, L, (int)c0);
-    lc_pass2<LOGM1, true><<<dim3(g2, n), kThr, s2, st>>>(Y, Fs, B, (int)c0, 0);
+    lc_spectrum<LOGM1><<<dim3(g2, n), kThr, ssp, st>>>(Y, Fs, (int)c0);
   }
   for (long long c0 = 0; c0 < pairs; c0 += 65535) {
     const unsigned n = (unsigned)std::min<long long>(65535, pairs - c0);
     lc_pass1<T, LOGM1><<<dim3(g13, n), kThr, s13, st>>>((const T*)u, nullptr, Y, B, H, L, (int)c0);
-    lc_pass2<LOGM1, false><<<dim3(g2, n), kThr, s2, st>>>(Y, Fs, B, (int)c0, 0);
+  }
+  for (long long c0 = 0; c0 < H; c0 += 65535) {
+    const unsigned n = (unsigned)std::min<long long>(65535, H - c0);
+    lc_pass2<LOGM1><<<dim3(g2, n), kThr, s2, st>>>(Y, Fs, B, (int)c0, 0);
+  }
+  for (long long c0 = 0; c0 < pairs; c0 += 65535) {
+    const unsigned n = (unsigned)std::min<long long>(65535, pairs - c0);
     lc_pass3<T, LOGM1><<<dim3(g13, n), kThr, s13, st>>>(Y, (const T*)u, D, (T*)y, B, H, L, (int)c0);
   }
   return cudaGetLastError();
