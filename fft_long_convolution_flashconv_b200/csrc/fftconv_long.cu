@@ -317,6 +317,21 @@ __global__ void __launch_bounds__(kThr) lc_pass3(const float2* __restrict__ Y, c
   const int tid = threadIdx.x, g = tid / G2::TG, tg = tid - g * G2::TG;
   const int n10 = blockIdx.x * kNB, p = p0 + (int)blockIdx.y;
   fill_twiddles<kLM2>(tw, tid);
+  // u for the D u term, loaded first so that its latency hides under the transform
+  const int nbp = (B + 1) / 2, h = p / nbp, bp = p - h * nbp;
+  const size_t r0 = row_of(2 * bp, h, H, L);
+  const bool has1 = 2 * bp + 1 < B;
+  const size_t r1 = has1 ? row_of(2 * bp + 1, h, H, L) : r0;
+  const float dh = D[h];
+  constexpr int kPer = kM2 * kNB / kThr;
+  float du0[kPer], du1[kPer];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int idx = tid + k * kThr, n2 = idx / kNB, c = idx - n2 * kNB;
+    const long long n = (long long)(n10 + c) + (long long)M1 * n2;
+    du0[k] = n < L ? dh * ld_io(u + r0 + n) : 0.f;
+    du1[k] = (has1 && n < L) ? dh * ld_io(u + r1 + n) : 0.f;
+  }
   __syncthreads();
   const int n1 = n10 + g;
   const float2* yrow = Y + ((size_t)p * M1 + n1) * kM2;
@@ -333,18 +348,14 @@ __global__ void __launch_bounds__(kThr) lc_pass3(const float2* __restrict__ Y, c
 #pragma unroll
     for (int r = 0; r < G2::R0; ++r) tile[(tg + i * G2::TG + r * (kM2 / G2::R0)) * G2::TS + g] = v[i * G2::R0 + r];
   __syncthreads();
-  const int nbp = (B + 1) / 2, h = p / nbp, bp = p - h * nbp;
-  const size_t r0 = row_of(2 * bp, h, H, L);
-  const bool has1 = 2 * bp + 1 < B;
-  const size_t r1 = has1 ? row_of(2 * bp + 1, h, H, L) : r0;
-  const float dh = D[h];
-  for (int idx = tid; idx < kM2 * kNB; idx += kThr) {
-    const int n2 = idx / kNB, c = idx - n2 * kNB;
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int idx = tid + k * kThr, n2 = idx / kNB, c = idx - n2 * kNB;
     const long long n = (long long)(n10 + c) + (long long)M1 * n2;
     if (n < L) {
       const float2 z = tile[n2 * G2::TS + c];
-      y[r0 + n] = st_io<T>(fmaf(dh, ld_io(u + r0 + n), z.x));
-      if (has1) y[r1 + n] = st_io<T>(fmaf(dh, ld_io(u + r1 + n), z.y));
+      y[r0 + n] = st_io<T>(z.x + du0[k]);
+      if (has1) y[r1 + n] = st_io<T>(z.y + du1[k]);
     }
   }
 }
