@@ -208,17 +208,20 @@ __global__ void __launch_bounds__(kThr) lc_spectrum(const float2* __restrict__ Y
 
 // grid (M2 / G1, channels): CTA = G1 consecutive k2 of every row pair of one
 // channel h (pairs p = h ceil(B / 2) + bp).  Per pair: the forward M1-point
-// DFT over n1, the product with Fs[h], the inverse DFT, the conjugate
-// twiddle, back into Y.  The next pair's columns are copied into the second
-// staging tile while this one is transformed; the channel's spectrum slice
-// stays in registers across the pairs where it fits (M1 <= 256).
+// DFT over n1, the product with the filter spectrum F^, the inverse DFT, the
+// conjugate twiddle, back into Y.  The next item's columns are copied into
+// the second staging tile while this one is transformed.  Where the
+// spectrum slice fits in registers (M1 <= 256), the CTA computes it itself
+// first, from the filter's pass-1 output Yf[h] (F^ = forward DFT / M); past
+// that it reads F^ from Fs[h][k2][k1], written by lc_spectrum.
 template <int LOGM1>
-__global__ void __launch_bounds__(kThr) lc_pass2(float2* __restrict__ Y, const float2* __restrict__ Fs, int B,
+__global__ void __launch_bounds__(kThr) lc_pass2(float2* __restrict__ Y, const float2* __restrict__ Fsrc, int B,
                                                  int h0, int conj_filter) {
   using G1 = Grp<LOGM1>;
-  constexpr int M1 = 1 << LOGM1, GK = G1::G;
+  constexpr int M1 = 1 << LOGM1, M = M1 * kM2, GK = G1::G;
   constexpr bool kFreg = G1::RM <= 16;
   constexpr int kReg = (int)G1::region(M1);
+  constexpr int q0 = kFreg ? 0 : 1;          // item 0 is the filter, items 1.. the pairs
   extern __shared__ float2 lsm[];
   float2* tw = lsm + 2 * kReg;               // [tile 0][tile 1][FFT twiddles][four-step tables]
   float2* thi = tw + FftPlan<LOGM1>::TWN;
@@ -228,33 +231,24 @@ __global__ void __launch_bounds__(kThr) lc_pass2(float2* __restrict__ Y, const f
   const int nbp = (B + 1) / 2;
   fill_twiddles<LOGM1>(tw, tid);
   fill_step_twiddles<LOGM1>(thi, tlo, tid);
-  auto prefetch = [&](int bp) {  // columns k20 .. k20 + GK of pair bp into tile bp % 2
-    float2* tile = lsm + (bp & 1) * kReg;
-    const float2* yp = Y + ((size_t)h * nbp + bp) * M1 * kM2 + k20;
+  auto prefetch = [&](int q) {  // columns k20 .. k20 + GK of item q into tile q % 2
+    float2* tile = lsm + (q & 1) * kReg;
+    const float2* yp = (q == 0 ? Fsrc + (size_t)h * M1 * kM2 : Y + ((size_t)h * nbp + (q - 1)) * M1 * kM2) + k20;
     for (int idx = 2 * tid; idx < M1 * GK; idx += 2 * kThr) {
       const int n1 = idx / GK, c = idx - n1 * GK;
       cp_async16(tile + n1 * G1::TS + c, yp + (size_t)n1 * kM2 + c);
     }
     cp_async_commit();
   };
-  prefetch(0);
-  const float2* fs = Fs + ((size_t)h * kM2 + k2) * M1;
+  prefetch(q0);
+  const float2* fs = Fsrc + ((size_t)h * kM2 + k2) * M1;  // Fs layout (kFreg false)
   const float sgn = conj_filter ? -1.f : 1.f;
   float2 F[kFreg ? G1::RM : 1];
-  if constexpr (kFreg) {
-#pragma unroll
-    for (int i = 0; i < G1::PER_L; ++i)
-#pragma unroll
-      for (int r = 0; r < G1::RL; ++r) {
-        const float2 f = fs[tg + i * G1::TG + r * (M1 / G1::RL)];
-        F[i * G1::RL + r] = make_float2(f.x, sgn * f.y);
-      }
-  }
-  for (int bp = 0; bp < nbp; ++bp) {
-    float2* tile = lsm + (bp & 1) * kReg;
+  for (int q = q0; q <= nbp; ++q) {
+    float2* tile = lsm + (q & 1) * kReg;
     float2* gbuf = tile;                     // the FFT buffers share the current tile's region
-    if (bp + 1 < nbp) {
-      prefetch(bp + 1);  // tile (bp + 1) % 2 was released by the barrier that ended pair bp - 1
+    if (q < nbp) {
+      prefetch(q + 1);  // tile (q + 1) % 2 was released by the barrier that ended item q - 1
       cp_async_wait<1>();
     } else {
       cp_async_wait<0>();
@@ -266,6 +260,15 @@ __global__ void __launch_bounds__(kThr) lc_pass2(float2* __restrict__ Y, const f
 #pragma unroll
       for (int r = 0; r < G1::R0; ++r) v[i * G1::R0 + r] = tile[(tg + i * G1::TG + r * (M1 / G1::R0)) * G1::TS + g];
     fft_fwd<LOGM1>(v, gbuf + g * G1::BUF, tg, tw);
+    if (q == 0) {  // the filter: v[i RL + r] = X[M2 k1 + k2], k1 = j + r M1 / RL
+      if constexpr (kFreg) {
+        constexpr float inv_m = 1.0f / (float)M;
+#pragma unroll
+        for (int k = 0; k < G1::RM; ++k) F[k] = make_float2(v[k].x * inv_m, sgn * v[k].y * inv_m);
+      }
+      __syncthreads();  // tile 0 is free for the prefetch of item 2
+      continue;
+    }
 #pragma unroll
     for (int i = 0; i < G1::PER_L; ++i)
 #pragma unroll
@@ -291,12 +294,12 @@ __global__ void __launch_bounds__(kThr) lc_pass2(float2* __restrict__ Y, const f
         tile[n1 * G1::TS + g] = cmul(v[i * G1::R0 + r], cconj(step_twiddle(thi, tlo, n1, k2)));
       }
     __syncthreads();
-    float2* yp = Y + ((size_t)h * nbp + bp) * M1 * kM2 + k20;
+    float2* yp = Y + ((size_t)h * nbp + (q - 1)) * M1 * kM2 + k20;
     for (int idx = tid; idx < M1 * GK; idx += kThr) {
       const int n1 = idx / GK, c = idx - n1 * GK;
       yp[(size_t)n1 * kM2 + c] = tile[n1 * G1::TS + c];
     }
-    __syncthreads();  // tile bp % 2 is free for the prefetch of pair bp + 2
+    __syncthreads();  // tile q % 2 is free for the prefetch of item q + 2
   }
 }
 
@@ -391,12 +394,14 @@ cudaError_t long_conv_t(const void* u, const float* f, const float* D, void* y, 
   if ((e = smem_optin<lc_pass2<LOGM1>>(s2)) != cudaSuccess) return e;
   if ((e = smem_optin<lc_pass3<T, LOGM1>>(s13)) != cudaSuccess) return e;
   const unsigned g13 = M1 / kNB, g2 = kM2 / Grp<LOGM1>::G;
-  // filter spectra (pass 1 on the H filter rows, through the Y area), then
+  // pass 1 on the H filter rows: into the Fs area, where pass 2 takes the
+  // spectra from (M1 <= 256), or through the Y area into lc_spectrum; then
   // passes 1 and 3 per row pair and pass 2 per channel
+  constexpr bool fused_spectrum = Grp<LOGM1>::RM <= 16;
   for (long long c0 = 0; c0 < H; c0 += 65535) {
     const unsigned n = (unsigned)std::min<long long>(65535, H - c0);
-    lc_pass1<float, LOGM1><<<dim3(g13, n), kThr, s13, st>>>(nullptr, f, Y, B, H, L, (int)c0);
-    lc_spectrum<LOGM1><<<dim3(g2, n), kThr, ssp, st>>>(Y, Fs, (int)c0);
+    lc_pass1<float, LOGM1><<<dim3(g13, n), kThr, s13, st>>>(nullptr, f, fused_spectrum ? Fs : Y, B, H, L, (int)c0);
+    if (!fused_spectrum) lc_spectrum<LOGM1><<<dim3(g2, n), kThr, ssp, st>>>(Y, Fs, (int)c0);
   }
   for (long long c0 = 0; c0 < pairs; c0 += 65535) {
     const unsigned n = (unsigned)std::min<long long>(65535, pairs - c0);
