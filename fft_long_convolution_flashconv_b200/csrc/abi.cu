@@ -165,7 +165,7 @@ FC_API fc_status fftconv_long_fwd(const void* u, const float* f, const float* D,
   FC_REQUIRE(f && D, FC_EINVAL, "null f or D");
   FC_REQUIRE(aligned(f, 16) && aligned(D, 4), FC_EINVAL, "f must be 16-byte aligned, D 4-byte aligned");
   const long long pairs = (long long)H * ((B + 1) / 2);
-  FC_REQUIRE(pairs <= (1LL << 30), FC_EUNSUPPORTED, "H * ceil(B / 2) = %lld > 2^30", pairs);
+  FC_REQUIRE(pairs <= (1LL << 29), FC_EUNSUPPORTED, "H * ceil(B / 2) = %lld > 2^29", pairs);
   FC_REQUIRE(workspace && aligned(workspace, 256), FC_EINVAL, "workspace must be non-null and 256-byte aligned");
   const size_t need = fftconv_long_workspace(B, H, L);
   FC_REQUIRE(ws_bytes >= need, FC_EINVAL, "workspace too small: %zu < %zu bytes", ws_bytes, need);

@@ -95,11 +95,13 @@ __device__ __forceinline__ size_t row_of(int b, int h, int H, int L) { return ((
 }  // namespace
 
 // ---------------------------------------------------------------- pass 1
-// grid (M1 / kNB, pairs): CTA = 16 consecutive n1 of one row pair (or, with
-// f != nullptr, of one channel's filter).  Y[pair][n1][k2] = w_M^(n1 k2) DFT_M2(x[n1 + M1 n2]).
+// grid (M1 / kNB, rows): CTA = 16 consecutive n1 of one item q = q0 +
+// blockIdx.y: the filter of channel q for q < nfr (into Yf), else row pair
+// q - nfr (into Y).  Out[item][n1][k2] = w_M^(n1 k2) DFT_M2(x[n1 + M1 n2]).
 template <typename T, int LOGM1>
 __global__ void __launch_bounds__(kThr) lc_pass1(const T* __restrict__ u, const float* __restrict__ f,
-                                                 float2* __restrict__ Y, int B, int H, int L, int p0) {
+                                                 float2* __restrict__ Y, float2* __restrict__ Yf, int B, int H,
+                                                 int L, int q0, int nfr) {
   using G2 = Grp<kLM2>;
   static_assert(G2::G == kNB, "one thread group per n1 of the CTA");
   constexpr int M1 = 1 << LOGM1;
@@ -110,14 +112,16 @@ __global__ void __launch_bounds__(kThr) lc_pass1(const T* __restrict__ u, const 
   float2* thi = tw + FftPlan<kLM2>::TWN;     // four-step twiddle tables
   float2* tlo = thi + M1;
   const int tid = threadIdx.x, g = tid / G2::TG, tg = tid - g * G2::TG;
-  const int n10 = blockIdx.x * kNB, p = p0 + (int)blockIdx.y;
+  const int n10 = blockIdx.x * kNB, q = q0 + (int)blockIdx.y;
+  const bool filt = q < nfr;
+  const int p = filt ? q : q - nfr;
   fill_twiddles<kLM2>(tw, tid);
   fill_step_twiddles<LOGM1>(thi, tlo, tid);
   // the two real rows of the pair (channel h, batches 2 bp and 2 bp + 1), or the filter
   const float* fr = nullptr;
   const T* u0 = nullptr;
   const T* u1 = nullptr;
-  if (f) {
+  if (filt) {
     fr = f + (size_t)p * L;
   } else {
     const int nbp = (B + 1) / 2, h = p / nbp, bp = p - h * nbp;
@@ -147,7 +151,7 @@ __global__ void __launch_bounds__(kThr) lc_pass1(const T* __restrict__ u, const 
   fft_fwd<kLM2>(v, gbuf + g * G2::BUF, tg, tw);
   // v[i RL + r] = bin k2 = j + r M2 / RL, j = tg + i TG; twiddle and store row n1 of Y
   const int n1 = n10 + g;
-  float2* yrow = Y + ((size_t)p * M1 + n1) * kM2;
+  float2* yrow = (filt ? Yf : Y) + ((size_t)p * M1 + n1) * kM2;
 #pragma unroll
   for (int i = 0; i < G2::PER_L; ++i)
 #pragma unroll
@@ -389,23 +393,26 @@ cudaError_t long_conv_t(const void* u, const float* f, const float* D, void* y, 
   constexpr size_t s2 = sizeof(float2) * (2 * Grp<LOGM1>::region(M1) + FftPlan<LOGM1>::TWN + M1 + kM2);
   cudaError_t e;
   if ((e = smem_optin<lc_pass1<T, LOGM1>>(s13)) != cudaSuccess) return e;
-  if ((e = smem_optin<lc_pass1<float, LOGM1>>(s13)) != cudaSuccess) return e;
   if ((e = smem_optin<lc_spectrum<LOGM1>>(ssp)) != cudaSuccess) return e;
   if ((e = smem_optin<lc_pass2<LOGM1>>(s2)) != cudaSuccess) return e;
   if ((e = smem_optin<lc_pass3<T, LOGM1>>(s13)) != cudaSuccess) return e;
   const unsigned g13 = M1 / kNB, g2 = kM2 / Grp<LOGM1>::G;
-  // pass 1 on the H filter rows: into the Fs area, where pass 2 takes the
-  // spectra from (M1 <= 256), or through the Y area into lc_spectrum; then
-  // passes 1 and 3 per row pair and pass 2 per channel
+  // pass 1 on the H filter rows and the row pairs; where pass 2 takes the
+  // spectra from the filters' pass-1 output (M1 <= 256) in one launch, the
+  // filters' output in the Fs area; otherwise the filters first, through the
+  // Y area into lc_spectrum.  Then pass 2 per channel and pass 3 per row pair.
   constexpr bool fused_spectrum = Grp<LOGM1>::RM <= 16;
-  for (long long c0 = 0; c0 < H; c0 += 65535) {
-    const unsigned n = (unsigned)std::min<long long>(65535, H - c0);
-    lc_pass1<float, LOGM1><<<dim3(g13, n), kThr, s13, st>>>(nullptr, f, fused_spectrum ? Fs : Y, B, H, L, (int)c0);
-    if (!fused_spectrum) lc_spectrum<LOGM1><<<dim3(g2, n), kThr, ssp, st>>>(Y, Fs, (int)c0);
+  const long long q_first = fused_spectrum ? 0 : H;
+  if (!fused_spectrum) {
+    for (long long c0 = 0; c0 < H; c0 += 65535) {
+      const unsigned n = (unsigned)std::min<long long>(65535, H - c0);
+      lc_pass1<T, LOGM1><<<dim3(g13, n), kThr, s13, st>>>((const T*)u, f, Y, Y, B, H, L, (int)c0, H);
+      lc_spectrum<LOGM1><<<dim3(g2, n), kThr, ssp, st>>>(Y, Fs, (int)c0);
+    }
   }
-  for (long long c0 = 0; c0 < pairs; c0 += 65535) {
-    const unsigned n = (unsigned)std::min<long long>(65535, pairs - c0);
-    lc_pass1<T, LOGM1><<<dim3(g13, n), kThr, s13, st>>>((const T*)u, nullptr, Y, B, H, L, (int)c0);
+  for (long long c0 = q_first; c0 < H + pairs; c0 += 65535) {
+    const unsigned n = (unsigned)std::min<long long>(65535, H + pairs - c0);
+    lc_pass1<T, LOGM1><<<dim3(g13, n), kThr, s13, st>>>((const T*)u, f, Y, Fs, B, H, L, (int)c0, H);
   }
   for (long long c0 = 0; c0 < H; c0 += 65535) {
     const unsigned n = (unsigned)std::min<long long>(65535, H - c0);

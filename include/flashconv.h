@@ -139,7 +139,7 @@ FC_API size_t fftconv_long_workspace(int B, int H, int L);
  * EEG clips with filters as long as the clip; §2 "Convolutional view": the
  * causal crop of the linear convolution, y[t] = sum_{s<=t} f[t-s] u[s] + D u[t].
  * u, y: B x H x L in `dtype`; f: H x L floats; D: H floats.  Limits:
- * 1 <= L <= 65536 (any length); H * ceil(B / 2) <= 2^30.  For L <= 8192
+ * 1 <= L <= 65536 (any length); H * ceil(B / 2) <= 2^29.  For L <= 8192
  * this is fftconv_fwd (workspace unused, may be null).  For L > 8192:
  * workspace (256-byte aligned, caller-owned, >= fftconv_long_workspace
  * bytes; contents overwritten) holds the spectra of one zero-padded FFT
