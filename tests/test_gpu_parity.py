@@ -506,6 +506,46 @@ def test_fftconv_long_matches_oracle(B, H, L, dtype):
     assert O.row_rel_err(y.reshape(-1, L), ref.reshape(-1, L)) < TOL[dtype]
 
 
+def test_fftconv_long_bench_size_sampled_rows():
+    """The EEG-length bench shape (B=8, H=256, L=12000, fp32) in the launch
+    configuration the bench times; sampled rows (first, last, a row whose pair
+    partner is the other half of its pair, channels at both ends) against the
+    direct fp64 convolution one row at a time."""
+    B, H, L = 8, 256, 12000
+    rng = np.random.default_rng(12000)
+    u = rng.normal(size=(B, H, L)).astype(np.float32)
+    f = (rng.normal(size=(H, L)) * np.exp(-np.arange(L) / 4000.0)).astype(np.float32)
+    D = rng.normal(size=H).astype(np.float32)
+    y = host(api.fftconv_long_fwd(dev(u), dev(f), dev(D)))
+    for b, h in [(0, 0), (1, 0), (7, 255), (6, 255), (3, 128), (4, 17)]:
+        ref = cref.causal_conv(u[b:b + 1, h:h + 1].astype(np.float64), f[h:h + 1], D[h:h + 1])
+        assert O.row_rel_err(y[b, h][None], ref.reshape(1, L)) < TOL["f32"], (b, h)
+
+
+@pytest.mark.parametrize("L", [8193, 12000, 40000, 65536])
+def test_fftconv_long_shift_filters_are_exact(L):
+    """A filter that is a unit impulse at tap s shifts the input by s: y[t] =
+    u[t - s] + D u[t] for t >= s, D u[t] before.  Taps at both ends of the
+    four-step index split (s = 0, 1, 255, 256, M1 - 1, L - 1) land on exactly the
+    right outputs; with an integer-valued u the results are exact up to the
+    fp32 rounding of the transforms."""
+    M = 1 << int(np.ceil(np.log2(2 * L - 1)))
+    M1 = M // 256
+    shifts = [0, 1, 255, 256, M1 - 1, L - 1]
+    H, B = len(shifts), 3
+    rng = np.random.default_rng(L)
+    u = rng.integers(-4, 5, size=(B, H, L)).astype(np.float32)
+    f = np.zeros((H, L), np.float32)
+    for h, s in enumerate(shifts):
+        f[h, s] = 1.0
+    D = np.full(H, 0.5, np.float32)
+    y = host(api.fftconv_long_fwd(dev(u), dev(f), dev(D)))
+    for h, s in enumerate(shifts):
+        want = 0.5 * u[:, h].astype(np.float64)
+        want[:, s:] += u[:, h, :L - s]
+        assert np.max(np.abs(y[:, h] - want)) < 1e-3, (L, s)
+
+
 def test_fftconv_long_short_lengths_are_fftconv_fwd():
     B, H, L = 3, 4, 5000
     rng = np.random.default_rng(5)
