@@ -15,10 +15,15 @@
 //   pass 2  per k2: the M1-point DFT over n1, the product with F^ / M, the
 //           inverse M1-point DFT and the conjugate twiddle
 //   pass 3  per n1: the inverse M2-point DFT, the crop to n < L, + D u
-// F^ comes from passes 1 and 2 run on the filter once per channel.  Every DFT
-// is the register/shared-memory Stockham FFT of fft_stockham.cuh, one group of
-// TG threads per sequence; each pass stages its tile through shared memory so
-// that global reads and writes run along the contiguous index.
+// F^ comes from passes 1 and 2 run on the filter once per channel: pass 1
+// takes the H filters and the row pairs in one launch, and pass 2 (one CTA per
+// block of k2 and channel, looping over the channel's pairs) first transforms
+// its slice of the filter's pass-1 output and keeps it in registers (for
+// M1 = 512 the slice does not fit, and lc_spectrum writes F^ to the workspace
+// first).  Every DFT is the register/shared-memory Stockham FFT of
+// fft_stockham.cuh, one group of TG threads per sequence; each pass stages its
+// tile through shared memory (the same region as the FFT buffers) so that
+// global reads and writes run along the contiguous index.
 #include "fftconv_impl.cuh"
 #include "kernels.cuh"
 
