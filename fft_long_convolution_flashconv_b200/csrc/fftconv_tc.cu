@@ -44,14 +44,18 @@
 //                (its filter's F^ and its pair), then the previous round's
 //                outputs of the same tuple (epilogue) from the other stage-A'
 //                accumulator;
-//   warps 12..14 bulk copies of the next round's rows and filters (one lane per
-//                warp, each with its own byte count on the copy barrier) and the
-//                stage-A operand from the staged rows;
+//   warps 12..14 bulk copies of the rows and filters two rounds ahead (two
+//                staging buffers; one lane per warp, each with its own byte
+//                count on the buffer's copy barrier) and the stage-A operand
+//                from the staged rows (two operand buffers, so the operand of
+//                round j + 1 is written while stage A of round j reads);
 //   warp 15      issues every MMA: stage A of round j + 1 as soon as its operand
 //                is written, stage A' of round j once the register pass is done.
 // Tensor memory: C, S; two stage-A accumulators and two stage-A' accumulators,
 // so stage A of the next round and stage A' of this one run under the
-// register pass.  All waits are on mbarriers with a time bound; a wait that
+// register pass.  The stage-A' operand Z has one buffer: the register pass of
+// round j writes it once stage A' of round j - 1 has completed (which the
+// epilogue of round j - 1 waits for anyway).  All waits are on mbarriers with a time bound; a wait that
 // runs out marks the CTA aborted and counts it in a device counter, after
 // which the issuing threads complete every phase by plain arrivals (no more
 // copies or MMAs), nothing is written to y, and the CTA drains its MMAs and
@@ -90,11 +94,14 @@ constexpr uint32_t kXBytes = 64 * 3 * kMaxNC * 2;           // stage-A operand [
 constexpr uint32_t kZBytes = 2 * kN1 * kN2 * kSlots * 2;    // stage-A' operand, 256 K-rows (re | im)
 // shared memory layout (bytes)
 constexpr uint32_t kOCa = 0, kOCb = kCBytes, kOTw = 2 * kCBytes;
-constexpr uint32_t kOSU = kOTw + kTwBytes;                  // staged input rows (2 per tuple)
-constexpr uint32_t kOSF = kOSU + 2 * kSlots * kRowBytes;    // staged filters
-constexpr uint32_t kOX = kOSF + kMaxF * kFBytes;
-constexpr uint32_t kOZ = kOX + kXBytes;                     // two buffers
-constexpr uint32_t kOBar = kOZ + 2 * kZBytes;               // mbarriers: tables, copies, A[2], A'[2], drain, Z[2]
+constexpr uint32_t kSUBytes = 2 * kSlots * kRowBytes;      // one round's staged input rows (2 per tuple)
+constexpr uint32_t kSFBytes = kMaxF * kFBytes;              // one round's staged filters
+constexpr uint32_t kOSU = kOTw + kTwBytes;                  // two staging buffers: round j in buffer j % 2
+constexpr uint32_t kOSF = kOSU + 2 * kSUBytes;
+constexpr uint32_t kOX = kOSF + 2 * kSFBytes;               // two stage-A operand buffers: round j in j % 2
+constexpr uint32_t kOZ = kOX + 2 * kXBytes;                 // one stage-A' operand buffer
+// mbarriers: tables, copies[0], A[2], A'[2], drain, Z[2], copies[1]
+constexpr uint32_t kOBar = kOZ + kZBytes;
 constexpr uint32_t kOMisc = kOBar + 8 * 10;                 // TMEM base, abort flag
 constexpr uint32_t kSmem = kOMisc + 16;
 static_assert(kSmem <= 232448, "shared memory budget");
@@ -290,7 +297,8 @@ __global__ void __launch_bounds__(kThr, 1) fftconv_tc_kernel(const T* __restrict
   uint16_t* yb = reinterpret_cast<uint16_t*>(y);
   uint64_t* const bars = reinterpret_cast<uint64_t*>(sm + kOBar);
   uint64_t* const mbar_tab = bars + 0;
-  uint64_t* const mbar_ld = bars + 1;  // one arrival per loader
+  uint64_t* const mbar_ld0 = bars + 1;  // copies into staging buffer 0 / 1: one arrival per loader
+  uint64_t* const mbar_ld1 = bars + 9;
   uint64_t* const mbar_a = bars + 2;   // [2] stage A of a round done
   uint64_t* const mbar_b = bars + 4;   // [2] stage A' of a round done
   uint64_t* const mbar_fin = bars + 6;
@@ -314,6 +322,7 @@ __global__ void __launch_bounds__(kThr, 1) fftconv_tc_kernel(const T* __restrict
     for (int i = 0; i < 7; ++i) tc::mbar_init(bars + i, i == 1 ? kFillWarps : 1);
     tc::mbar_init(mbar_z, kCompWarps);
     tc::mbar_init(mbar_z + 1, kCompWarps);
+    tc::mbar_init(mbar_ld1, kFillWarps);
     *abort_p = 0u;
     tc::fence_mbar_init();
   }
@@ -332,39 +341,41 @@ __global__ void __launch_bounds__(kThr, 1) fftconv_tc_kernel(const T* __restrict
   };
   auto aborted = [&]() { return *reinterpret_cast<volatile unsigned int*>(abort_p) != 0u; };
 
-  // ---- copies of a round's inputs: loader lq copies tuple lq's rows and filter lq with its
-  // own byte count on the copy barrier, so the copies issue from three schedulers at once
-  float dn0 = 0.f, dn1 = 0.f;  // D of the channels whose filters are in flight (operand thread 0)
-  bool ld_out = false;         // a copy phase is in flight (loaders)
-  bool ld_live = false;        // ... and its byte count includes the filter (loaders)
-  uint32_t ph_ld = 0;
-  auto issue_u = [&](const Round& R) {
-    ld_out = true;
-    ld_live = !aborted();
+  // ---- copies of a round's inputs into staging buffer sb (round j uses buffer j % 2): loader
+  // lq copies tuple lq's rows and filter lq with its own byte count on the buffer's copy
+  // barrier, so the copies issue from three schedulers at once
+  uint32_t ld_out = 0u, ld_par = 0u;  // bit sb: a copy phase into buffer sb is in flight, its parity (loaders)
+  auto issue_u = [&](const Round& R, int sb, bool& live) {
+    uint64_t* const mb = sb ? mbar_ld1 : mbar_ld0;
+    live = !aborted();
     const bool row0 = lq < R.np, row1 = row0 && 2 * R.p(lq) + 1 < B, filt = lq < R.nf;
-    const uint32_t bytes = ld_live ? (row0 ? kRowBytes : 0u) + (row1 ? kRowBytes : 0u) + (filt ? kFBytes : 0u) : 0u;
-    tc::mbar_expect_tx(mbar_ld, bytes);
-    if (ld_live && row0) {
+    const uint32_t bytes = live ? (row0 ? kRowBytes : 0u) + (row1 ? kRowBytes : 0u) + (filt ? kFBytes : 0u) : 0u;
+    tc::mbar_expect_tx(mb, bytes);
+    if (live && row0) {
       const uint16_t* src = ub + ((size_t)(2 * R.p(lq)) * H + R.h(lq)) * kL;
-      tc::bulk_g2s(s0 + kOSU + (uint32_t)(2 * lq) * kRowBytes, src, kRowBytes, mbar_ld);
-      if (row1) tc::bulk_g2s(s0 + kOSU + (uint32_t)(2 * lq + 1) * kRowBytes, src + (size_t)H * kL, kRowBytes, mbar_ld);
+      const uint32_t dst = s0 + kOSU + (uint32_t)sb * kSUBytes + (uint32_t)(2 * lq) * kRowBytes;
+      tc::bulk_g2s(dst, src, kRowBytes, mb);
+      if (row1) tc::bulk_g2s(dst + kRowBytes, src + (size_t)H * kL, kRowBytes, mb);
     }
   };
-  auto issue_f = [&](const Round& R) {  // after issue_u of the same round
-    if (ld_live && lq < R.nf)
-      tc::bulk_g2s(s0 + kOSF + (uint32_t)lq * kFBytes, f + (size_t)R.ch(lq) * kL, kFBytes, mbar_ld);
-    if (ft == 0) {  // unconditional loads (valid channels), first used by the fill one round later
-      dn0 = __ldg(D + R.ch(0));
-      dn1 = __ldg(D + R.ch(R.nf - 1));
-    }
+  auto issue_f = [&](const Round& R, int sb, bool live) {  // after issue_u of the same round
+    if (live && lq < R.nf)
+      tc::bulk_g2s(s0 + kOSF + (uint32_t)sb * kSFBytes + (uint32_t)lq * kFBytes, f + (size_t)R.ch(lq) * kL, kFBytes,
+                   sb ? mbar_ld1 : mbar_ld0);
+  };
+  auto mark_out = [&](int sb, int jr) {  // round jr's copies are in flight in buffer sb
+    ld_out |= 1u << sb;
+    ld_par = (ld_par & ~(1u << sb)) | ((uint32_t)((jr >> 1) & 1) << sb);
   };
   // ---- staged inputs -> stage-A operand (operand threads): MN-major, 64 K-rows (n1) x 3 NC
   // columns [Xr | Xi | -Xr]; column blocks of each part: the filters, then the pairs.
   // Thread ft owns the 16-byte chunks ft and ft + 96 of every staged row (8 values n2 = 8 hf ..
   // of row n1 = chunk / 2).
-  auto fill_x = [&](const Round& R, float d0, float d1) {
+  auto fill_x = [&](const Round& R, int sb, float d0, float d1) {
     const uint32_t lbo = (uint32_t)(3 * R.NC / 8) * 128;  // next 8 K-rows
-    uint8_t* const X = sm + kOX;
+    uint8_t* const X = sm + kOX + (uint32_t)sb * kXBytes;
+    const uint8_t* const su = sm + kOSU + (uint32_t)sb * kSUBytes;
+    const uint8_t* const sf = sm + kOSF + (uint32_t)sb * kSFBytes;
 #pragma unroll
     for (int pass = 0; pass < 2; ++pass) {
       const int chunk = ft + 96 * pass;
@@ -376,13 +387,13 @@ __global__ void __launch_bounds__(kThr, 1) fftconv_tc_kernel(const T* __restrict
         for (int k = 0; k < 2 * kSlots; ++k) {  // staged row k = 2 t + c
           v[k] = make_uint4(0, 0, 0, 0);
           if ((k >> 1) < R.np && 2 * R.p(k >> 1) + (k & 1) < B)
-            v[k] = *reinterpret_cast<const uint4*>(sm + kOSU + (uint32_t)k * kRowBytes + (uint32_t)chunk * 16);
+            v[k] = *reinterpret_cast<const uint4*>(su + (uint32_t)k * kRowBytes + (uint32_t)chunk * 16);
         }
         float4 fa[kMaxF], fb[kMaxF];
 #pragma unroll
         for (int q = 0; q < kMaxF; ++q) {
           if (q < R.nf) {
-            const uint8_t* src = sm + kOSF + (uint32_t)q * kFBytes + (uint32_t)chunk * 32;  // taps 8 chunk ..
+            const uint8_t* src = sf + (uint32_t)q * kFBytes + (uint32_t)chunk * 32;  // taps 8 chunk ..
             fa[q] = *reinterpret_cast<const float4*>(src);
             fb[q] = *reinterpret_cast<const float4*>(src + 16);
           }
@@ -423,11 +434,22 @@ __global__ void __launch_bounds__(kThr, 1) fftconv_tc_kernel(const T* __restrict
     tc::bulk_g2s(cb, Op<T>::cb(), kCBytes, mbar_tab);
     tc::bulk_g2s(s0 + kOTw, g_tw1k, kTwBytes, mbar_tab);
   }
-  if (loader && nloc > 0) issue_u(cur0.get());
+  bool live0 = false, live1 = false;
+  RoundCursor cur1 = cur0;
+  cur1.advance();
+  if (loader && nloc > 0) issue_u(cur0.get(), 0, live0);
+  if (loader && nloc > 1) issue_u(cur1.get(), 1, live1);
   // the filter is written by the kernel this one may be launched as a
   // programmatic dependent of: read it only after the wait
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (loader && nloc > 0) issue_f(cur0.get());
+  if (loader && nloc > 0) {
+    mark_out(0, 0);
+    issue_f(cur0.get(), 0, live0);
+  }
+  if (loader && nloc > 1) {
+    mark_out(1, 1);
+    issue_f(cur1.get(), 1, live1);
+  }
   wait_bar(mbar_tab, 0);
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_p;
@@ -497,12 +519,16 @@ __global__ void __launch_bounds__(kThr, 1) fftconv_tc_kernel(const T* __restrict
         dft16<true>(xr, xi);
         twiddle<true>(xr, xi, twp);
       }
-      // Z buffer `buf` was read by stage A' of round i - 2 (issued after that round's arrivals,
-      // so this round's arrival cannot fall into the same phase of mbar_z[buf])
-      if (i >= 2) wait_bar(mbar_b + buf, (uint32_t)((i - 2) >> 1) & 1u);
+      // the one Z buffer was read by stage A' of round i - 1, whose completion also releases the
+      // previous round's outputs for the epilogue below (stage A' of round i - 1 is issued after
+      // that round's arrivals, so this round's arrival cannot fall into the same phase of mbar_z)
+      if (i >= 1) {
+        wait_bar(mbar_b + (buf ^ 1), (uint32_t)((i - 1) >> 1) & 1u);
+        tc::fence_after_sync();
+      }
       if (valid) {
         const uint32_t lboZ = (uint32_t)(R.np * kN2 / 8) * 128;  // Z: MN-major, 256 K-rows (re k1 | im k1) x np*16
-        uint8_t* z = sm + kOZ + (uint32_t)buf * kZBytes + (uint32_t)(2 * slot) * 128 + (uint32_t)(row >> 3) * lboZ +
+        uint8_t* z = sm + kOZ + (uint32_t)(2 * slot) * 128 + (uint32_t)(row >> 3) * lboZ +
                      (uint32_t)(row & 7) * 16;
         *reinterpret_cast<uint4*>(z) = make_uint4(Op<T>::pack(xr[0], xr[1]), Op<T>::pack(xr[2], xr[3]),
                                                   Op<T>::pack(xr[4], xr[5]), Op<T>::pack(xr[6], xr[7]));
@@ -521,8 +547,6 @@ __global__ void __launch_bounds__(kThr, 1) fftconv_tc_kernel(const T* __restrict
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(mbar_z + buf);
       if (i >= 1) {
-        wait_bar(mbar_b + (buf ^ 1), (uint32_t)((i - 1) >> 1) & 1u);
-        tc::fence_after_sync();
         epilogue(Rprev, buf ^ 1);
         tc::fence_before_sync();
       }
@@ -535,31 +559,43 @@ __global__ void __launch_bounds__(kThr, 1) fftconv_tc_kernel(const T* __restrict
       epilogue(Rprev, last & 1);
     }
   } else if (filler) {
-    // ================= operand warps: round j's operand from its staged inputs, then the copies
-    // of round j + 1
+    // ================= operand warps: round j's operand (operand buffer j % 2) from its staged
+    // inputs (staging buffer j % 2), then the copies of round j + 2 into that staging buffer
     float dc0 = 0.f, dc1 = 0.f;  // D of the round being filled (operand thread 0)
-    RoundCursor cf = cur0, cl = cur0;  // rounds to fill, to load
+    RoundCursor cf = cur0, cl = cur1;  // rounds to fill, to load (two ahead)
     cl.advance();
+    if (ft == 0 && nloc > 0) {  // D of round 0; the D of round j + 1 is loaded during round j
+      const Round R0 = cur0.get();
+      dc0 = __ldg(D + R0.ch(0));
+      dc1 = __ldg(D + R0.ch(R0.nf - 1));
+    }
     for (int j = 0; j < nloc; ++j) {
-      wait_bar(mbar_ld, ph_ld);
-      ph_ld ^= 1u;
-      ld_out = false;
-      dc0 = dn0;
-      dc1 = dn1;
-      if (j >= 1) wait_bar(mbar_a + ((j - 1) & 1), (uint32_t)((j - 1) >> 1) & 1u);  // stage A of round j - 1 read X
+      const int sb = j & 1;
+      wait_bar(sb ? mbar_ld1 : mbar_ld0, (uint32_t)(j >> 1) & 1u);
+      ld_out &= ~(1u << sb);
+      if (j >= 2) wait_bar(mbar_a + sb, (uint32_t)((j - 2) >> 1) & 1u);  // stage A of round j - 2 read X[sb]
       const Round Rj = cf.get();
       cf.advance();
-      fill_x(Rj, dc0, dc1);
+      fill_x(Rj, sb, dc0, dc1);
       tc::fence_smem_to_async();
       nbar_sync(1, 32 * (kFillWarps + 1));  // operand of round j complete (the MMA warp waits here)
-      if (loader && j + 1 < nloc) {
+      if (loader && j + 2 < nloc) {  // every operand thread is past its reads of staging buffer sb
+        bool live;
+        mark_out(sb, j + 2);
         const Round Rn = cl.get();
-        cl.advance();
-        issue_u(Rn);
-        issue_f(Rn);
+        issue_u(Rn, sb, live);
+        issue_f(Rn, sb, live);
+      }
+      cl.advance();
+      if (ft == 0 && j + 1 < nloc) {
+        const Round Rn = cf.get();
+        dc0 = __ldg(D + Rn.ch(0));
+        dc1 = __ldg(D + Rn.ch(Rn.nf - 1));
       }
     }
-    if (loader && ld_out) (void)tc::mbar_wait_bounded(mbar_ld, ph_ld, kWaitNs);  // copies in flight have landed
+    // copies still in flight (only after a wait that ran out) have landed
+    if (loader && (ld_out & 1u)) (void)tc::mbar_wait_bounded(mbar_ld0, ld_par & 1u, kWaitNs);
+    if (loader && (ld_out & 2u)) (void)tc::mbar_wait_bounded(mbar_ld1, (ld_par >> 1) & 1u, kWaitNs);
   } else if (mma_warp) {
     // ================= MMA warp: stage A of round j + 1 once its operand is filled, stage A' of
     // round j once the register pass is done
@@ -571,8 +607,9 @@ __global__ void __launch_bounds__(kThr, 1) fftconv_tc_kernel(const T* __restrict
       const uint32_t lbo = (uint32_t)(3 * R.NC / 8) * 128;
       const uint32_t idA = tc::idesc_f16(128, 2 * R.NC, Op<T>::bf16, 0, 1);
       const uint32_t dA = tmem + (buf ? kTA1 : kTA0);
-      const uint64_t b0 = tc::desc_kmajor(s0 + kOX, lbo, 128);
-      const uint64_t b1 = tc::desc_kmajor(s0 + kOX + (uint32_t)(R.NC / 8) * 128, lbo, 128);
+      const uint32_t xa = s0 + kOX + (uint32_t)buf * kXBytes;
+      const uint64_t b0 = tc::desc_kmajor(xa, lbo, 128);
+      const uint64_t b1 = tc::desc_kmajor(xa + (uint32_t)(R.NC / 8) * 128, lbo, 128);
       const uint64_t step = (uint64_t)((2 * lbo) >> 4);  // next 16 K-rows (address field in 16-byte units)
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
@@ -589,7 +626,7 @@ __global__ void __launch_bounds__(kThr, 1) fftconv_tc_kernel(const T* __restrict
       }
       const uint32_t lboZ = (uint32_t)(R.np * kN2 / 8) * 128;
       const uint32_t idB = tc::idesc_f16(128, R.np * kN2, Op<T>::bf16, 1, 1);
-      const uint32_t zr = s0 + kOZ + (uint32_t)buf * kZBytes;
+      const uint32_t zr = s0 + kOZ;
       const uint64_t a0 = tc::desc_kmajor(ca, kCSbo, kCLbo), a1 = tc::desc_kmajor(cb, kCSbo, kCLbo);
       const uint64_t z0 = tc::desc_kmajor(zr, lboZ, 128), z1 = tc::desc_kmajor(zr + 16 * lboZ, lboZ, 128);
       const uint64_t astep = (uint64_t)((2 * kCSbo) >> 4), zstep = (uint64_t)((2 * lboZ) >> 4);
