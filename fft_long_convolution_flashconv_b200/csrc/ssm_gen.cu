@@ -97,16 +97,22 @@ constexpr uint64_t kGWaitNs = 2000000000ull;
 // never stored, so those reads may land on the next tile: the tiles then take
 // 18 KB each instead of 36 KB and four CTAs fit on an SM.  The control words
 // sit past every byte an MMA reads.
-template <bool SHORT>
+// COMPACT (SHORT with single tables): no remainder tables, and Q and the exact
+// powers sit in the never-stored stretch of the AH tile, which leaves 36 KB per
+// CTA (six CTAs of 128 threads per SM).
+template <bool SHORT, bool COMPACT = false>
 struct GenLayout {
   static constexpr uint32_t tab = SHORT ? kGTab / 2 : kGTab;
-  static constexpr uint32_t ahh = 0, ahl = tab, qh = 2 * tab, ql = qh + kGQ;
-  static constexpr uint32_t mma_end = (ahl + kGTab > ql + kGQ) ? ahl + kGTab : ql + kGQ;
+  static constexpr uint32_t ahh = 0, ahl = COMPACT ? 0 : tab, qh = COMPACT ? tab : 2 * tab,
+                            ql = COMPACT ? qh : qh + kGQ;
+  static constexpr uint32_t mma_end = COMPACT ? kGTab : ((ahl + kGTab > ql + kGQ) ? ahl + kGTab : ql + kGQ);
   // exact powers A, A^4, A^16, A^128, A^512 per mode; in SHORT they sit in the
   // stretch that only feeds never-stored rows
-  static constexpr uint32_t pw = SHORT ? ql + kGQ : mma_end;
-  static constexpr uint32_t red = pw + 64 * 5 * 8, mbar = red + 32, tmem = mbar + 8;
+  static constexpr uint32_t pw = SHORT ? (COMPACT ? qh + kGQ : ql + kGQ) : mma_end;
+  // the control words sit past every byte an MMA reads
+  static constexpr uint32_t red = COMPACT ? mma_end : pw + 64 * 5 * 8, mbar = red + 32, tmem = mbar + 8;
   static constexpr uint32_t bytes = (tmem + 8 > mma_end) ? tmem + 8 : mma_end;
+  static_assert(!COMPACT || pw + 64 * 5 * 8 <= kGTab, "COMPACT: Q and the powers inside the AH tile's extent");
 };
 __device__ __forceinline__ uint32_t gsplit(float a, float b, uint32_t& lo) {
   const __half2 h = __floats2half2_rn(a, b);
@@ -120,8 +126,10 @@ __device__ __forceinline__ uint32_t goff(int r, int n) {  // K elements (2n, 2n+
 }
 }  // namespace
 
-template <bool SHORT, bool HI>
-__global__ void __launch_bounds__(kGThr, SHORT ? 4 : 2) ssm_gen_tc_kernel(const float* __restrict__ dt,
+// THR = 128 (SHORT with single tables): each thread covers two row-group
+// phases, so that all of a 768-channel launch fits one wave of CTAs.
+template <bool SHORT, bool HI, int THR = kGThr>
+__global__ void __launch_bounds__(THR, THR == 128 ? 6 : (SHORT ? 4 : 2)) ssm_gen_tc_kernel(const float* __restrict__ dt,
                                                                           const float2* __restrict__ lam,
                                                                           const float2* __restrict__ Bp,
                                                                           const float2* __restrict__ Cp, int H, int N,
@@ -129,8 +137,10 @@ __global__ void __launch_bounds__(kGThr, SHORT ? 4 : 2) ssm_gen_tc_kernel(const 
   // a convolution launched as this kernel's programmatic dependent may start
   // its prologue now; it reads f only after this grid has completed
   asm volatile("griddepcontrol.launch_dependents;");
-  using LY = GenLayout<SHORT>;
-  constexpr int NG = SHORT ? 2 : 4;  // row groups g = gq + 4 r this thread may fill
+  static_assert(THR == kGThr || (THR == 128 && SHORT && HI), "128 threads only for short single-table rows");
+  using LY = GenLayout<SHORT, THR == 128>;
+  constexpr int NG = SHORT ? 2 : 4;  // row groups g = gq + 4 r a phase gq may fill
+  constexpr int NV = kGThr / THR;     // row-group phases per thread: gq = tid / 64 + 2 v
   extern __shared__ __align__(1024) uint8_t gtsm[];
   struct {
     uint8_t* ahh;
@@ -148,7 +158,7 @@ __global__ void __launch_bounds__(kGThr, SHORT ? 4 : 2) ssm_gen_tc_kernel(const 
   const int units = (L + kGUnitTaps - 1) / kGUnitTaps;
   const int u0 = blockIdx.x * kGUnits, u1 = min(units, u0 + kGUnits);
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int n = tid & 63, gq = tid >> 6;  // this thread's mode and row-group phase (0..3)
+  const int n = tid & 63, gq0 = tid >> 6;  // this thread's mode and first row-group phase
   const float d = dt[h];
   if (warp == 0) tc::tmem_alloc(sm.tmem_p, 32);
   if (tid == 0) {
@@ -156,7 +166,7 @@ __global__ void __launch_bounds__(kGThr, SHORT ? 4 : 2) ssm_gen_tc_kernel(const 
     tc::fence_mbar_init();
   }
   // exact powers, five per mode, spread over the CTA
-  for (int idx = tid; idx < 64 * 5; idx += kGThr) {
+  for (int idx = tid; idx < 64 * 5; idx += THR) {
     const int m = idx / 5, e = idx - 5 * m;
     float2 v = make_float2(0.f, 0.f);
     if (m < N) {
@@ -178,7 +188,7 @@ __global__ void __launch_bounds__(kGThr, SHORT ? 4 : 2) ssm_gen_tc_kernel(const 
   __syncthreads();
   mx = 0.f;
 #pragma unroll
-  for (int i = 0; i < kGThr / 32; ++i) mx = fmaxf(mx, sm.red[i]);
+  for (int i = 0; i < THR / 32; ++i) mx = fmaxf(mx, sm.red[i]);
   float scale = 1.f, inv = 1.f;
   if (mx > 0.f && mx <= 3.0e38f) {
     int ex = 0;
@@ -191,22 +201,24 @@ __global__ void __launch_bounds__(kGThr, SHORT ? 4 : 2) ssm_gen_tc_kernel(const 
   const float2 a1 = sm.pw[n * 5 + 0], a4 = sm.pw[n * 5 + 1], a16 = sm.pw[n * 5 + 2];
   const float2 a128 = sm.pw[n * 5 + 3], a512 = sm.pw[n * 5 + 4];
   const float2 one = n < N ? make_float2(1.f, 0.f) : make_float2(0.f, 0.f);
-  float2 m8[8], G[NG];
+  float2 m8[8], G[NV][NG];
   m8[0] = one;
 #pragma unroll
   for (int m = 1; m < 8; ++m) m8[m] = cmul(m8[m - 1], a16);
-  float2 g128 = one, p4 = one;
 #pragma unroll
-  for (int i = 0; i < 3; ++i)
-    if (i < gq) {
-      g128 = cmul(g128, a128);
-      p4 = cmul(p4, a4);
-    }
-  G[0] = g128;
+  for (int vv = 0; vv < NV; ++vv) {
+    const int gq = gq0 + 2 * vv;
+    float2 g128 = one, p4 = one;
 #pragma unroll
-  for (int r = 1; r < NG; ++r) G[r] = cmul(G[r - 1], a512);
-  // Q rows tl = 4 gq .. 4 gq + 3
-  {
+    for (int i = 0; i < 3; ++i)
+      if (i < gq) {
+        g128 = cmul(g128, a128);
+        p4 = cmul(p4, a4);
+      }
+    G[vv][0] = g128;
+#pragma unroll
+    for (int r = 1; r < NG; ++r) G[vv][r] = cmul(G[vv][r - 1], a512);
+    // Q rows tl = 4 gq .. 4 gq + 3
     float2 p = cmul(make_float2(w.x * scale, w.y * scale), p4);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -228,10 +240,11 @@ __global__ void __launch_bounds__(kGThr, SHORT ? 4 : 2) ssm_gen_tc_kernel(const 
     const float2 base = n >= N ? make_float2(0.f, 0.f)
                         : th0 == 0 ? make_float2(1.f, 0.f) : ssm_pow(d, lm.x, lm.y, 16.0 * th0);
 #pragma unroll
-    for (int r = 0; r < NG; ++r) {
-      const int g = gq + 4 * r;
+    for (int vr = 0; vr < NV * NG; ++vr) {
+      const int vv = vr / NG, r = vr - vv * NG;
+      const int g = gq0 + 2 * vv + 4 * r;
       if (8 * g >= rows) continue;  // rows past the end are never stored
-      const float2 pg = cmul(base, G[r]);
+      const float2 pg = cmul(base, G[vv][r]);
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
         const float2 v = cmul(pg, m8[m]);
@@ -509,6 +522,16 @@ static cudaError_t gen_tc(const float* dt, const float* lam, const float* Bp, co
   }
   const int units = (L + kGUnitTaps - 1) / kGUnitTaps;
   const bool short_rows = L <= kGUnitTaps / 2;
+  if constexpr (HI) {
+    if (short_rows) {  // 128-thread CTAs in the compact layout
+      constexpr size_t csm = GenLayout<true, true>::bytes;
+      cudaError_t e = smem_optin<ssm_gen_tc_kernel<true, true, 128>>(csm);
+      if (e != cudaSuccess) return e;
+      ssm_gen_tc_kernel<true, true, 128><<<dim3((units + kGUnits - 1) / kGUnits, H), 128, csm, st>>>(dt, l2, b2, c2, H,
+                                                                                                   N, L, f);
+      return cudaGetLastError();
+    }
+  }
   auto kern = short_rows ? ssm_gen_tc_kernel<true, HI> : ssm_gen_tc_kernel<false, HI>;
   const size_t smem = short_rows ? GenLayout<true>::bytes : GenLayout<false>::bytes;
   cudaError_t e = short_rows ? smem_optin<ssm_gen_tc_kernel<true, HI>>(smem)
