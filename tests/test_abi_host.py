@@ -187,3 +187,20 @@ def test_long_conv_rejects_bad_arguments():
     assert lib.fftconv_long_fwd(P, P2, P3, P + 64, 2, 3, 12000, P3, ws, 0, None) == _lib.FC_EINVAL
     # L <= 8192 goes through fftconv_fwd's validation
     assert lib.fftconv_long_fwd(P, P2, P3, y, 2, 3, 4096, None, 0, 7, None) == _lib.FC_EINVAL
+    # more row pairs than the pass grids index
+    far = P + (1 << 50)  # an output that cannot overlap the (fake) input of this size
+    assert lib.fftconv_long_fwd(P, P2, P3, far, 2, (1 << 29) + 1, 9000, P3, 1 << 62, 0, None) == _lib.FC_EUNSUPPORTED
+    assert "2^29" in _err()
+
+
+@pytest.mark.parametrize("B,H,L,M", [(2, 3, 12000, 32768), (3, 2, 8193, 32768), (5, 7, 20000, 65536),
+                                     (1, 1, 32768, 65536), (1, 1, 32769, 131072), (4, 2, 65536, 131072)])
+def test_long_conv_workspace_holds_pair_and_filter_spectra(B, H, L, M):
+    """The workspace of the four-step long convolution: the complex fp32
+    spectra of the H * ceil(B / 2) row pairs and of the H filters at the
+    transform length M = 2^ceil(log2(2L - 1)), each part rounded up to 256
+    bytes."""
+    lib = _lib.load()
+    r256 = lambda b: (b + 255) // 256 * 256
+    pairs = H * ((B + 1) // 2)
+    assert lib.fftconv_long_workspace(B, H, L) == r256(pairs * M * 8) + r256(H * M * 8)
