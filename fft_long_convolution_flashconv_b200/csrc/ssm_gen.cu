@@ -322,20 +322,27 @@ namespace {
 constexpr int kG64Units = 2;                    // 8192-tap units per CTA
 constexpr int kG64Cols = 64, kG64UnitTaps = kGRows * kG64Cols;
 constexpr uint32_t kG64Q = (kG64Cols / 8) * kGSbo;
+// COMPACT (single tables): no remainder tables, 58 KB, three CTAs of 128 threads per SM.
+template <bool COMPACT = false>
 struct Gen64Layout {
-  static constexpr uint32_t ahh = 0, ahl = kGTab, qh = 2 * kGTab, ql = qh + kG64Q, pw = ql + kG64Q;
+  static constexpr uint32_t ahh = 0, ahl = COMPACT ? 0 : kGTab, qh = COMPACT ? kGTab : 2 * kGTab,
+                            ql = COMPACT ? qh : qh + kG64Q, pw = ql + kG64Q;
   static constexpr uint32_t red = pw + 64 * 5 * 8, mbar = red + 32, tmem = mbar + 8, bytes = tmem + 8;
 };
 }  // namespace
 
-template <bool HI>
-__global__ void __launch_bounds__(kGThr, 2) ssm_gen_tc64_kernel(const float* __restrict__ dt,
+// THR = 128 (single tables): each thread covers two row-group phases, so three
+// CTAs fit an SM.
+template <bool HI, int THR = kGThr>
+__global__ void __launch_bounds__(THR, THR == 128 ? 3 : 2) ssm_gen_tc64_kernel(const float* __restrict__ dt,
                                                                 const float2* __restrict__ lam,
                                                                 const float2* __restrict__ Bp,
                                                                 const float2* __restrict__ Cp, int H, int N, int L,
                                                                 float* __restrict__ f) {
   asm volatile("griddepcontrol.launch_dependents;");  // see ssm_gen_tc_kernel
-  using LY = Gen64Layout;
+  static_assert(THR == kGThr || (THR == 128 && HI), "128 threads only with single tables");
+  using LY = Gen64Layout<THR == 128>;
+  constexpr int NV = kGThr / THR;  // row-group phases per thread: gq = tid / 64 + 2 v
   extern __shared__ __align__(1024) uint8_t gtsm[];
   uint8_t* ahh = gtsm + LY::ahh;
   uint8_t* ahl = gtsm + LY::ahl;
@@ -349,14 +356,14 @@ __global__ void __launch_bounds__(kGThr, 2) ssm_gen_tc64_kernel(const float* __r
   const int units = (L + kG64UnitTaps - 1) / kG64UnitTaps;
   const int u0 = blockIdx.x * kG64Units, u1 = min(units, u0 + kG64Units);
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int n = tid & 63, gq = tid >> 6;  // this thread's mode and row-group phase (0..3)
+  const int n = tid & 63, gq0 = tid >> 6;  // this thread's mode and first row-group phase
   const float d = dt[h];
   if (warp == 0) tc::tmem_alloc(tmem_p, 64);
   if (tid == 0) {
     tc::mbar_init(mbar, 1);
     tc::fence_mbar_init();
   }
-  for (int idx = tid; idx < 64 * 5; idx += kGThr) {
+  for (int idx = tid; idx < 64 * 5; idx += THR) {
     const int m = idx / 5, e = idx - 5 * m;
     float2 v = make_float2(0.f, 0.f);
     if (m < N) {
@@ -378,7 +385,7 @@ __global__ void __launch_bounds__(kGThr, 2) ssm_gen_tc64_kernel(const float* __r
   __syncthreads();
   mx = 0.f;
 #pragma unroll
-  for (int i = 0; i < kGThr / 32; ++i) mx = fmaxf(mx, red[i]);
+  for (int i = 0; i < THR / 32; ++i) mx = fmaxf(mx, red[i]);
   float scale = 1.f, inv = 1.f;
   if (mx > 0.f && mx <= 3.0e38f) {
     int ex = 0;
@@ -389,22 +396,24 @@ __global__ void __launch_bounds__(kGThr, 2) ssm_gen_tc64_kernel(const float* __r
   const float2 a1 = pw[n * 5 + 0], a16 = pw[n * 5 + 1], a64 = pw[n * 5 + 2];
   const float2 a512 = pw[n * 5 + 3], a2048 = pw[n * 5 + 4];
   const float2 one = n < N ? make_float2(1.f, 0.f) : make_float2(0.f, 0.f);
-  float2 m8[8], G[4];
+  float2 m8[8], G[NV][4];
   m8[0] = one;
 #pragma unroll
   for (int m = 1; m < 8; ++m) m8[m] = cmul(m8[m - 1], a64);
-  float2 g512 = one, p16 = one;
 #pragma unroll
-  for (int i = 0; i < 3; ++i)
-    if (i < gq) {
-      g512 = cmul(g512, a512);
-      p16 = cmul(p16, a16);
-    }
-  G[0] = g512;
+  for (int vv = 0; vv < NV; ++vv) {
+    const int gq = gq0 + 2 * vv;
+    float2 g512 = one, p16 = one;
 #pragma unroll
-  for (int r = 1; r < 4; ++r) G[r] = cmul(G[r - 1], a2048);
-  // Q rows tl = 16 gq .. 16 gq + 15
-  {
+    for (int i = 0; i < 3; ++i)
+      if (i < gq) {
+        g512 = cmul(g512, a512);
+        p16 = cmul(p16, a16);
+      }
+    G[vv][0] = g512;
+#pragma unroll
+    for (int r = 1; r < 4; ++r) G[vv][r] = cmul(G[vv][r - 1], a2048);
+    // Q rows tl = 16 gq .. 16 gq + 15
     float2 p = cmul(make_float2(w.x * scale, w.y * scale), p16);
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
@@ -417,7 +426,7 @@ __global__ void __launch_bounds__(kGThr, 2) ssm_gen_tc64_kernel(const float* __r
   }
   const uint32_t idesc = tc::idesc_f16(kGRows, kG64Cols, 0);
   const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-  const int half = warp >> 2;  // output columns 32 half .. 32 half + 31
+  const int half0 = warp >> 2;  // output columns 32 half .. 32 half + 31 (both halves with 128 threads)
   const bool vec_ok = (L & 3) == 0;
   uint32_t phase = 0;
   bool failed = false;
@@ -431,9 +440,10 @@ __global__ void __launch_bounds__(kGThr, 2) ssm_gen_tc64_kernel(const float* __r
       __syncthreads();
     }
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int g = gq + 4 * r;
-      const float2 pg = cmul(base, G[r]);
+    for (int vr = 0; vr < NV * 4; ++vr) {
+      const int vv = vr / 4, r = vr - 4 * vv;
+      const int g = gq0 + 2 * vv + 4 * r;
+      const float2 pg = cmul(base, G[vv][r]);
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
         // rows past the end feed only never-stored outputs: zero them
@@ -475,6 +485,8 @@ __global__ void __launch_bounds__(kGThr, 2) ssm_gen_tc64_kernel(const float* __r
       break;
     }
     tc::fence_after_sync();
+#pragma unroll 1
+    for (int half = half0; half < 2; half += 2 / NV) {
     float v[32];
     tc::tmem_ld16x2_wait(tmem + lane_off + (uint32_t)(32 * half), tmem + lane_off + (uint32_t)(32 * half + 16), v,
                          v + 16);
@@ -492,6 +504,7 @@ __global__ void __launch_bounds__(kGThr, 2) ssm_gen_tc64_kernel(const float* __r
         for (int j = 0; j < 32; ++j)
           if (t0 + j < L) fp[j] = v[j] * inv;
       }
+    }
     }
   }
   if (failed && tid == 0) atomicAdd(&g_gen_tc_timeouts, 1u);
@@ -514,10 +527,17 @@ static cudaError_t gen_tc(const float* dt, const float* lam, const float* Bp, co
   const float2* c2 = reinterpret_cast<const float2*>(Cp);
   if (L > 2 * kGUnitTaps) {
     const int units = (L + kG64UnitTaps - 1) / kG64UnitTaps;
-    cudaError_t e = smem_optin<ssm_gen_tc64_kernel<HI>>(Gen64Layout::bytes);
-    if (e != cudaSuccess) return e;
     dim3 grid((units + kG64Units - 1) / kG64Units, H);
-    ssm_gen_tc64_kernel<HI><<<grid, kGThr, Gen64Layout::bytes, st>>>(dt, l2, b2, c2, H, N, L, f);
+    if constexpr (HI) {  // 128-thread CTAs in the compact layout
+      constexpr size_t csm = Gen64Layout<true>::bytes;
+      cudaError_t e = smem_optin<ssm_gen_tc64_kernel<true, 128>>(csm);
+      if (e != cudaSuccess) return e;
+      ssm_gen_tc64_kernel<true, 128><<<grid, 128, csm, st>>>(dt, l2, b2, c2, H, N, L, f);
+      return cudaGetLastError();
+    }
+    cudaError_t e = smem_optin<ssm_gen_tc64_kernel<HI>>(Gen64Layout<>::bytes);
+    if (e != cudaSuccess) return e;
+    ssm_gen_tc64_kernel<HI><<<grid, kGThr, Gen64Layout<>::bytes, st>>>(dt, l2, b2, c2, H, N, L, f);
     return cudaGetLastError();
   }
   const int units = (L + kGUnitTaps - 1) / kGUnitTaps;
