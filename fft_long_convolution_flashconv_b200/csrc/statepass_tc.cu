@@ -77,6 +77,11 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t&
 __device__ __forceinline__ uint32_t toff(int r, int k8) {
   return (uint32_t)(r >> 3) * kSbo + (uint32_t)k8 * kLbo + (uint32_t)(r & 7) * 16u;
 }
+// the u chunks arrive by asynchronous copies and go unpadded (K-major, 128-byte core-matrix stride)
+constexpr uint32_t kLboU = 128, kSboU = (kKS / 8) * 128;
+__device__ __forceinline__ uint32_t toff_u(int r, int k8) {
+  return (uint32_t)(r >> 3) * kSboU + (uint32_t)k8 * kLboU + (uint32_t)(r & 7) * 16u;
+}
 
 __device__ __forceinline__ void cp_async16(uint32_t saddr, const void* g) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(g) : "memory");
@@ -101,11 +106,11 @@ constexpr uint32_t tmem_cols() {
 // The accumulator is double-buffered in TMEM so that chunk c+1's MMA runs during
 // chunk c's recurrence, and the u chunks are double-buffered in shared memory.
 constexpr int kThrS = 256;
-template <int NC>
+template <int NC, bool LO>
 struct StateSmem2 {
-  uint8_t ph[kTab];                // A: P hi, 128 rows (2n + re/im) x 128 K (il)
-  uint8_t pl[kTab];                // A: P lo
-  uint8_t ub[2][(NC / 8) * kSbo];  // B: u chunk, NC rows (ih) x 128 K (il), double-buffered
+  uint8_t ph[kTab];                 // A: P hi, 128 rows (2n + re/im) x 128 K (il)
+  uint8_t pl[LO ? kTab : 16];       // A: P lo (bf16 only)
+  uint8_t ub[2][(NC / 8) * kSboU];  // B: u chunk, NC rows (ih) x 128 K (il), double-buffered
   float2 part[128];                // the upper half's partial sums
   uint64_t mbar[2];
   uint32_t tmem_base;
@@ -115,16 +120,16 @@ template <int NC>
 __device__ __forceinline__ void stage_u2(uint8_t* dst, const uint16_t* src, int tid) {
   const uint32_t d0 = tc::smem_u32(dst);
   for (int q = tid; q < NC * 16; q += kThrS)  // 16-byte vector: row ih = q / 16, K group q % 16
-    cp_async16(d0 + toff(q >> 4, q & 15), src + (size_t)q * 8);
+    cp_async16(d0 + toff_u(q >> 4, q & 15), src + (size_t)q * 8);
 }
 
 template <typename T, int NC>
-__global__ void __launch_bounds__(kThrS, 2) sp_state_tc_kernel(const T* __restrict__ u, const float* __restrict__ dt,
+__global__ void __launch_bounds__(kThrS, Op16<T>::bf16 ? 2 : 3) sp_state_tc_kernel(const T* __restrict__ u, const float* __restrict__ dt,
                                                                 const float2* __restrict__ lam,
                                                                 const float2* __restrict__ Bp, int H, int L, int N,
                                                                 float2* __restrict__ s_ws) {
   extern __shared__ __align__(1024) uint8_t smraw[];
-  StateSmem2<NC>& sm = *reinterpret_cast<StateSmem2<NC>*>(smraw);
+  StateSmem2<NC, Op16<T>::bf16 != 0>& sm = *reinterpret_cast<StateSmem2<NC, Op16<T>::bf16 != 0>*>(smraw);
   constexpr int Tc = NC * kKS;
   constexpr int HC = NC / 2;  // columns per half
   const int h = blockIdx.x, b = blockIdx.y;
@@ -172,9 +177,11 @@ __global__ void __launch_bounds__(kThrS, 2) sp_state_tc_kernel(const T* __restri
       split2<T>(im[2 * m], im[2 * m + 1], ih_[m], il_[m]);
     }
     *reinterpret_cast<uint4*>(sm.ph + toff(2 * n, g)) = make_uint4(rh[0], rh[1], rh[2], rh[3]);
-    *reinterpret_cast<uint4*>(sm.pl + toff(2 * n, g)) = make_uint4(rl[0], rl[1], rl[2], rl[3]);
     *reinterpret_cast<uint4*>(sm.ph + toff(2 * n + 1, g)) = make_uint4(ih_[0], ih_[1], ih_[2], ih_[3]);
-    *reinterpret_cast<uint4*>(sm.pl + toff(2 * n + 1, g)) = make_uint4(il_[0], il_[1], il_[2], il_[3]);
+    if constexpr (Op16<T>::bf16 != 0) {
+      *reinterpret_cast<uint4*>(sm.pl + toff(2 * n, g)) = make_uint4(rl[0], rl[1], rl[2], rl[3]);
+      *reinterpret_cast<uint4*>(sm.pl + toff(2 * n + 1, g)) = make_uint4(il_[0], il_[1], il_[2], il_[3]);
+    }
   }
 
   // this lane's mode: row r = lane -> mode lane / 2, real (even) or imaginary (odd) part
@@ -197,13 +204,13 @@ __global__ void __launch_bounds__(kThrS, 2) sp_state_tc_kernel(const T* __restri
     const uint32_t tm = sm.tmem_base + (uint32_t)((c & 1) * tmem_cols<NC>());
 #pragma unroll
     for (int kk = 0; kk < kKS / 16; ++kk)
-      tc::mma_f16(tm, tc::desc_kmajor(pa + kk * 2 * kLbo, kLbo, kSbo), tc::desc_kmajor(ua + kk * 2 * kLbo, kLbo, kSbo),
-                  idesc, kk > 0 ? 1u : 0u);
+      tc::mma_f16(tm, tc::desc_kmajor(pa + kk * 2 * kLbo, kLbo, kSbo),
+                  tc::desc_kmajor(ua + kk * 2 * kLboU, kLboU, kSboU), idesc, kk > 0 ? 1u : 0u);
     if constexpr (Op16<T>::bf16) {  // fp16 P alone carries 11 bits; bf16 P needs its remainder
 #pragma unroll
       for (int kk = 0; kk < kKS / 16; ++kk)
-        tc::mma_f16(tm, tc::desc_kmajor(pb + kk * 2 * kLbo, kLbo, kSbo), tc::desc_kmajor(ua + kk * 2 * kLbo, kLbo, kSbo),
-                    idesc, 1u);
+        tc::mma_f16(tm, tc::desc_kmajor(pb + kk * 2 * kLbo, kLbo, kSbo),
+                    tc::desc_kmajor(ua + kk * 2 * kLboU, kLboU, kSboU), idesc, 1u);
     }
     tc::mma_commit(&sm.mbar[c & 1]);
   };
@@ -494,7 +501,7 @@ static cudaError_t sp_tc_t(const void* u, void* y, const float* dt, const float*
                            bool corr, cudaStream_t st) {
   dim3 grid(H, B);
   if (!corr) {
-    const size_t smem = sizeof(StateSmem2<NC>) + 1024;
+    const size_t smem = sizeof(StateSmem2<NC, Op16<T>::bf16 != 0>) + 1024;
     auto kern = sp_state_tc_kernel<T, NC>;
     cudaError_t e = smem_optin<sp_state_tc_kernel<T, NC>>(smem);
     if (e != cudaSuccess) return e;
