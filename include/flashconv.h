@@ -207,9 +207,11 @@ FC_API fc_status ssm_conv_fwd(const void* u, const float* dt, const float* lambd
  * where they are fftconv_fwd's tensor-core kernel (the chunk filter then
  * comes from single fp16 tables, about 11 significant bits, for N <= 64).
  * With 16-bit I/O, those chunks and N <= 64, the end states and the
- * initial-state term are tensor-core GEMMs against tables split hi/lo into
- * 16-bit parts (about 22 significant bits; 16 for the bfloat16 u-side
- * table), with u as an exact 16-bit operand. */
+ * initial-state term are tensor-core GEMMs with u as an exact 16-bit operand:
+ * the end states against a power table split hi/lo into 16-bit parts for
+ * bfloat16 u (about 16 significant bits) and a single fp16 table for fp16 u
+ * (11 bits); the initial-state term against single fp16 tables (11 bits,
+ * below the rounding of y itself). */
 FC_API size_t fftconv_statepass_workspace(int B, int H, int L, int N, int chunk);
 FC_API fc_status fftconv_statepass(const void* u, const float* dt, const float* lambda, const float* Bp,
                                    const float* Cp, const float* D, void* y, int B, int H, int L, int N,
