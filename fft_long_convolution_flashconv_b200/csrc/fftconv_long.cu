@@ -71,10 +71,11 @@ struct Grp {  // one length-N sequence per group of TG threads
   static constexpr int SH = ILog2<R0>::v;
   static constexpr int BUF = N + (N >> SH);
   static constexpr int PER0 = RM / R0, PER_L = RM / RL;
-  // row stride (in float2) of a [position][G] staging tile: with G + 32 / TG
-  // the 32 lanes of a warp (32 / TG sequences x TG positions) spread evenly
-  // over the shared-memory banks
-  static constexpr int TS = G + 32 / TG;
+  // row stride (in float2) of a [position][G] staging tile: with G + 2 the 32
+  // lanes of a warp (32 / TG sequences x TG positions, TG = 8 or 16) hit every
+  // 8-byte bank pair exactly twice, and rows stay 16-byte aligned
+  static constexpr int TS = G + 2;
+  static_assert(TG == 8 || TG == 16, "stride chosen for 8 or 16 threads per sequence");
   // a staging tile of `rows` positions and the group FFT buffers share one
   // region: the tile is read into registers before the first buffer store
   // (after a CTA barrier inside the transform) and written only after a
@@ -224,7 +225,7 @@ __global__ void __launch_bounds__(kThr) lc_spectrum(const float2* __restrict__ Y
 // first, from the filter's pass-1 output Yf[h] (F^ = forward DFT / M); past
 // that it reads F^ from Fs[h][k2][k1], written by lc_spectrum.
 template <int LOGM1>
-__global__ void __launch_bounds__(kThr) lc_pass2(float2* __restrict__ Y, const float2* __restrict__ Fsrc, int B,
+__global__ void __launch_bounds__(kThr, LOGM1 == 9 ? 1 : 3) lc_pass2(float2* __restrict__ Y, const float2* __restrict__ Fsrc, int B,
                                                  int h0, int conj_filter) {
   using G1 = Grp<LOGM1>;
   constexpr int M1 = 1 << LOGM1, M = M1 * kM2, GK = G1::G;
